@@ -1,0 +1,421 @@
+#!/usr/bin/env python
+"""Benchmark: exact tiled GQA attention on B200, Qwen3-8B shapes.
+
+One step = the whole hot path once: attn_prefill on the Qwen3-8B-shaped causal
+prefill (B=4, Hq=32, Hkv=8, Lq=Lk=8192, D=128) followed by attn_decode on the
+Qwen3-8B-shaped decode batch (B=64, Hq=32, Hkv=8, D=128, cache lengths drawn
+uniform in [1024, 32768]).  Inputs are seeded synthetic N(0,1) bf16 tensors,
+resident in HBM before the timed region, each larger than the 126 MB L2.
+
+The JSON line's `value` is prefill TFLOP/s (algorithmic FLOPs: visible
+query/key pairs only), `decode` holds decode HBM GB/s; both are timed with
+CUDA events on the launching stream, per call.  `e2e` repeats the step
+through the public Python API with host buffers: pinned-host -> device copies
+of the step's inputs (prefill q/k/v, decode q) and device -> host copies of
+the outputs (out, lse) inside the timed region; the decode KV cache is
+resident device state, as in serving.
+
+Multi-GPU (torchrun): every rank runs the same per-rank workload on its own
+GPU (independent sequences -- the path has no exchange step), timing is the
+max over ranks, and `value` sums the work of all ranks ("scaling": "weak").
+
+`--impl reference` times the fp64 CPU oracle on a bounded sample of the same
+workloads on this host's cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from exact_tiled_attention_gqa_b200 import roofline as RL          # noqa: E402
+from exact_tiled_attention_gqa_b200 import workloads as W          # noqa: E402
+
+METRIC = "prefill TFLOP/s & decode HBM GB/s (frac. of roofline), Qwen3-8B GQA shapes"
+PREFILL = W.QWEN_PREFILL_8K_B4
+DECODE = W.QWEN_DECODE
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU seconds per oracle sample")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------------------
+# clocks sampled during the timed region
+# --------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: str):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        loaded = [s for s, p in zip(sm, power) if p > 300.0] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm),
+                "power_w_max": max(power) if power else None}
+
+
+def physical_gpu_id(local_rank: int) -> str:
+    """nvidia-smi's id for this process's GPU (CUDA_VISIBLE_DEVICES may remap ordinals)."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").strip()
+    if vis:
+        ids = [x.strip() for x in vis.split(",") if x.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return str(local_rank)
+
+
+# --------------------------------------------------------------------------
+# our arm
+# --------------------------------------------------------------------------
+def run_ours(args, rank, world, local_rank):
+    import exact_tiled_attention_gqa_b200 as attn
+    from exact_tiled_attention_gqa_b200 import build
+
+    build.build()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist_mod
+        dist = dist_mod
+    peaks = RL.measured_peaks()
+
+    # ---- inputs (per rank: its own sequences; seeds differ by rank) ----
+    seed = args.seed + 1000 * rank
+    q_h, k_h, v_h = W.prefill_inputs_for(PREFILL, seed=seed, device="cpu")
+    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    dq, dk, dv, dsl = W.decode_inputs_for(DECODE, seed=seed, device=dev)
+    seqlens_host = dsl.cpu()
+    p_flops = RL.prefill_flops(PREFILL.B, PREFILL.Hq, PREFILL.Lq, PREFILL.Lk, PREFILL.D, PREFILL.is_causal)
+    d_bytes = RL.decode_bytes(seqlens_host.tolist(), DECODE.B, DECODE.Hq, DECODE.Hkv, DECODE.D)
+    p_out = torch.empty_like(q)
+    p_lse = torch.empty((PREFILL.B, PREFILL.Hq, PREFILL.Lq), dtype=torch.float32, device=dev)
+    d_out = torch.empty_like(dq)
+    d_lse = torch.empty((DECODE.B, DECODE.Hq), dtype=torch.float32, device=dev)
+    ws = torch.empty(attn.decode_workspace_size(DECODE.B, DECODE.Hq, DECODE.Hkv, DECODE.Lmax, DECODE.D),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        attn.prefill(q, k, v, is_causal=True, out=p_out, lse=p_lse, stream=stream)
+        attn.decode(dq, dk, dv, dsl, out=d_out, lse=d_lse, workspace=ws, stream=stream)
+
+    def barrier():
+        if dist is not None:
+            dist.barrier()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert attn.device_error(reset=True) == 0, "device error word set during warm-up"
+
+    # ---- timed region: K steps, events around each call on the launching stream ----
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    sampler = ClockSampler(physical_gpu_id(local_rank))
+    barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        attn.prefill(q, k, v, is_causal=True, out=p_out, lse=p_lse, stream=stream)
+        ev[i][1].record(stream)
+        attn.decode(dq, dk, dv, dsl, out=d_out, lse=d_lse, workspace=ws, stream=stream)
+        ev[i][2].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clocks = sampler.stop()
+    total_ms = t_start.elapsed_time(t_end)
+    pre_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    dec_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    derr = attn.device_error(reset=True)
+    assert derr == 0, f"device error word {derr:#x} after the timed region"
+
+    def max_over_ranks(x):
+        if dist is None:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    total_ms = max_over_ranks(total_ms)
+    pre_avg = max_over_ranks(sum(pre_ms) / len(pre_ms))
+    dec_avg = max_over_ranks(sum(dec_ms) / len(dec_ms))
+
+    # ---- end to end through the public API with host buffers ----
+    pin = lambda t: t.cpu().pin_memory()
+    hq, hk, hv, hdq = pin(q_h), pin(k_h), pin(v_h), pin(dq)
+    ho, hl = torch.empty_like(hq).pin_memory(), torch.empty(p_lse.shape, dtype=torch.float32).pin_memory()
+    hdo, hdl = torch.empty_like(hdq).pin_memory(), torch.empty(d_lse.shape, dtype=torch.float32).pin_memory()
+    e2e_pre, e2e_dec = [], []
+    for i in range(args.e2e_steps + 1):
+        e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        e[0].record(stream)
+        q.copy_(hq, non_blocking=True)
+        k.copy_(hk, non_blocking=True)
+        v.copy_(hv, non_blocking=True)
+        attn.prefill(q, k, v, is_causal=True, out=p_out, lse=p_lse, stream=stream)
+        ho.copy_(p_out, non_blocking=True)
+        hl.copy_(p_lse, non_blocking=True)
+        e[1].record(stream)
+        dq.copy_(hdq, non_blocking=True)
+        attn.decode(dq, dk, dv, dsl, out=d_out, lse=d_lse, workspace=ws, stream=stream)
+        hdo.copy_(d_out, non_blocking=True)
+        hdl.copy_(d_lse, non_blocking=True)
+        e[2].record(stream)
+        torch.cuda.synchronize()
+        if i > 0:   # the first is a warm-up of the copy path
+            e2e_pre.append(e[0].elapsed_time(e[1]))
+            e2e_dec.append(e[1].elapsed_time(e[2]))
+    e2e_pre_ms = max_over_ranks(sum(e2e_pre) / len(e2e_pre))
+    e2e_dec_ms = max_over_ranks(sum(e2e_dec) / len(e2e_dec))
+    h2d = (hq.numel() + hk.numel() + hv.numel() + hdq.numel()) * 2
+    d2h = (ho.numel() + hdo.numel()) * 2 + (hl.numel() + hdl.numel()) * 4
+
+    if rank != 0:
+        return None
+    pre_tflops = world * p_flops / (pre_avg * 1e-3) / 1e12
+    dec_gbs = world * d_bytes / (dec_avg * 1e-3) / 1e9
+    peak_t = float(peaks["bf16_tflops"])
+    peak_b = float(peaks["hbm_gbs"])
+    traffic = load_traffic()
+    line = {
+        "metric": METRIC,
+        "value": round(pre_tflops, 2),
+        "unit": "TFLOP/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(total_ms / args.steps, 4),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic N(0,1) bf16, seeded; Qwen3-8B attention shapes, no weights",
+        "config": {
+            "workload": f"{PREFILL.name} + {DECODE.name}",
+            "prefill": {"B": PREFILL.B, "Hq": PREFILL.Hq, "Hkv": PREFILL.Hkv, "Lq": PREFILL.Lq, "Lk": PREFILL.Lk,
+                        "D": PREFILL.D, "is_causal": True, "flops_per_call": p_flops},
+            "decode": {"B": DECODE.B, "Hq": DECODE.Hq, "Hkv": DECODE.Hkv, "Lmax": DECODE.Lmax, "D": DECODE.D,
+                       "seqlens": "uniform [1024, 32768]", "bytes_per_call": d_bytes},
+            "l2": "inputs larger than L2 (prefill q/k/v 403 MB, decode cache 8.6 GB); no flush",
+            "parallelism": f"replicas x{world} (independent sequences per GPU)",
+        },
+        "decode": {"value": round(dec_gbs, 1), "unit": "GB/s", "ms_per_call": round(dec_avg, 4),
+                   "frac_of_measured_hbm": round(dec_gbs / world / peak_b, 4),
+                   "frac_of_8000": round(dec_gbs / world / 8000.0, 4)},
+        "roofline": {"bound": "tensor", "kernel": "attn_prefill_sm100_kernel",
+                     "achieved": round(pre_tflops / world, 2), "peak": peak_t, "unit": "TFLOP/s",
+                     "frac": round(pre_tflops / world / peak_t, 4),
+                     "peak_source": f"{peaks['source']} bf16_tflops (burst)",
+                     "frac_of_sustained": round(pre_tflops / world / float(peaks.get("bf16_tflops_sustained", peak_t)), 4),
+                     "traffic": traffic.get("attn_prefill_sm100_kernel"),
+                     "ms_per_call": round(pre_avg, 4)},
+        "roofline_decode": {"bound": "hbm", "kernel": "attn_decode_split_kernel + attn_decode_combine_kernel",
+                            "achieved": round(dec_gbs / world, 1), "peak": peak_b, "unit": "GB/s",
+                            "frac": round(dec_gbs / world / peak_b, 4),
+                            "peak_source": f"{peaks['source']} hbm_gbs",
+                            "traffic": traffic.get("attn_decode_split_kernel")},
+        "e2e": {"value": round(world * p_flops / (e2e_pre_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+                "decode_gbs": round(world * d_bytes / (e2e_dec_ms * 1e-3) / 1e9, 1),
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "what": "pinned host -> device inputs, attn_prefill / attn_decode, device -> host outputs; "
+                        "decode KV cache resident"},
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(args, q_h, k_h, v_h, dq.cpu(), dk, dv, seqlens_host)
+    return line
+
+
+def load_traffic():
+    """Per-launch DRAM bytes from the committed ncu summary, if one matches the current kernels."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return {}
+    with open(path) as f:
+        return json.load(f)
+
+
+# --------------------------------------------------------------------------
+# the oracle on this host's cores (bounded samples)
+# --------------------------------------------------------------------------
+def _prefill_sample_rows(n):
+    return sorted(set(int(x) for x in np.linspace(0, PREFILL.Lq - 1, n)))
+
+
+def oracle_prefill_rate(q_h, k_h, v_h, n_rows):
+    import oracle
+    rows = _prefill_sample_rows(n_rows)
+    qb, kb, vb = q_h[:1], k_h[:1], v_h[:1]
+    flops = sum(4 * PREFILL.D * min(PREFILL.Lk, r + PREFILL.Lk - PREFILL.Lq + 1) for r in rows) * PREFILL.Hq
+    t0 = time.perf_counter()
+    oracle.attention_prefill(qb, kb, vb, PREFILL.scale, True, rows=rows)
+    dt = time.perf_counter() - t0
+    return flops, dt, rows
+
+
+def cpu_baseline(args, q_h, k_h, v_h, dq_h, dk, dv, seqlens_host):
+    import oracle
+    cores = oracle.num_threads(0)
+    # calibrate, then size the sample to about args.cpu_seconds
+    f0, t0, _ = oracle_prefill_rate(q_h, k_h, v_h, 8)
+    n = int(max(8, min(PREFILL.Lq, 8 * args.cpu_seconds / max(t0, 1e-3))))
+    flops, dt, rows = oracle_prefill_rate(q_h, k_h, v_h, n)
+    pre = flops / dt / 1e12
+    # decode: whole (b, h) rows of the Qwen3-8B decode batch, cache slices copied to the host
+    G = DECODE.G
+    sel = [(b, g) for b in range(DECODE.B) for g in range(DECODE.Hkv)]
+    rng = np.random.default_rng(0)
+    rng.shuffle(sel)
+    done_bytes, dt_dec, used = 0, 0.0, 0
+    for b, g in sel:
+        n_b = int(seqlens_host[b])
+        kb = dk[b:b + 1, g:g + 1, :n_b].cpu()
+        vb = dv[b:b + 1, g:g + 1, :n_b].cpu()
+        qb = dq_h[b:b + 1, g * G:(g + 1) * G]
+        t0 = time.perf_counter()
+        oracle.attention_decode(qb, kb, vb, np.array([n_b], np.int32), DECODE.scale)
+        dt_dec += time.perf_counter() - t0
+        done_bytes += n_b * DECODE.D * 2 * 2 + G * DECODE.D * 2 * 2 + G * 4
+        used += 1
+        if dt_dec > args.cpu_seconds / 2:
+            break
+    return {"value": round(pre, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+            "sample": f"prefill: batch 0, all 32 heads, {len(rows)} query rows spread over 0..8191 "
+                      f"({flops / 1e9:.1f} GFLOP in {dt:.1f} s); fp64 C eager attention, OpenMP",
+            "decode": {"value": round(done_bytes / dt_dec / 1e9, 4), "unit": "GB/s",
+                       "sample": f"{used} (batch, KV head) groups of the decode batch, {dt_dec:.1f} s"}}
+
+
+def run_reference(args, rank, world):
+    """The oracle as it stands, on this host's cores, each step a bounded sample."""
+    if rank != 0:
+        return None
+    import oracle
+    oracle.build()
+    q_h, k_h, v_h = W.prefill_inputs_for(PREFILL, seed=args.seed, device="cpu")
+    cores = oracle.num_threads(0)
+    f0, t0, _ = oracle_prefill_rate(q_h, k_h, v_h, 8)
+    budget = 120.0 / max(1, args.steps + args.warmup)          # whole run within a few minutes
+    n = int(max(8, min(PREFILL.Lq, 8 * budget / max(t0, 1e-3))))
+    for _ in range(args.warmup):
+        oracle_prefill_rate(q_h, k_h, v_h, 8)
+    flops_t, dt_t = 0, 0.0
+    for _ in range(args.steps):
+        f, dt, rows = oracle_prefill_rate(q_h, k_h, v_h, n)
+        flops_t += f
+        dt_t += dt
+    val = flops_t / dt_t / 1e12
+    return {
+        "metric": METRIC, "value": round(val, 6), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(1e3 * dt_t / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic N(0,1) bf16, seeded",
+        "impl": "reference",
+        "config": {"workload": f"{PREFILL.name} (sampled query rows)", "rows_per_step": n},
+        "cpu_baseline": {"value": round(val, 6), "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                         "sample": f"batch 0, all heads, {n} query rows per step"},
+        "e2e": {"value": round(val, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        line = run_reference(args, rank, world)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+        return
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if line is not None:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

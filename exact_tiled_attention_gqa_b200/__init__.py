@@ -1,0 +1,119 @@
+"""Exact tiled grouped-query attention for NVIDIA B200 (sm_100a).
+
+Two calls, both thin wrappers over the C ABI in ``include/attn_gqa.h``:
+
+* ``prefill(q, k, v, is_causal=True)`` -- softmax(scale Q K^T + mask) V with
+  the bottom-right causal mask, for Q [B,Hq,Lq,D] and K/V [B,Hkv,Lk,D] bf16.
+* ``decode(q, k_cache, v_cache, seqlens)`` -- one new token per sequence
+  against a KV cache [B,Hkv,Lmax,D] whose rows 0..seqlens[b]-1 are valid.
+
+Both return ``(out, lse)``: out bf16 shaped like q, lse fp32 (natural log).
+PyTorch supplies device memory and the current stream; every step of the
+computation runs in the library's CUDA kernels.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from typing import Optional
+
+import torch
+
+from . import _native
+from ._native import AttnError
+
+__all__ = ["prefill", "decode", "decode_workspace_size", "device_error", "AttnError", "library_path"]
+
+
+def library_path() -> str:
+    return _native.LIB_PATH
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_handle(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check_tensor(name: str, t: torch.Tensor, dtype: torch.dtype, ndim: int) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must be {ndim}-d, got shape {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: Optional[float] = None,
+            is_causal: bool = True, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+            want_lse: bool = True, stream=None):
+    """Exact GQA attention.  q [B,Hq,Lq,D], k/v [B,Hkv,Lk,D] bf16 (CUDA, contiguous)."""
+    for n, t in (("q", q), ("k", k), ("v", v)):
+        _check_tensor(n, t, torch.bfloat16, 4)
+    B, Hq, Lq, D = q.shape
+    Hkv, Lk = k.shape[1], k.shape[2]
+    if k.shape[0] != B or k.shape[3] != D or v.shape != k.shape:
+        raise ValueError(f"shape mismatch: q {tuple(q.shape)} k {tuple(k.shape)} v {tuple(v.shape)}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    else:
+        _check_tensor("out", out, torch.bfloat16, 4)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    elif lse is not None:
+        _check_tensor("lse", lse, torch.float32, 3)
+    with torch.cuda.device(q.device):
+        st = _native.lib().attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Lq, Lk, D,
+                                        float(scale), int(bool(is_causal)), _stream_handle(stream))
+    _native.check(st, "attn_prefill")
+    return out, lse
+
+
+def decode_workspace_size(B: int, Hq: int, Hkv: int, Lmax: int, D: int) -> int:
+    return int(_native.lib().attn_decode_workspace_size(B, Hq, Hkv, Lmax, D))
+
+
+def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, seqlens: torch.Tensor, *,
+           scale: Optional[float] = None, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+           want_lse: bool = True, workspace: Optional[torch.Tensor] = None, stream=None):
+    """One query token per sequence.  q [B,Hq,D], caches [B,Hkv,Lmax,D] bf16, seqlens int32 [B] (CUDA)."""
+    _check_tensor("q", q, torch.bfloat16, 3)
+    _check_tensor("k_cache", k_cache, torch.bfloat16, 4)
+    _check_tensor("v_cache", v_cache, torch.bfloat16, 4)
+    _check_tensor("seqlens", seqlens, torch.int32, 1)
+    B, Hq, D = q.shape
+    Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
+    if k_cache.shape[0] != B or k_cache.shape[3] != D or v_cache.shape != k_cache.shape or seqlens.shape[0] != B:
+        raise ValueError("shape mismatch between q, the caches and seqlens")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    need = decode_workspace_size(B, Hq, Hkv, Lmax, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    with torch.cuda.device(q.device):
+        st = _native.lib().attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(out), _ptr(lse),
+                                       B, Hq, Hkv, Lmax, D, float(scale), _ptr(workspace), workspace.numel(),
+                                       _stream_handle(stream))
+    _native.check(st, "attn_decode")
+    return out, lse
+
+
+def device_error(reset: bool = True) -> int:
+    """Synchronise and return (and by default clear) the device-side error word."""
+    flags = ctypes.c_uint(0)
+    _native.check(_native.lib().attn_device_error(ctypes.byref(flags), int(bool(reset))), "attn_device_error")
+    return int(flags.value)

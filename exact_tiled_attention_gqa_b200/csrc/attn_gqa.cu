@@ -1,0 +1,304 @@
+// attn_gqa.cu -- the C ABI of include/attn_gqa.h: argument checks, TMA
+// descriptors and kernel launches.  All arithmetic happens in the kernels of
+// prefill_sm100.cuh and decode_sm100.cuh; this file only validates, describes
+// the caller's tensors to the TMA unit and enqueues work on the caller's
+// stream.  There is no other code path: no fallback, no host compute.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdint>
+#include <cstdio>
+#include <mutex>
+
+#include "../../include/attn_gqa.h"
+#include "decode_sm100.cuh"
+#include "prefill_sm100.cuh"
+
+namespace attn {
+namespace {
+
+thread_local char g_last_error[320] = "";
+
+int fail(int status, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_last_error, sizeof g_last_error, fmt, ap);
+    va_end(ap);
+    return status;
+}
+
+int ok() {
+    g_last_error[0] = '\0';
+    return ATTN_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---- cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda) ----
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* sym = nullptr;
+        cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &sym, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(sym);
+    });
+    return fn;
+}
+
+// A dense bf16 tensor [d2][d1][d0] (d0 contiguous) read in boxes of
+// (box0, box1, box2) elements with 128-byte swizzle; out-of-range rows read as 0.
+int encode_bf16_3d(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0,
+                   uint32_t box1, uint32_t box2, const char* what) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the CUDA driver");
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {d0 * 2, d0 * d1 * 2};
+    cuuint32_t box[3] = {box0, box1, box2};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for %s", (int)r, what);
+    return ATTN_OK;
+}
+
+// Allow a kernel its dynamic shared memory (once per device and kernel).
+template <typename Kernel>
+int ensure_smem(Kernel kernel, int bytes, int* done_mask_per_device) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= 64) return fail(ATTN_ERR_CUDA, "device ordinal %d out of range", dev);
+    if (__atomic_load_n(&done_mask_per_device[dev], __ATOMIC_ACQUIRE)) return ATTN_OK;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "cudaFuncSetAttribute: %s", cudaGetErrorString(e));
+    __atomic_store_n(&done_mask_per_device[dev], 1, __ATOMIC_RELEASE);
+    return ATTN_OK;
+}
+
+int check_launch(const char* what) {
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString(e));
+    return ATTN_OK;
+}
+
+// Rows that see no key at all (Lk == 0): O = 0, LSE = -inf.
+__global__ void fill_no_key_rows_kernel(__nv_bfloat16* out, float* lse, size_t rows, int D) {
+    const size_t n = rows * static_cast<size_t>(D);
+    for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+        out[i] = __float2bfloat16(0.0f);
+        if (lse != nullptr && i % D == 0) lse[i / D] = -INFINITY;
+    }
+}
+
+template <int D>
+int launch_prefill(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
+                   int Lq, int Lk, float scale, int is_causal, cudaStream_t stream) {
+    static int smem_done[64];
+    using L = PrefillSmem<D>;
+    const int G = Hq / Hkv;
+    const int P = kBM / G;
+    CUtensorMap tq, tk, tv;
+    int st;
+    if ((st = encode_bf16_3d(&tq, q, D, Lq, static_cast<uint64_t>(B) * Hq, 64, P, G, "q")) != ATTN_OK) return st;
+    if ((st = encode_bf16_3d(&tk, k, D, Lk, static_cast<uint64_t>(B) * Hkv, 64, kBN, 1, "k")) != ATTN_OK) return st;
+    if ((st = encode_bf16_3d(&tv, v, D, Lk, static_cast<uint64_t>(B) * Hkv, 64, kBN, 1, "v")) != ATTN_OK) return st;
+    if ((st = ensure_smem(attn_prefill_sm100_kernel<D>, L::kAlloc, smem_done)) != ATTN_OK) return st;
+    PrefillParams prm;
+    prm.out = out;
+    prm.lse = lse;
+    prm.B = B;
+    prm.Hq = Hq;
+    prm.Hkv = Hkv;
+    prm.Lq = Lq;
+    prm.Lk = Lk;
+    prm.G = G;
+    prm.P = P;
+    prm.n_mblk = (Lq + 2 * P - 1) / (2 * P);
+    prm.is_causal = is_causal ? 1 : 0;
+    prm.scale_log2 = scale * kLog2e;
+    const long long grid = static_cast<long long>(B) * Hkv * prm.n_mblk;
+    if (grid > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "prefill grid too large (%lld CTAs)", grid);
+    attn_prefill_sm100_kernel<D><<<static_cast<unsigned>(grid), kPrefillThreads, L::kAlloc, stream>>>(tq, tk, tv, prm);
+    return check_launch("attn_prefill_sm100_kernel");
+}
+
+// Cache rows per decode split: the largest power of two in [256, 4096] that
+// still gives about four waves of CTAs on a 148-SM part.
+int decode_chunk(int B, int Hkv, int Lmax) {
+    const long long target = 148LL * 2 * 4;
+    int chunk = 4096;
+    while (chunk > 256 && static_cast<long long>(B) * Hkv * ((Lmax + chunk - 1) / chunk) < target) chunk >>= 1;
+    return chunk;
+}
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+struct DecodeLayout {
+    int chunk, n_splits;
+    size_t o_bytes, lse_off, total;
+};
+
+DecodeLayout decode_layout(int B, int Hq, int Hkv, int Lmax, int D) {
+    DecodeLayout d;
+    d.chunk = decode_chunk(B, Hkv, Lmax);
+    d.n_splits = (Lmax + d.chunk - 1) / d.chunk;
+    const size_t rows = static_cast<size_t>(B) * Hq * d.n_splits;
+    d.o_bytes = align256(rows * D * sizeof(float));
+    d.lse_off = d.o_bytes;
+    d.total = d.o_bytes + align256(rows * sizeof(float));
+    return d;
+}
+
+template <int D, int KPW>
+int launch_decode_split(const CUtensorMap& tk, const CUtensorMap& tv, const DecodeParams& prm, cudaStream_t stream) {
+    static int smem_done[64];
+    using L = DecodeSmem<D>;
+    int st;
+    if ((st = ensure_smem(attn_decode_split_kernel<D, KPW>, L::kAlloc, smem_done)) != ATTN_OK) return st;
+    dim3 grid(prm.n_splits, prm.Hkv, prm.B);
+    attn_decode_split_kernel<D, KPW><<<grid, kDecThreads, L::kAlloc, stream>>>(tk, tv, prm);
+    return check_launch("attn_decode_split_kernel");
+}
+
+template <int D>
+int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* seqlens, void* out, float* lse, int B,
+                  int Hq, int Hkv, int Lmax, float scale, void* workspace, cudaStream_t stream) {
+    const DecodeLayout lay = decode_layout(B, Hq, Hkv, Lmax, D);
+    CUtensorMap tk, tv;
+    int st;
+    if ((st = encode_bf16_3d(&tk, kc, D, Lmax, static_cast<uint64_t>(B) * Hkv, 64, kDecKT, 1, "k_cache")) != ATTN_OK)
+        return st;
+    if ((st = encode_bf16_3d(&tv, vc, D, Lmax, static_cast<uint64_t>(B) * Hkv, 64, kDecKT, 1, "v_cache")) != ATTN_OK)
+        return st;
+    DecodeParams prm;
+    prm.q = static_cast<const __nv_bfloat16*>(q);
+    prm.seqlens = seqlens;
+    prm.o_part = static_cast<float*>(workspace);
+    prm.lse_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + lay.lse_off);
+    prm.B = B;
+    prm.Hq = Hq;
+    prm.Hkv = Hkv;
+    prm.Lmax = Lmax;
+    prm.G = Hq / Hkv;
+    prm.chunk = lay.chunk;
+    prm.n_splits = lay.n_splits;
+    prm.scale_log2 = scale * kLog2e;
+    if (prm.n_splits > 65535 || Hkv > 65535 || B > 65535)
+        return fail(ATTN_ERR_UNSUPPORTED, "decode grid (%d, %d, %d) exceeds launch limits", prm.n_splits, Hkv, B);
+    if (prm.G <= 16)
+        st = launch_decode_split<D, 16>(tk, tv, prm, stream);
+    else if (prm.G <= 32)
+        st = launch_decode_split<D, 32>(tk, tv, prm, stream);
+    else
+        st = launch_decode_split<D, 64>(tk, tv, prm, stream);
+    if (st != ATTN_OK) return st;
+    const int rows = B * Hq;
+    attn_decode_combine_kernel<D><<<(rows + 3) / 4, 128, 0, stream>>>(prm, static_cast<__nv_bfloat16*>(out), lse);
+    return check_launch("attn_decode_combine_kernel");
+}
+
+int check_common(const void* q, const void* k, const void* v, const void* out, const float* lse, int B, int Hq,
+                 int Hkv, int L1, int L2, int D, float scale, const char* l1name, const char* l2name) {
+    if (!q || !k || !v || !out) return fail(ATTN_ERR_INVALID_ARG, "null tensor pointer");
+    if (B < 0 || L1 < 0 || L2 < 0)
+        return fail(ATTN_ERR_INVALID_ARG, "negative size (B=%d %s=%d %s=%d)", B, l1name, L1, l2name, L2);
+    if (Hq < 1 || Hkv < 1) return fail(ATTN_ERR_INVALID_ARG, "head counts must be >= 1 (Hq=%d Hkv=%d)", Hq, Hkv);
+    if (Hq % Hkv != 0) return fail(ATTN_ERR_INVALID_ARG, "Hq=%d is not a multiple of Hkv=%d", Hq, Hkv);
+    if (!(std::isfinite(scale) && scale > 0.0f)) return fail(ATTN_ERR_INVALID_ARG, "scale must be finite and > 0");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+        return fail(ATTN_ERR_INVALID_ARG, "tensor base addresses must be 16-byte aligned");
+    if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))
+        return fail(ATTN_ERR_INVALID_ARG, "lse must be 4-byte aligned");
+    if (D != 64 && D != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim D=%d (built: 64, 128)", D);
+    return ATTN_OK;
+}
+
+}  // namespace
+}  // namespace attn
+
+using namespace attn;
+
+extern "C" int attn_prefill(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
+                            int Hkv, int Lq, int Lk, int D, float scale, int is_causal, void* stream) {
+    int st = check_common(q, k, v, out, lse, B, Hq, Hkv, Lq, Lk, D, scale, "Lq", "Lk");
+    if (st != ATTN_OK) return st;
+    if (Hq / Hkv > kBM) return fail(ATTN_ERR_UNSUPPORTED, "group size G=%d > %d", Hq / Hkv, kBM);
+    if (static_cast<long long>(B) * Hq > 0x7fffffffLL || static_cast<long long>(B) * Hkv > 0x7fffffffLL)
+        return fail(ATTN_ERR_UNSUPPORTED, "B*H too large");
+    if (B == 0 || Lq == 0) return ok();
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (Lk == 0) {
+        const size_t rows = static_cast<size_t>(B) * Hq * Lq;
+        fill_no_key_rows_kernel<<<1184, 256, 0, s>>>(static_cast<__nv_bfloat16*>(out), lse, rows, D);
+        st = check_launch("fill_no_key_rows_kernel");
+        return st == ATTN_OK ? ok() : st;
+    }
+    st = (D == 128) ? launch_prefill<128>(q, k, v, out, lse, B, Hq, Hkv, Lq, Lk, scale, is_causal, s)
+                    : launch_prefill<64>(q, k, v, out, lse, B, Hq, Hkv, Lq, Lk, scale, is_causal, s);
+    return st == ATTN_OK ? ok() : st;
+}
+
+extern "C" size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int D) {
+    if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Lmax < 1 || (D != 64 && D != 128) || Hq / Hkv > 64)
+        return 0;
+    if (B == 0) return 0;
+    return decode_layout(B, Hq, Hkv, Lmax, D).total;
+}
+
+extern "C" int attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens, void* out,
+                           float* lse, int B, int Hq, int Hkv, int Lmax, int D, float scale, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+    int st = check_common(q, k_cache, v_cache, out, lse, B, Hq, Hkv, Lmax, Lmax, D, scale, "Lmax", "Lmax");
+    if (st != ATTN_OK) return st;
+    if (!seqlens) return fail(ATTN_ERR_INVALID_ARG, "null seqlens");
+    if (reinterpret_cast<uintptr_t>(seqlens) & 3u) return fail(ATTN_ERR_INVALID_ARG, "seqlens must be 4-byte aligned");
+    if (Lmax < 1) return fail(ATTN_ERR_INVALID_ARG, "Lmax must be >= 1");
+    if (Hq / Hkv > 64) return fail(ATTN_ERR_UNSUPPORTED, "decode group size G=%d > 64", Hq / Hkv);
+    if (static_cast<long long>(B) * Hq > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "B*Hq too large");
+    if (B == 0) return ok();
+    const size_t need = decode_layout(B, Hq, Hkv, Lmax, D).total;
+    if (!workspace || workspace_bytes < need)
+        return fail(ATTN_ERR_WORKSPACE, "decode workspace needs %zu bytes, got %zu", need,
+                    workspace ? workspace_bytes : static_cast<size_t>(0));
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+        return fail(ATTN_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = (D == 128) ? launch_decode<128>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s)
+                    : launch_decode<64>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s);
+    return st == ATTN_OK ? ok() : st;
+}
+
+extern "C" const char* attn_status_string(int status) {
+    switch (status) {
+        case ATTN_OK: return "ATTN_OK";
+        case ATTN_ERR_INVALID_ARG: return "ATTN_ERR_INVALID_ARG";
+        case ATTN_ERR_UNSUPPORTED: return "ATTN_ERR_UNSUPPORTED";
+        case ATTN_ERR_WORKSPACE: return "ATTN_ERR_WORKSPACE";
+        case ATTN_ERR_CUDA: return "ATTN_ERR_CUDA";
+        default: return "ATTN_ERR_UNKNOWN";
+    }
+}
+
+extern "C" const char* attn_last_error(void) { return g_last_error; }
+
+extern "C" int attn_device_error(unsigned int* flags, int reset) {
+    if (!flags) return fail(ATTN_ERR_INVALID_ARG, "null flags");
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "cudaDeviceSynchronize: %s", cudaGetErrorString(e));
+    e = cudaMemcpyFromSymbol(flags, g_attn_err, sizeof(unsigned int));
+    if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "reading the device error word: %s", cudaGetErrorString(e));
+    if (reset) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_attn_err, &zero, sizeof zero);
+        if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "clearing the device error word: %s", cudaGetErrorString(e));
+    }
+    return ok();
+}

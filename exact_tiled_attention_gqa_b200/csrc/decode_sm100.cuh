@@ -1,0 +1,369 @@
+// decode_sm100.cuh -- split-KV GQA decode and its log-sum-exp combine.
+//
+// What it computes: for each sequence b and query head h, one new query row
+// against cache rows 0 .. seqlens[b]-1 of KV head h / G (no mask: the new
+// token sees every cached key -- the "use_cache" and is_causal sections of
+// the SDPA / FlashAttention selection guide).  Decode is bound by reading the
+// cache (NVIDIA attention page, "Prefill and decode are two different
+// tasks"), so the kernel is built around streaming K and V once at full HBM
+// bandwidth:
+//
+//   split kernel  grid (split, KV head, batch).  A CTA owns `chunk` cache rows
+//                 of one (b, KV head): a producer warp streams 64-row K and V
+//                 tiles into a ring of shared-memory stages with TMA (128-byte
+//                 swizzle, so the ldmatrix reads below are conflict-free); four
+//                 compute warps multiply the G query heads of the group (as
+//                 the M rows of m16n8k16 tensor-core MMAs, padded to 16) with
+//                 each tile once, run an online softmax, and accumulate P V.
+//                 Warps sharing a 16-row block split the tile's keys and merge
+//                 through shared memory at the end; the CTA writes one
+//                 normalised partial output and its log2-sum-exp per row.
+//   combine       one warp per (b, h): LSE-weighted sum of that row's partials.
+//
+// Splitting the cache length and merging by log-sum-exp is the single-GPU
+// form of the KV parallelism on the NVIDIA page ("Parameter four").
+#pragma once
+
+#include "ptx_sm100.cuh"
+#include "device_error.cuh"
+
+namespace attn {
+
+constexpr int kDecThreads = 160;   // warps 0-3 compute, warp 4 TMA producer
+constexpr int kDecKT = 64;         // cache rows per tile
+
+template <int D>
+struct DecodeSmem {
+    static constexpr int kKB = D / 64;
+    static constexpr int kBlockBytes = kDecKT * 128;        // 64 rows x 128 bytes
+    static constexpr int kTileBytes = kDecKT * D * 2;       // one K or V tile
+    static constexpr int kStageBytes = 2 * kTileBytes;      // K then V
+    static constexpr int kStages = (D == 128) ? 3 : 6;
+    static constexpr int kRingBytes = kStages * kStageBytes;
+    // end-of-CTA merge area (reuses the ring): m[4][16], l[4][16], O[4][16][D]
+    static constexpr int kMergeBytes = 4 * 16 * 4 * 2 + 4 * 16 * D * 4;
+    static_assert(kMergeBytes <= kRingBytes, "merge area must fit in the ring");
+    static constexpr int kBarOff = kRingBytes;
+    static constexpr int kBytes = kBarOff + 2 * kStages * 8 + 16;
+    static constexpr int kAlloc = kBytes + 1024;
+};
+
+struct DecodeParams {
+    const __nv_bfloat16* q;   // [B,Hq,D]
+    const int* seqlens;       // [B]
+    float* o_part;            // [B,Hq,n_splits,D]
+    float* lse_part;          // [B,Hq,n_splits] (log2 domain)
+    int B, Hq, Hkv, Lmax, G;
+    int chunk;                // cache rows per split (multiple of 64)
+    int n_splits;
+    float scale_log2;
+};
+
+__device__ __forceinline__ int decode_seqlen(const DecodeParams& p, int b) {
+    int n = p.seqlens[b];
+    if (n < 0 || n > p.Lmax) {
+        atomicOr(&g_attn_err, kDevErrSeqlen);
+        n = n < 0 ? 0 : p.Lmax;
+    }
+    return n;
+}
+
+// KPW = cache rows of each 64-row tile handled by one compute warp (16, 32 or 64)
+template <int D, int KPW>
+__global__ void __maxnreg__(200)
+    attn_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
+                             const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
+    using L = DecodeSmem<D>;
+    constexpr int kNT = KPW / 8;          // 8-key n-tiles of S per warp
+    constexpr int kWPM = kDecKT / KPW;    // warps per 16-row block
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_base = smem_u32(smem_raw);
+    const uint32_t base = (raw_base + 1023u) & ~1023u;
+    uint8_t* smem = smem_raw + (base - raw_base);
+
+    const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int seqlen = decode_seqlen(p, b);
+    const int k_begin = split * p.chunk;
+    if (k_begin >= seqlen) return;   // uniform: this split has no rows
+    const int k_end = min(k_begin + p.chunk, seqlen);
+    const int n_tiles = (k_end - k_begin + kDecKT - 1) / kDecKT;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t ring = base;
+    const uint32_t bar0 = base + L::kBarOff;
+    auto bar_full = [&](int s) { return bar0 + 8u * s; };
+    auto bar_empty = [&](int s) { return bar0 + 8u * (L::kStages + s); };
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kBarOff + 2 * L::kStages * 8);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < L::kStages; ++s) {
+            mbar_init(bar_full(s), 1);
+            mbar_init(bar_empty(s), 4);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp == 4) {
+        // ================= TMA producer =================
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            const int kv_row = b * p.Hkv + g;
+            int issued = 0;
+            for (int t = 0; t < n_tiles; ++t) {
+                const int s = t % L::kStages;
+                const uint32_t round = static_cast<uint32_t>(t / L::kStages);
+                if (!mbar_wait(bar_empty(s), (round & 1u) ^ 1u, abort_flag, &g_attn_err, kDevErrTimeout)) break;
+                mbar_arrive_expect_tx(bar_full(s), L::kStageBytes);
+                const uint32_t dst = ring + s * L::kStageBytes;
+                for (int kb = 0; kb < L::kKB; ++kb) {
+                    tma_load_3d(dst + kb * L::kBlockBytes, &tm_k, bar_full(s), kb * 64, k_begin + t * kDecKT, kv_row);
+                    tma_load_3d(dst + L::kTileBytes + kb * L::kBlockBytes, &tm_v, bar_full(s), kb * 64,
+                                k_begin + t * kDecKT, kv_row);
+                }
+                issued = t + 1;
+            }
+            if (issued < n_tiles) {
+                // unwinding after a timeout: let issued copies land first
+                for (int t = max(0, issued - L::kStages); t < issued; ++t) {
+                    const uint64_t t0 = global_timer_ns();
+                    while (!mbar_try_wait(bar_full(t % L::kStages), static_cast<uint32_t>(t / L::kStages) & 1u) &&
+                           global_timer_ns() - t0 < 100000000ull) {
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        return;   // the producer takes no part in the merge below
+    }
+
+    // ================= compute warps =================
+    const int mt = warp / kWPM;           // 16-row block of query heads
+    const int ws = warp % kWPM;           // which slice of each tile's keys
+    const int key_off = ws * KPW;
+    const int grp = lane >> 2, tq = lane & 3;
+    const int h0 = g * p.G + mt * 16;     // first query head of this block
+    const int row_a = mt * 16 + grp, row_b = row_a + 8;   // rows (within the group) this thread holds
+
+    // Q as m16n8k16 A fragments (rows beyond G are zero)
+    uint32_t qa[D / 16][4];
+    {
+        const uint32_t* qrow_a = reinterpret_cast<const uint32_t*>(p.q + (static_cast<size_t>(b) * p.Hq + h0 + grp) * D);
+        const uint32_t* qrow_b = reinterpret_cast<const uint32_t*>(p.q + (static_cast<size_t>(b) * p.Hq + h0 + grp + 8) * D);
+        const bool va = row_a < p.G, vb = row_b < p.G;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const int c = (kk * 16 + 2 * tq) >> 1;   // bf16x2 index
+            qa[kk][0] = va ? __ldg(qrow_a + c) : 0u;
+            qa[kk][1] = vb ? __ldg(qrow_b + c) : 0u;
+            qa[kk][2] = va ? __ldg(qrow_a + c + 4) : 0u;
+            qa[kk][3] = vb ? __ldg(qrow_b + c + 4) : 0u;
+        }
+    }
+
+    float oacc[D / 8][4];
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.0f;
+    float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.0f, l_b = 0.0f;
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+
+    for (int t = 0; t < n_tiles; ++t) {
+        const int s = t % L::kStages;
+        ok = mbar_wait(bar_full(s), static_cast<uint32_t>(t / L::kStages) & 1u, abort_flag, &g_attn_err, kDevErrTimeout);
+        if (!ok) break;
+        const uint32_t kbase = ring + s * L::kStageBytes;
+        const uint32_t vbase = kbase + L::kTileBytes;
+        const int tile_key0 = k_begin + t * kDecKT + key_off;   // absolute row of this warp's first key
+        const bool tail = (k_begin + (t + 1) * kDecKT > k_end);
+
+        // ---- S = Q K^T over this warp's KPW keys ----
+        float sacc[kNT][4];
+#pragma unroll
+        for (int i = 0; i < kNT; ++i) sacc[i][0] = sacc[i][1] = sacc[i][2] = sacc[i][3] = 0.0f;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t region = kbase + (kk >> 2) * L::kBlockBytes;
+            const int cbase = (kk & 3) * 2;
+#pragma unroll
+            for (int np = 0; np < kNT / 2; ++np) {
+                const int mi = lane >> 3, rr = lane & 7;
+                const int key_local = key_off + np * 16 + ((mi >> 1) << 3) + rr;
+                const int c = cbase + (mi & 1);
+                const uint32_t addr = region + key_local * 128 + ((c ^ (key_local & 7)) << 4);
+                uint32_t r0, r1, r2, r3;
+                ldmatrix_x4(addr, r0, r1, r2, r3);
+                mma_bf16_16816(sacc[2 * np], qa[kk], r0, r1);
+                mma_bf16_16816(sacc[2 * np + 1], qa[kk], r2, r3);
+            }
+        }
+        // ---- mask rows beyond the valid length (only the last tile) ----
+        if (tail) {
+#pragma unroll
+            for (int nt = 0; nt < kNT; ++nt) {
+                const int key = tile_key0 + nt * 8 + 2 * tq;
+                if (key >= k_end) sacc[nt][0] = sacc[nt][2] = -INFINITY;
+                if (key + 1 >= k_end) sacc[nt][1] = sacc[nt][3] = -INFINITY;
+            }
+        }
+        // ---- online softmax (log2 domain), rows a and b ----
+        float mx_a = -INFINITY, mx_b = -INFINITY;
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt) {
+            mx_a = fmaxf(mx_a, fmaxf(sacc[nt][0], sacc[nt][1]));
+            mx_b = fmaxf(mx_b, fmaxf(sacc[nt][2], sacc[nt][3]));
+        }
+        mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 1));
+        mx_a = fmaxf(mx_a, __shfl_xor_sync(0xffffffffu, mx_a, 2));
+        mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 1));
+        mx_b = fmaxf(mx_b, __shfl_xor_sync(0xffffffffu, mx_b, 2));
+        const float mn_a = fmaxf(m_a, mx_a * sl2), mn_b = fmaxf(m_b, mx_b * sl2);
+        const float f_a = (m_a == -INFINITY) ? 0.0f : ex2_approx(m_a - mn_a);
+        const float f_b = (m_b == -INFINITY) ? 0.0f : ex2_approx(m_b - mn_b);
+        const float ms_a = (mn_a == -INFINITY) ? 0.0f : mn_a;
+        const float ms_b = (mn_b == -INFINITY) ? 0.0f : mn_b;
+        m_a = mn_a;
+        m_b = mn_b;
+        float ps_a = 0.0f, ps_b = 0.0f;
+#pragma unroll
+        for (int nt = 0; nt < kNT; ++nt) {
+            sacc[nt][0] = ex2_approx(fmaf(sacc[nt][0], sl2, -ms_a));
+            sacc[nt][1] = ex2_approx(fmaf(sacc[nt][1], sl2, -ms_a));
+            sacc[nt][2] = ex2_approx(fmaf(sacc[nt][2], sl2, -ms_b));
+            sacc[nt][3] = ex2_approx(fmaf(sacc[nt][3], sl2, -ms_b));
+            ps_a += sacc[nt][0] + sacc[nt][1];
+            ps_b += sacc[nt][2] + sacc[nt][3];
+        }
+        l_a = l_a * f_a + ps_a;
+        l_b = l_b * f_b + ps_b;
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) {
+            oacc[i][0] *= f_a;
+            oacc[i][1] *= f_a;
+            oacc[i][2] *= f_b;
+            oacc[i][3] *= f_b;
+        }
+        // ---- O += P V ----
+#pragma unroll
+        for (int k2 = 0; k2 < KPW / 16; ++k2) {
+            uint32_t a[4];
+            a[0] = pack_bf16x2(sacc[2 * k2][0], sacc[2 * k2][1]);
+            a[1] = pack_bf16x2(sacc[2 * k2][2], sacc[2 * k2][3]);
+            a[2] = pack_bf16x2(sacc[2 * k2 + 1][0], sacc[2 * k2 + 1][1]);
+            a[3] = pack_bf16x2(sacc[2 * k2 + 1][2], sacc[2 * k2 + 1][3]);
+            // keys held by this thread's V fragments: rows klo, klo+1 (r0, r2) and klo+8, klo+9 (r1, r3)
+            const int klo = tile_key0 + k2 * 16 + 2 * tq;
+            uint32_t keep_lo = 0xffffffffu, keep_hi = 0xffffffffu;
+            if (tail) {
+                keep_lo = (klo < k_end ? 0x0000ffffu : 0u) | (klo + 1 < k_end ? 0xffff0000u : 0u);
+                keep_hi = (klo + 8 < k_end ? 0x0000ffffu : 0u) | (klo + 9 < k_end ? 0xffff0000u : 0u);
+            }
+#pragma unroll
+            for (int nd = 0; nd < D / 16; ++nd) {
+                const int mi = lane >> 3, rr = lane & 7;
+                const int key_local = key_off + k2 * 16 + ((mi & 1) << 3) + rr;
+                const int dchunk = nd * 2 + (mi >> 1);
+                const uint32_t addr = vbase + (dchunk >> 3) * L::kBlockBytes + key_local * 128 +
+                                      (((dchunk & 7) ^ (key_local & 7)) << 4);
+                uint32_t r0, r1, r2, r3;
+                ldmatrix_x4_trans(addr, r0, r1, r2, r3);
+                // rows past the valid length may hold anything (NaN): zero them so 0 * NaN cannot appear
+                r0 &= keep_lo;
+                r2 &= keep_lo;
+                r1 &= keep_hi;
+                r3 &= keep_hi;
+                mma_bf16_16816(oacc[2 * nd], a, r0, r1);
+                mma_bf16_16816(oacc[2 * nd + 1], a, r2, r3);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_empty(s));
+    }
+
+    // ---- merge the warps of each 16-row block through shared memory ----
+    l_a += __shfl_xor_sync(0xffffffffu, l_a, 1);
+    l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
+    l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
+    l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+    asm volatile("bar.sync 1, 128;" ::: "memory");   // every compute warp is done with the ring
+    float* sm_m = reinterpret_cast<float*>(smem);
+    float* sm_l = sm_m + 4 * 16;
+    float* sm_o = sm_l + 4 * 16;
+    if (tq == 0) {
+        sm_m[warp * 16 + grp] = m_a;
+        sm_m[warp * 16 + grp + 8] = m_b;
+        sm_l[warp * 16 + grp] = l_a;
+        sm_l[warp * 16 + grp + 8] = l_b;
+    }
+#pragma unroll
+    for (int nt = 0; nt < D / 8; ++nt) {
+        const int d = nt * 8 + 2 * tq;
+        float* oa = sm_o + (warp * 16 + grp) * D + d;
+        float* ob = sm_o + (warp * 16 + grp + 8) * D + d;
+        oa[0] = oacc[nt][0];
+        oa[1] = oacc[nt][1];
+        ob[0] = oacc[nt][2];
+        ob[1] = oacc[nt][3];
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (!ok) return;
+    for (int idx = threadIdx.x; idx < p.G * D; idx += 128) {
+        const int row = idx / D, d = idx % D;
+        const int blk = row >> 4, rr = row & 15;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kWPM; ++w) M = fmaxf(M, sm_m[(blk * kWPM + w) * 16 + rr]);
+        float Lsum = 0.0f, acc = 0.0f;
+#pragma unroll
+        for (int w = 0; w < kWPM; ++w) {
+            const int ww = blk * kWPM + w;
+            const float mw = sm_m[ww * 16 + rr];
+            const float sc = (mw == -INFINITY) ? 0.0f : ex2_approx(mw - M);
+            Lsum += sm_l[ww * 16 + rr] * sc;
+            acc += sm_o[(ww * 16 + rr) * D + d] * sc;
+        }
+        const int h = g * p.G + row;
+        const size_t prow = (static_cast<size_t>(b) * p.Hq + h) * p.n_splits + split;
+        p.o_part[prow * D + d] = (Lsum > 0.0f) ? acc / Lsum : 0.0f;
+        if (d == 0) p.lse_part[prow] = (Lsum > 0.0f) ? M + __log2f(Lsum) : -INFINITY;
+    }
+}
+
+// One warp per (b, h): out = sum_s 2^(lse_s - lse) O_s,  lse = log2 sum_s 2^lse_s.
+template <int D>
+__global__ void __launch_bounds__(128)
+    attn_decode_combine_kernel(const DecodeParams p, __nv_bfloat16* out, float* lse) {
+    const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= p.B * p.Hq) return;
+    const int b = row / p.Hq;
+    const int seqlen = decode_seqlen(p, b);
+    const int n_valid = (seqlen + p.chunk - 1) / p.chunk;
+    const float* lp = p.lse_part + static_cast<size_t>(row) * p.n_splits;
+    const float* op = p.o_part + static_cast<size_t>(row) * p.n_splits * D;
+    constexpr int kPer = D / 32;
+    float M = -INFINITY;
+    for (int s = 0; s < n_valid; ++s) M = fmaxf(M, lp[s]);
+    float acc[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) acc[i] = 0.0f;
+    float Lsum = 0.0f;
+    for (int s = 0; s < n_valid; ++s) {
+        const float w = (lp[s] == -INFINITY) ? 0.0f : ex2_approx(lp[s] - M);
+        Lsum += w;
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) acc[i] += w * op[static_cast<size_t>(s) * D + lane * kPer + i];
+    }
+    const float inv = (Lsum > 0.0f) ? 1.0f / Lsum : 0.0f;
+    __nv_bfloat16* o = out + static_cast<size_t>(row) * D + lane * kPer;
+#pragma unroll
+    for (int i = 0; i < kPer; i += 2) {
+        const uint32_t v2 = pack_bf16x2(acc[i] * inv, acc[i + 1] * inv);
+        *reinterpret_cast<uint32_t*>(o + i) = v2;
+    }
+    if (lse != nullptr && lane == 0) lse[row] = (Lsum > 0.0f) ? (M + __log2f(Lsum)) * kLn2 : -INFINITY;
+}
+
+}  // namespace attn

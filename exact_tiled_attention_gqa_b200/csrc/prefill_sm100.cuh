@@ -1,0 +1,417 @@
+// prefill_sm100.cuh -- exact tiled GQA prefill on the sm_100a tensor cores.
+//
+// What it computes: O = softmax(scale * Q K^T + bottom-right causal mask) V
+// and LSE per row, for Q [B,Hq,Lq,D], K/V [B,Hkv,Lk,D] (bf16), exactly, with
+// an online softmax so the score table only ever exists one 128x128 tile at a
+// time in tensor memory.  Sources: the SDPA / FlashAttention selection guide
+// ("eager attention memory": tile the table, keep a max and a sum per row;
+// "is_causal mask alignment": bottom-right alignment, query i sees key j iff
+// j <= i + Lk - Lq; "long inputs": a block kernel skips fully masked blocks)
+// and the NVIDIA attention page ("Parameter one: group size": G query heads
+// share one KV head).
+//
+// Work unit (one CTA): one batch b, one KV head g, and 2*P consecutive query
+// positions, as two "Q tiles" of M = 128 rows.  A Q tile packs the G query
+// heads of the group with P = 128 / G positions each (row r = head r / P,
+// position p0 + r % P), so every K/V tile staged in shared memory feeds all
+// G heads of the group and both Q tiles.
+//
+// Roles (320 threads):
+//   warps 0-3  softmax warpgroup for Q tile 0 (thread = TMEM lane = row)
+//   warps 4-7  softmax warpgroup for Q tile 1
+//   warp  8    TMA producer: Q tiles once, then K_j, V_j into a ring of stages
+//   warp  9    TMEM allocator and single-thread tcgen05.mma issuer
+//
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D).
+// P_q (bf16, two per column) overwrites the first 64 columns of S_q once the
+// softmax has read S_q, and feeds O_q += P_q V_j as the TMEM A operand.
+//
+// Per key tile j the MMA thread issues, in order:
+//   O0 += P0(j) V_j ; S0(j+1) = Q0 K_{j+1}^T ; O1 += P1(j) V_j ; S1(j+1) = Q1 K_{j+1}^T
+// so the tensor cores work on one Q tile while the other's softmax runs.
+// A commit after S_q(j+1) also covers O_q += P_q(j) V_j, so when the softmax
+// sees S_q(j+1) its O_q is settled and may be rescaled in place.
+//
+// Online softmax, in the log2 domain (x2 = x * scale * log2 e): per row a
+// running max m and sum l.  The max used for the exponentials is only raised
+// when a tile's max exceeds it by more than kRescaleLog2 (= 8, a factor 256);
+// otherwise exponentials up to 2^8 are accumulated as they are.  The result
+// is the same exact quantity -- O = sum_j 2^(s2_j - m) v_j / sum_j 2^(s2_j - m)
+// holds for any m -- and the O rescale in TMEM is skipped on most tiles.
+#pragma once
+
+#include "ptx_sm100.cuh"
+#include "device_error.cuh"
+
+namespace attn {
+
+constexpr int kPrefillThreads = 320;
+constexpr int kBM = 128;               // rows per Q tile (MMA M)
+constexpr int kBN = 128;               // keys per K/V tile
+constexpr float kRescaleLog2 = 8.0f;
+
+template <int D>
+struct PrefillSmem {
+    static constexpr int kKB = D / 64;                    // 128-byte column blocks per row
+    static constexpr int kQTileBytes = kBM * D * 2;      // one Q tile
+    static constexpr int kKVTileBytes = kBN * D * 2;     // one K or V tile
+    static constexpr int kBlockBytes = 128 * 128;        // one 128-row x 128-byte block
+    static constexpr int kStages = (D == 128) ? 4 : 8;
+    static constexpr int kQOff = 0;
+    static constexpr int kKVOff = 2 * kQTileBytes;
+    static constexpr int kBarOff = kKVOff + kStages * kKVTileBytes;
+    // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2], drain
+    static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 1;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;   // tmem base (u32), abort flag (int)
+    static constexpr int kBytes = kMiscOff + 16;
+    static constexpr int kAlloc = kBytes + 1024;              // slack to align the base to 1 KiB
+};
+
+struct PrefillParams {
+    void* out;          // [B,Hq,Lq,D] bf16
+    float* lse;         // [B,Hq,Lq] or nullptr
+    int B, Hq, Hkv, Lq, Lk;
+    int G, P;           // group size, positions per Q tile (P = 128 / G)
+    int n_mblk;         // ceil(Lq / (2P))
+    int is_causal;
+    float scale_log2;   // scale * log2(e)
+};
+
+template <int D>
+__global__ void __maxnreg__(200)
+    attn_prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
+                              const __grid_constant__ CUtensorMap tm_k,
+                              const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
+    using L = PrefillSmem<D>;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_base = smem_u32(smem_raw);
+    const uint32_t base = (raw_base + 1023u) & ~1023u;
+    uint8_t* smem = smem_raw + (base - raw_base);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    // ---- work unit: heaviest (latest) position blocks first ----
+    const int bh_count = p.B * p.Hkv;
+    const int mblk = p.n_mblk - 1 - static_cast<int>(blockIdx.x) / bh_count;
+    const int bh = static_cast<int>(blockIdx.x) % bh_count;
+    const int b = bh / p.Hkv;
+    const int g = bh % p.Hkv;
+    const int P = p.P;
+    const int rows_used = p.G * P;
+    const int p_begin = mblk * 2 * P;
+    const long off = static_cast<long>(p.Lk) - static_cast<long>(p.Lq);
+    int n_kt;
+    {
+        const int p_last = min(p_begin + 2 * P, p.Lq) - 1;
+        const long last_key = p.is_causal ? min(static_cast<long>(p_last) + off, static_cast<long>(p.Lk) - 1)
+                                          : static_cast<long>(p.Lk) - 1;
+        n_kt = last_key < 0 ? 0 : static_cast<int>(last_key / kBN) + 1;
+    }
+
+    // ---- shared memory map ----
+    const uint32_t sQ = base + L::kQOff;
+    const uint32_t sKV = base + L::kKVOff;
+    const uint32_t bar0 = base + L::kBarOff;
+    const uint32_t bar_q_full = bar0;
+    auto bar_kv_full = [&](int s) { return bar0 + 8u * (1 + s); };
+    auto bar_kv_empty = [&](int s) { return bar0 + 8u * (1 + L::kStages + s); };
+    auto bar_s_full = [&](int q) { return bar0 + 8u * (1 + 2 * L::kStages + q); };
+    auto bar_p_full = [&](int q) { return bar0 + 8u * (3 + 2 * L::kStages + q); };
+    auto bar_o_done = [&](int q) { return bar0 + 8u * (5 + 2 * L::kStages + q); };
+    const uint32_t bar_drain = bar0 + 8u * (7 + 2 * L::kStages);
+    uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+
+    if (threadIdx.x == 0) {
+        mbar_init(bar_q_full, 1);
+        for (int s = 0; s < L::kStages; ++s) {
+            mbar_init(bar_kv_full(s), 1);
+            mbar_init(bar_kv_empty(s), 1);
+        }
+        for (int q = 0; q < 2; ++q) {
+            mbar_init(bar_s_full(q), 1);
+            mbar_init(bar_p_full(q), 128);
+            mbar_init(bar_o_done(q), 1);
+        }
+        mbar_init(bar_drain, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    // Q rows the TMA box does not cover (G does not divide 128) must hold
+    // finite values: zero them through the generic proxy, then hand them over.
+    if (rows_used < kBM) {
+        const int pad_bytes_per_block = (kBM - rows_used) * 128;
+        for (int q = 0; q < 2; ++q)
+            for (int kb = 0; kb < L::kKB; ++kb) {
+                uint8_t* blk = smem + L::kQOff + q * L::kQTileBytes + kb * L::kBlockBytes + rows_used * 128;
+                for (int i = threadIdx.x * 16; i < pad_bytes_per_block; i += kPrefillThreads * 16)
+                    *reinterpret_cast<uint4*>(blk + i) = make_uint4(0, 0, 0, 0);
+            }
+        fence_proxy_async_smem();
+    }
+    if (warp == 9) {
+        tmem_alloc(smem_u32(tmem_base_ptr), 512);
+        tmem_relinquish();
+    }
+    tc_fence_before_sync();
+    __syncthreads();
+    tc_fence_after_sync();
+    const uint32_t tmem = *tmem_base_ptr;
+
+    if (warp == 8) {
+        // ================= TMA producer =================
+        if (lane == 0 && n_kt > 0) {
+            tma_prefetch_desc(&tm_q);
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            const int q_head0 = b * p.Hq + g * p.G;
+            mbar_arrive_expect_tx(bar_q_full, 2u * L::kKB * rows_used * 128u);
+            for (int q = 0; q < 2; ++q)
+                for (int kb = 0; kb < L::kKB; ++kb)
+                    tma_load_3d(sQ + q * L::kQTileBytes + kb * L::kBlockBytes, &tm_q, bar_q_full, kb * 64,
+                                p_begin + q * P, q_head0);
+            const int kv_row = b * p.Hkv + g;
+            int issued = 0;
+            bool ok = true;
+            for (int t = 0; t < 2 * n_kt && ok; ++t) {
+                const int s = t % L::kStages;
+                const uint32_t round = static_cast<uint32_t>(t / L::kStages);
+                ok = mbar_wait(bar_kv_empty(s), (round & 1u) ^ 1u, abort_flag, &g_attn_err, kDevErrTimeout);
+                if (!ok) break;
+                mbar_arrive_expect_tx(bar_kv_full(s), L::kKVTileBytes);
+                const CUtensorMap* map = (t & 1) ? &tm_v : &tm_k;
+                const int j = t >> 1;
+                for (int kb = 0; kb < L::kKB; ++kb)
+                    tma_load_3d(sKV + s * L::kKVTileBytes + kb * L::kBlockBytes, map, bar_kv_full(s), kb * 64,
+                                j * kBN, kv_row);
+                issued = t + 1;
+            }
+            if (!ok) {
+                // Unwinding: let the copies already issued land before the CTA exits.
+                for (int t = max(0, issued - L::kStages); t < issued; ++t) {
+                    const int s = t % L::kStages;
+                    const uint64_t t0 = global_timer_ns();
+                    while (!mbar_try_wait(bar_kv_full(s), static_cast<uint32_t>(t / L::kStages) & 1u) &&
+                           global_timer_ns() - t0 < 100000000ull) {
+                    }
+                }
+                const uint64_t t0 = global_timer_ns();
+                while (!mbar_try_wait(bar_q_full, 0) && global_timer_ns() - t0 < 100000000ull) {
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 9) {
+        // ================= MMA issuer =================
+        if (lane == 0 && n_kt > 0) {
+            constexpr uint32_t kIdescQK = umma_idesc_bf16_f32(kBM, kBN, false);
+            constexpr uint32_t kIdescPV = umma_idesc_bf16_f32(kBM, D, true);
+            const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
+            const uint32_t tO[2] = {tmem + 256u, tmem + 256u + D};
+            auto slot_of = [&](int t) { return t % L::kStages; };
+            auto par_of = [&](int t) { return static_cast<uint32_t>(t / L::kStages) & 1u; };
+            // S_q = Q_q K^T : M=128, N=128, K=D in steps of 16 (32 bytes)
+            auto issue_qk = [&](int q, int t) {
+                const uint32_t a0 = sQ + q * L::kQTileBytes;
+                const uint32_t b0 = sKV + slot_of(t) * L::kKVTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t koff = (kk >> 2) * L::kBlockBytes + (kk & 3) * 32;
+                    umma_ss(tS[q], umma_sdesc_sw128(a0 + koff, 16, 1024), umma_sdesc_sw128(b0 + koff, 16, 1024),
+                            kIdescQK, kk > 0 ? 1u : 0u);
+                }
+            };
+            // O_q += P_q V : M=128, N=D, K=128 keys in steps of 16 (8 TMEM columns of P)
+            auto issue_pv = [&](int q, int t, bool acc) {
+                const uint32_t b0 = sKV + slot_of(t) * L::kKVTileBytes;
+#pragma unroll
+                for (int kk = 0; kk < kBN / 16; ++kk)
+                    umma_ts(tO[q], tS[q] + kk * 8, umma_sdesc_sw128(b0 + kk * 2048, L::kBlockBytes, 1024),
+                            kIdescPV, (acc || kk > 0) ? 1u : 0u);
+            };
+            bool ok = mbar_wait(bar_q_full, 0, abort_flag, &g_attn_err, kDevErrTimeout);
+            if (ok) ok = mbar_wait(bar_kv_full(slot_of(0)), par_of(0), abort_flag, &g_attn_err, kDevErrTimeout);
+            if (ok) {
+                tc_fence_after_sync();
+                issue_qk(0, 0);
+                umma_commit(bar_s_full(0));
+                issue_qk(1, 0);
+                umma_commit(bar_s_full(1));
+                umma_commit(bar_kv_empty(slot_of(0)));
+            }
+            for (int j = 0; j < n_kt && ok; ++j) {
+                const int tv = 2 * j + 1, tk = 2 * j + 2;
+                const bool last = (j + 1 == n_kt);
+                ok = mbar_wait(bar_kv_full(slot_of(tv)), par_of(tv), abort_flag, &g_attn_err, kDevErrTimeout) &&
+                     mbar_wait(bar_p_full(0), static_cast<uint32_t>(j) & 1u, abort_flag, &g_attn_err, kDevErrTimeout);
+                if (!ok) break;
+                tc_fence_after_sync();
+                issue_pv(0, tv, j > 0);
+                if (last) umma_commit(bar_o_done(0));
+                if (!last) {
+                    ok = mbar_wait(bar_kv_full(slot_of(tk)), par_of(tk), abort_flag, &g_attn_err, kDevErrTimeout);
+                    if (!ok) break;
+                    tc_fence_after_sync();
+                    issue_qk(0, tk);
+                    umma_commit(bar_s_full(0));
+                }
+                ok = mbar_wait(bar_p_full(1), static_cast<uint32_t>(j) & 1u, abort_flag, &g_attn_err, kDevErrTimeout);
+                if (!ok) break;
+                tc_fence_after_sync();
+                issue_pv(1, tv, j > 0);
+                if (last) umma_commit(bar_o_done(1));
+                umma_commit(bar_kv_empty(slot_of(tv)));
+                if (!last) {
+                    issue_qk(1, tk);
+                    umma_commit(bar_s_full(1));
+                    umma_commit(bar_kv_empty(slot_of(tk)));
+                }
+            }
+            // Drain: no MMA may still be running when TMEM is released.
+            umma_commit(bar_drain);
+            const uint64_t t0 = global_timer_ns();
+            while (!mbar_try_wait(bar_drain, 0) && global_timer_ns() - t0 < 100000000ull) {
+            }
+        }
+        __syncwarp();
+    } else {
+        // ================= softmax warpgroups =================
+        const int q = warp >> 2;                 // Q tile of this warpgroup
+        const int r = threadIdx.x & 127;         // row = TMEM lane
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t tS = tmem + (q ? 128u : 0u) + lane_off;
+        const uint32_t tO = tmem + 256u + (q ? static_cast<uint32_t>(D) : 0u) + lane_off;
+        const int head_local = r / P;
+        const int pos = p_begin + q * P + (r % P);
+        const bool row_valid = (r < rows_used) && (pos < p.Lq);
+        const int h = g * p.G + head_local;
+        // last visible key of this row, and the smallest such bound over the tile's rows
+        const long lk1 = static_cast<long>(p.Lk) - 1;
+        const long bound = p.is_causal ? min(static_cast<long>(pos) + off, lk1) : lk1;
+        const int tile_p0 = p_begin + q * P;
+        const long tile_min_bound = p.is_causal ? min(static_cast<long>(tile_p0) + off, lk1) : lk1;
+        const float sl2 = p.scale_log2;
+
+        float m_run = -INFINITY;   // running max used for the exponentials (log2 domain)
+        float l_run = 0.0f;        // running sum of exponentials
+        bool ok = true;
+        for (int j = 0; j < n_kt; ++j) {
+            ok = mbar_wait(bar_s_full(q), static_cast<uint32_t>(j) & 1u, abort_flag, &g_attn_err, kDevErrTimeout);
+            if (!ok) break;
+            tc_fence_after_sync();
+            uint32_t sr[128];
+            tmem_ld_32x32b_x32(tS + 0, sr + 0);
+            tmem_ld_32x32b_x32(tS + 32, sr + 32);
+            tmem_ld_32x32b_x32(tS + 64, sr + 64);
+            tmem_ld_32x32b_x32(tS + 96, sr + 96);
+            tmem_wait_ld();
+            reg_fence<128>(sr);
+            float s[kBN];
+#pragma unroll
+            for (int c = 0; c < kBN; ++c) s[c] = __uint_as_float(sr[c]);
+            const long key0 = static_cast<long>(j) * kBN;
+            if (key0 + kBN - 1 > tile_min_bound) {
+                // diagonal or ragged tile: mask keys beyond this row's bound
+#pragma unroll
+                for (int c = 0; c < kBN; ++c)
+                    if (key0 + c > bound) s[c] = -INFINITY;
+            }
+            float mx[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mx[i] = s[i];
+#pragma unroll
+            for (int c = 8; c < kBN; c += 8)
+#pragma unroll
+                for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[c + i]);
+            float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+            const float m_tile = tmax * sl2;   // -inf stays -inf
+            float factor = 1.0f;
+            if (m_tile > m_run + kRescaleLog2) {
+                factor = (m_run == -INFINITY) ? 0.0f : ex2_approx(m_run - m_tile);
+                m_run = m_tile;
+                l_run *= factor;
+            }
+            // rescale O_q in TMEM if any row of this warp raised its max (O holds
+            // the sum over tiles < j, settled: see the file comment)
+            if (j > 0 && __any_sync(0xffffffffu, factor != 1.0f)) {
+#pragma unroll 1
+                for (int c = 0; c < D; c += 32) {
+                    uint32_t orr[32];
+                    tmem_ld_32x32b_x32(tO + c, orr);
+                    tmem_wait_ld();
+                    reg_fence<32>(orr);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i)
+                        orr[i] = __float_as_uint(__uint_as_float(orr[i]) * factor);
+                    tmem_st_32x32b_x32(tO + c, orr);
+                }
+                tmem_wait_st();
+            }
+            const float m_sub = (m_run == -INFINITY) ? 0.0f : m_run;
+            float lsum[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) lsum[i] = 0.0f;
+            uint32_t pk[64];
+#pragma unroll
+            for (int c = 0; c < kBN; c += 2) {
+                const float e0 = ex2_approx(fmaf(s[c], sl2, -m_sub));
+                const float e1 = ex2_approx(fmaf(s[c + 1], sl2, -m_sub));
+                lsum[(c >> 1) & 7] += e0 + e1;
+                pk[c >> 1] = pack_bf16x2(e0, e1);
+            }
+            l_run += ((lsum[0] + lsum[1]) + (lsum[2] + lsum[3])) + ((lsum[4] + lsum[5]) + (lsum[6] + lsum[7]));
+            tmem_st_32x32b_x32(tS + 0, pk);
+            tmem_st_32x32b_x32(tS + 32, pk + 32);
+            tmem_wait_st();
+            tc_fence_before_sync();
+            mbar_arrive(bar_p_full(q));
+        }
+
+        // ---- epilogue: O / l -> bf16, LSE ----
+        bool have_o = ok && n_kt > 0;
+        if (have_o) {
+            have_o = mbar_wait(bar_o_done(q), 0, abort_flag, &g_attn_err, kDevErrTimeout);
+            tc_fence_after_sync();
+        }
+        const float inv_l = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
+        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) +
+                              ((static_cast<size_t>(b) * p.Hq + h) * p.Lq + (row_valid ? pos : 0)) * D;
+#pragma unroll 1
+        for (int c = 0; c < D; c += 32) {
+            uint32_t orr[32];
+            if (have_o) {
+                tmem_ld_32x32b_x32(tO + c, orr);
+                tmem_wait_ld();
+                reg_fence<32>(orr);
+            } else {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) orr[i] = 0u;
+            }
+            if (row_valid) {
+                uint32_t ob[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    ob[i] = pack_bf16x2(__uint_as_float(orr[2 * i]) * inv_l, __uint_as_float(orr[2 * i + 1]) * inv_l);
+                uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) dst[i] = make_uint4(ob[4 * i], ob[4 * i + 1], ob[4 * i + 2], ob[4 * i + 3]);
+            }
+        }
+        if (row_valid && p.lse != nullptr) {
+            const float lse = (l_run > 0.0f) ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
+            p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.Lq + pos] = lse;
+        }
+    }
+
+    // ---- teardown ----
+    tc_fence_before_sync();
+    __syncthreads();
+    if (warp == 9) {
+        tc_fence_after_sync();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace attn

@@ -1,0 +1,156 @@
+/*
+ * attn_gqa.h -- exact tiled grouped-query attention for NVIDIA B200 (sm_100a).
+ *
+ * The operation (both calls):
+ *
+ *   O = softmax(scale * Q K^T + mask) V
+ *
+ * computed exactly -- no approximation -- tile by tile with an online softmax
+ * that keeps only a running row maximum and row sum, so the Lq x Lk score
+ * table never reaches device memory.  This is the construction the page
+ * "어텐션 구현 고르기, SDPA·FlashAttention 메모리와 GPU 비용" (SDPA / FlashAttention
+ * selection guide) describes in its section on eager-attention memory: the
+ * score table is cut into on-chip blocks and only a max and a sum per row
+ * survive, memory grows linearly in length, and the result is the same as the
+ * eager computation up to the order of floating-point sums.
+ *
+ * Grouped-query heads: G = Hq / Hkv consecutive query heads share one key /
+ * value head; query head h reads KV head h / G.  G = 1 is multi-head and
+ * Hkv = 1 is multi-query attention (NVIDIA attention-optimisation page,
+ * "Parameter one: group size").
+ *
+ * Conventions shared by every call:
+ *   - Tensors are dense, row-major, and live in device memory owned by the
+ *     caller.  The library never frees or keeps a pointer after a call
+ *     returns (the kernels it launched may still be reading them: the
+ *     caller keeps them alive until `stream` has passed the work).
+ *   - bf16 tensors are passed as `const void*` / `void*` to 16-bit bfloat16
+ *     elements.  Base addresses must be 16-byte aligned.
+ *   - LSE is the natural-log log-sum-exp of the scaled, masked scores of a
+ *     row: LSE_i = m_i + ln(sum_j exp(scale * q_i.k_j - m_i)).  A row that
+ *     sees no key gets O = 0 and LSE = -inf.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *     call only enqueues work on it; none synchronises the host.
+ *   - Return value: ATTN_OK, or a negative attn_status_t.  Argument checks
+ *     happen before anything is enqueued, so a failed call has no effect.
+ *     attn_last_error() gives a one-line description of the last failure on
+ *     the calling thread.
+ */
+#ifndef ATTN_GQA_H
+#define ATTN_GQA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_INVALID_ARG = -1, /* null pointer, bad size, Hq % Hkv != 0, bad scale, misalignment */
+    ATTN_ERR_UNSUPPORTED = -2, /* valid but not built: D not in {64, 128}, group size too large */
+    ATTN_ERR_WORKSPACE = -3,   /* decode workspace missing or smaller than required */
+    ATTN_ERR_CUDA = -4         /* a CUDA runtime call or kernel launch failed */
+} attn_status_t;
+
+/*
+ * attn_prefill -- causal (or full) attention of Lq query rows against Lk keys.
+ *
+ * Defined by the SDPA / FlashAttention selection guide: the eager
+ * computation in "eager attention memory", its tiled equivalent in the same
+ * section, and the mask alignment of "is_causal mask alignment, the trap
+ * with a KV cache".  With is_causal != 0 the mask is aligned bottom-right:
+ * query row i (0-based) sees key j iff j <= i + (Lk - Lq).  For Lq == Lk this
+ * is the usual lower triangle; for Lq < Lk (a chunk of new tokens appended to
+ * Lk - Lq cached ones) the rows are the last Lq positions of the sequence.
+ * With is_causal == 0 every row sees all Lk keys.
+ *
+ *   q    [B, Hq,  Lq, D]  bf16, read
+ *   k    [B, Hkv, Lk, D]  bf16, read
+ *   v    [B, Hkv, Lk, D]  bf16, read
+ *   out  [B, Hq,  Lq, D]  bf16, written
+ *   lse  [B, Hq,  Lq]     fp32, written; may be NULL (not written)
+ *   scale: finite and > 0 (usually 1/sqrt(D))
+ *   D: 64 or 128.  G = Hq / Hkv: 1 .. 128.
+ *   B == 0 or Lq == 0: nothing to do, returns ATTN_OK.
+ *   Lk == 0: every row sees no key (O = 0, LSE = -inf).
+ *
+ * Errors: ATTN_ERR_INVALID_ARG for null q/k/v/out, negative sizes, Hq or
+ * Hkv < 1, Hq % Hkv != 0, non-finite or non-positive scale, or a base
+ * address not 16-byte aligned; ATTN_ERR_UNSUPPORTED for D outside {64, 128}
+ * or G > 128; ATTN_ERR_CUDA when a launch fails.
+ */
+int attn_prefill(const void* q, const void* k, const void* v, void* out, float* lse,
+                 int B, int Hq, int Hkv, int Lq, int Lk, int D, float scale, int is_causal,
+                 void* stream);
+
+/*
+ * attn_decode_workspace_size -- bytes of scratch attn_decode needs for these
+ * sizes (split-KV partial outputs and their log-sum-exps).  Depends only on
+ * the arguments.  Returns 0 for sizes attn_decode would reject.
+ */
+size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int D);
+
+/*
+ * attn_decode -- one new query token per sequence against a KV cache.
+ *
+ * Defined by the same guide's "use_cache" section and the is_causal section:
+ * cached keys and values of earlier tokens do not change, and the single new
+ * query row sees every cached key, so no mask is needed.  Sequence b has
+ * seqlens[b] valid cache rows, 0 .. seqlens[b]-1; rows at or beyond
+ * seqlens[b] are never used (they may hold anything, NaN included).
+ *
+ * The cache is split along its length; each piece is reduced with its own
+ * online softmax and the pieces are merged by their log-sum-exps (the
+ * single-GPU form of the KV parallelism on the NVIDIA attention page,
+ * "Parameter four: parallelism").
+ *
+ *   q        [B, Hq, D]          bf16, read
+ *   k_cache  [B, Hkv, Lmax, D]   bf16, read
+ *   v_cache  [B, Hkv, Lmax, D]   bf16, read
+ *   seqlens  [B]                 int32 in device memory, each in [0, Lmax];
+ *                                a value outside is clamped into range and
+ *                                flags ATTN_DEVERR_SEQLEN (attn_device_error)
+ *   out      [B, Hq, D]          bf16, written
+ *   lse      [B, Hq]             fp32, written; may be NULL
+ *   workspace: device memory of at least attn_decode_workspace_size(...)
+ *              bytes, 256-byte aligned, owned by the caller; its contents on
+ *              entry do not matter and on return are unspecified.  Two calls
+ *              in flight at once must not share one workspace.
+ *   D: 64 or 128.  G = Hq / Hkv: 1 .. 64.  B == 0 returns ATTN_OK.
+ *
+ * Errors: as attn_prefill, plus ATTN_ERR_WORKSPACE for a null or too small
+ * workspace.
+ */
+int attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,
+                void* out, float* lse, int B, int Hq, int Hkv, int Lmax, int D, float scale,
+                void* workspace, size_t workspace_bytes, void* stream);
+
+/* attn_status_string -- a static name for a status code; never NULL. */
+const char* attn_status_string(int status);
+
+/* attn_last_error -- description of the last failure on this host thread
+ * ("" if none).  The string stays valid until the thread's next call. */
+const char* attn_last_error(void);
+
+/*
+ * Device-side error word.  Kernels never trap: a wait that runs out of time
+ * (a pipeline barrier that never completes) or an out-of-range seqlens value
+ * sets a bit here and the kernel returns early.
+ */
+#define ATTN_DEVERR_TIMEOUT 0x1u  /* a pipeline wait gave up after ~2 s */
+#define ATTN_DEVERR_SEQLEN  0x2u  /* a seqlens value was outside [0, Lmax] */
+
+/*
+ * attn_device_error -- synchronise the current device, copy its error word
+ * into *flags and, if reset != 0, clear it.  Diagnostic call, not for the hot
+ * path.  Returns ATTN_OK or ATTN_ERR_CUDA / ATTN_ERR_INVALID_ARG.
+ */
+int attn_device_error(unsigned int* flags, int reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_GQA_H */

@@ -1,0 +1,115 @@
+"""The C ABI: every symbol the header declares is exported, and argument checks
+fail cleanly before anything reaches a GPU (these calls never launch work)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_tiled_attention_gqa_b200 import _native
+from exact_tiled_attention_gqa_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "attn_gqa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return _native.lib()
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(attn_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_calls():
+    assert declared_symbols() == sorted(_native.SIGNATURES)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_symbols():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    assert lib.attn_status_string(0) == b"ATTN_OK"
+    assert lib.attn_status_string(-1) == b"ATTN_ERR_INVALID_ARG"
+    assert lib.attn_status_string(-2) == b"ATTN_ERR_UNSUPPORTED"
+    assert lib.attn_status_string(-3) == b"ATTN_ERR_WORKSPACE"
+    assert lib.attn_status_string(-4) == b"ATTN_ERR_CUDA"
+    assert lib.attn_status_string(7) == b"ATTN_ERR_UNKNOWN"
+
+
+# fake, aligned addresses: only ever passed together with an invalid argument,
+# so the call returns before touching CUDA
+A = ctypes.c_void_p(0x10000)
+NULL = None
+
+
+def _prefill(lib, **kw):
+    args = dict(q=A, k=A, v=A, out=A, lse=NULL, B=1, Hq=8, Hkv=2, Lq=16, Lk=16, D=128, scale=0.1, causal=1)
+    args.update(kw)
+    return lib.attn_prefill(args["q"], args["k"], args["v"], args["out"], args["lse"], args["B"], args["Hq"],
+                            args["Hkv"], args["Lq"], args["Lk"], args["D"], args["scale"], args["causal"], None)
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(q=NULL), -1), (dict(out=NULL), -1), (dict(B=-1), -1), (dict(Lq=-3), -1), (dict(Lk=-1), -1),
+    (dict(Hq=0), -1), (dict(Hkv=0), -1), (dict(Hq=6, Hkv=4), -1), (dict(scale=0.0), -1),
+    (dict(scale=-1.0), -1), (dict(scale=float("nan")), -1), (dict(scale=float("inf")), -1),
+    (dict(q=ctypes.c_void_p(0x10008)), -1), (dict(lse=ctypes.c_void_p(0x10002)), -1),
+    (dict(D=96), -2), (dict(D=256), -2), (dict(Hq=256, Hkv=1), -2),
+])
+def test_prefill_rejects(lib, bad, code):
+    assert _prefill(lib, **bad) == code
+    assert lib.attn_last_error() != b""
+
+
+def test_prefill_empty_is_noop(lib):
+    assert _prefill(lib, B=0) == 0
+    assert _prefill(lib, Lq=0) == 0
+
+
+def _decode(lib, **kw):
+    args = dict(q=A, k=A, v=A, sl=A, out=A, lse=NULL, B=2, Hq=8, Hkv=2, Lmax=64, D=128, scale=0.1, ws=A,
+                wsb=1 << 30)
+    args.update(kw)
+    return lib.attn_decode(args["q"], args["k"], args["v"], args["sl"], args["out"], args["lse"], args["B"],
+                           args["Hq"], args["Hkv"], args["Lmax"], args["D"], args["scale"], args["ws"],
+                           args["wsb"], None)
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(sl=NULL), -1), (dict(sl=ctypes.c_void_p(0x10001)), -1), (dict(Lmax=0), -1), (dict(Hq=5, Hkv=2), -1),
+    (dict(k=NULL), -1), (dict(D=32), -2), (dict(Hq=128, Hkv=1), -2), (dict(ws=NULL), -3), (dict(wsb=16), -3),
+    (dict(ws=ctypes.c_void_p(0x10010)), -1),
+])
+def test_decode_rejects(lib, bad, code):
+    assert _decode(lib, **bad) == code
+
+
+def test_decode_empty_batch_is_noop(lib):
+    assert _decode(lib, B=0) == 0
+
+
+def test_workspace_size(lib):
+    f = lib.attn_decode_workspace_size
+    assert f(0, 8, 2, 64, 128) == 0
+    assert f(2, 8, 3, 64, 128) == 0        # Hq % Hkv
+    assert f(2, 8, 2, 64, 96) == 0         # D
+    assert f(2, 8, 2, 0, 128) == 0         # Lmax
+    assert f(1, 128, 1, 64, 128) == 0      # G > 64
+    a = f(2, 8, 2, 1000, 128)
+    assert a > 0 and a % 256 == 0
+    assert f(2, 8, 2, 100000, 128) >= a
+    # big enough for one fp32 partial row per split plus its lse
+    assert f(64, 32, 8, 32768, 128) >= 64 * 32 * (128 + 1) * 4
+
+
+def test_missing_library_raises(monkeypatch, tmp_path):
+    monkeypatch.setattr(_native, "_lib", None)
+    monkeypatch.setattr(_native, "LIB_PATH", str(tmp_path / "absent.so"))
+    with pytest.raises(RuntimeError, match="no fallback"):
+        _native.lib()

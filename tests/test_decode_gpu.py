@@ -1,0 +1,110 @@
+"""GPU parity for attn_decode (through the C ABI) against the fp64 oracle.
+
+Cache rows at or beyond seqlens[b] are filled with NaN to show they are never
+used.  Full-size workloads compare sampled (batch, head) rows.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from exact_tiled_attention_gqa_b200 import decode, device_error
+from exact_tiled_attention_gqa_b200 import workloads as W
+from parity import assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    device_error(reset=True)
+    yield
+    assert device_error(reset=True) == 0
+
+
+def _inputs(B, Hq, Hkv, Lmax, D, seqlens, seed):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(B, Hq, D, generator=g).to(torch.bfloat16)
+    k = torch.randn(B, Hkv, Lmax, D, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, Hkv, Lmax, D, generator=g).to(torch.bfloat16)
+    sl = torch.tensor(seqlens, dtype=torch.int32)
+    for b, n in enumerate(seqlens):
+        k[b, :, n:] = float("nan")
+        v[b, :, n:] = float("nan")
+    return q, k, v, sl
+
+
+def _check(oracle_mod, q, k, v, sl, what):
+    D = q.shape[-1]
+    out, lse = decode(q.cuda(), k.cuda(), v.cuda(), sl.cuda(), scale=1 / math.sqrt(D))
+    torch.cuda.synchronize()
+    assert device_error(reset=True) == 0
+    ref_o, ref_l = oracle_mod.attention_decode(q, k, v, sl, 1 / math.sqrt(D))
+    return assert_close(out, lse, ref_o, ref_l, what)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("G", [1, 2, 4, 8, 16, 32, 64, 3, 12, 24, 48])
+def test_group_sizes(oracle_mod, D, G):
+    Hkv = 2
+    seqlens = [700, 1, 333, 64, 65]
+    q, k, v, sl = _inputs(len(seqlens), G * Hkv, Hkv, 700, D, seqlens, seed=G * 10 + D)
+    _check(oracle_mod, q, k, v, sl, f"G{G} D{D}")
+
+
+@pytest.mark.parametrize("Lmax,seqlens", [(5000, [5000, 4097, 4096, 4095, 1, 2500]), (64, [64, 63]),
+                                          (1, [1, 1]), (9000, [0, 9000])])
+def test_split_edges(oracle_mod, Lmax, seqlens):
+    q, k, v, sl = _inputs(len(seqlens), 8, 2, Lmax, 128, seqlens, seed=Lmax)
+    _check(oracle_mod, q, k, v, sl, f"Lmax{Lmax}")
+
+
+def test_zero_length_sequence(oracle_mod):
+    q, k, v, sl = _inputs(2, 4, 1, 100, 128, [0, 50], seed=1)
+    out, lse = decode(q.cuda(), k.cuda(), v.cuda(), sl.cuda())
+    torch.cuda.synchronize()
+    assert torch.all(out[0] == 0) and torch.all(torch.isneginf(lse[0]))
+
+
+def test_decode_matches_prefill_last_row(oracle_mod):
+    from exact_tiled_attention_gqa_b200 import prefill
+    B, Hq, Hkv, L, D = 2, 8, 2, 400, 128
+    q, k, v = (t.cuda() for t in W.prefill_inputs(B, Hq, Hkv, L, L, D, seed=9))
+    po, pl = prefill(q, k, v, is_causal=True)
+    do, dl = decode(q[:, :, -1].contiguous(), k, v, torch.full((B,), L, dtype=torch.int32, device="cuda"))
+    torch.cuda.synchronize()
+    assert (po[:, :, -1].float() - do.float()).abs().max().item() <= 2e-2
+    assert (pl[:, :, -1] - dl).abs().max().item() <= 1e-3
+
+
+def _sampled_check(oracle_mod, shape, seed, n_pairs, fill_nan):
+    q, k, v, sl = W.decode_inputs_for(shape, seed=seed, device="cuda", fill_beyond=float("nan") if fill_nan else None)
+    out, lse = decode(q, k, v, sl)
+    torch.cuda.synchronize()
+    assert device_error(reset=True) == 0
+    rng = np.random.default_rng(seed)
+    G = shape.G
+    pairs = [(0, 0), (shape.B - 1, shape.Hq - 1)] + [
+        (int(rng.integers(shape.B)), int(rng.integers(shape.Hq))) for _ in range(n_pairs)]
+    for b, h in pairs:
+        g = h // G
+        n = int(sl[b])
+        qb = q[b:b + 1, h:h + 1].cpu()
+        kb = k[b:b + 1, g:g + 1, :n].cpu()
+        vb = v[b:b + 1, g:g + 1, :n].cpu()
+        ref_o, ref_l = oracle_mod.attention_decode(qb, kb, vb, np.array([n], np.int32), shape.scale)
+        assert_close(out[b:b + 1, h:h + 1], lse[b:b + 1, h:h + 1], ref_o, ref_l, f"{shape.name} b{b} h{h}")
+
+
+@pytest.mark.slow
+def test_qwen_decode_full_size_sampled(oracle_mod):
+    _sampled_check(oracle_mod, W.QWEN_DECODE, seed=0, n_pairs=24, fill_nan=True)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("G", W.GROUP_SWEEP)
+def test_group_sweep_full_size_sampled(oracle_mod, G):
+    _sampled_check(oracle_mod, W.group_sweep_decode(G), seed=G, n_pairs=6, fill_nan=False)

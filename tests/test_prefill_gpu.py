@@ -1,0 +1,115 @@
+"""GPU parity for attn_prefill (through the C ABI) against the fp64 oracle.
+
+Small cases compare every output; the full-size Qwen3-8B-shaped and chunked
+workloads compare sampled query rows (all heads) that the oracle computes one
+by one: first and last rows, tile edges, and rows right after spiked keys.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from exact_tiled_attention_gqa_b200 import device_error, prefill
+from exact_tiled_attention_gqa_b200 import workloads as W
+from parity import assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    device_error(reset=True)
+    yield
+    assert device_error(reset=True) == 0
+
+
+def _run(oracle_mod, B, Hq, Hkv, Lq, Lk, D, causal, seed=0, spike=0, rows=None):
+    q, k, v = W.prefill_inputs(B, Hq, Hkv, Lq, Lk, D, seed=seed, spike_every=spike)
+    scale = 1.0 / math.sqrt(D)
+    out, lse = prefill(q.cuda(), k.cuda(), v.cuda(), scale=scale, is_causal=causal)
+    torch.cuda.synchronize()
+    ref_o, ref_l = oracle_mod.attention_prefill(q, k, v, scale, causal, rows=rows)
+    if rows is not None:
+        out, lse = out[:, :, rows], lse[:, :, rows]
+    assert device_error(reset=True) == 0
+    return assert_close(out, lse, ref_o, ref_l, f"B{B} Hq{Hq} Hkv{Hkv} Lq{Lq} Lk{Lk} D{D} causal{causal}")
+
+
+def test_tiny_config(oracle_mod):
+    s = W.TINY_PREFILL
+    _run(oracle_mod, s.B, s.Hq, s.Hkv, s.Lq, s.Lk, s.D, True)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (8, 4), (8, 2), (16, 2), (6, 2), (32, 1), (5, 5)])
+def test_ragged_multi_tile(oracle_mod, D, causal, Hq, Hkv):
+    _run(oracle_mod, 2, Hq, Hkv, 300, 300, D, causal, seed=Hq * 7 + Hkv)
+
+
+@pytest.mark.parametrize("Lq,Lk", [(77, 500), (1, 500), (2, 257), (128, 640), (250, 129), (129, 128), (1, 1),
+                                   (3, 1), (200, 130), (513, 513)])
+def test_chunked_bottom_right(oracle_mod, Lq, Lk):
+    _run(oracle_mod, 1, 8, 2, Lq, Lk, 128, True, seed=Lq + Lk, spike=97)
+
+
+def test_group_of_128_and_64(oracle_mod):
+    _run(oracle_mod, 1, 128, 1, 40, 300, 128, True, seed=5)
+    _run(oracle_mod, 1, 64, 1, 70, 200, 64, True, seed=6)
+
+
+def test_no_keys_and_empty(oracle_mod):
+    q = torch.randn(1, 4, 5, 128).to(torch.bfloat16).cuda()
+    e = torch.empty(1, 2, 0, 128, dtype=torch.bfloat16, device="cuda")
+    out, lse = prefill(q, e, e, is_causal=True)
+    torch.cuda.synchronize()
+    assert torch.all(out == 0) and torch.all(torch.isneginf(lse))
+    q0 = torch.empty(1, 4, 0, 128, dtype=torch.bfloat16, device="cuda")
+    k = torch.randn(1, 2, 9, 128).to(torch.bfloat16).cuda()
+    out0, lse0 = prefill(q0, k, k)
+    assert out0.numel() == 0 and lse0.numel() == 0
+
+
+def test_large_scores_stay_finite(oracle_mod):
+    """Scores in the hundreds (inputs scaled by 8 and 4): the online max keeps exponentials bounded."""
+    q, k, v = W.prefill_inputs(1, 8, 2, 256, 256, 128, seed=11)
+    q, k = q * 8, k * 4
+    out, lse = prefill(q.cuda(), k.cuda(), v.cuda(), scale=1 / math.sqrt(128), is_causal=True)
+    torch.cuda.synchronize()
+    ref_o, ref_l = oracle_mod.attention_prefill(q, k, v, 1 / math.sqrt(128), True)
+    assert_close(out, lse, ref_o, ref_l, "large scores")
+
+
+def test_deterministic(oracle_mod):
+    q, k, v = (t.cuda() for t in W.prefill_inputs(2, 8, 2, 333, 333, 128, seed=3))
+    a, la = prefill(q, k, v)
+    b, lb = prefill(q, k, v)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b) and torch.equal(la, lb)
+
+
+def _sample_rows(Lq, extra=()):
+    rows = {0, 1, 2, Lq - 1, Lq - 2, Lq // 2}
+    for e in (31, 32, 33, 63, 64, 65, 127, 128, 129, 255, 256, 257):
+        for base in (0, Lq // 2 - Lq // 2 % 256, Lq - 300):
+            if 0 <= base + e < Lq:
+                rows.add(base + e)
+    rows.update(r for r in extra if 0 <= r < Lq)
+    return sorted(rows)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("shape", [W.QWEN_PREFILL_4K, W.QWEN_PREFILL_8K_B4, W.CHUNKED_16K, W.CHUNKED_32K],
+                         ids=lambda s: s.name)
+def test_full_size_sampled_rows(oracle_mod, shape):
+    off = shape.Lk - shape.Lq
+    # rows right after spiked keys (every 97th key), seen through the bottom-right offset
+    spikes = [j - off + d for j in range(0, shape.Lk, 97 * 16) for d in (0, 1)] if shape.spike_every else []
+    rows = _sample_rows(shape.Lq, spikes)
+    if shape.B > 1:
+        rows = rows[:48]
+    _run(oracle_mod, shape.B, shape.Hq, shape.Hkv, shape.Lq, shape.Lk, shape.D, shape.is_causal, seed=0,
+         spike=shape.spike_every, rows=rows)
