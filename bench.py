@@ -29,7 +29,6 @@ import json
 import math
 import os
 import statistics
-import subprocess
 import sys
 import threading
 import time
@@ -51,13 +50,17 @@ DECODE = W.QWEN_DECODE
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU seconds per oracle sample")
     ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--only", choices=["prefill", "decode"], default=None,
+                    help="profiling aid: time one call type only (the JSON line is then partial)")
+    ap.add_argument("--decode-batch", type=int, default=None,
+                    help="profiling aid: use the first N sequences of the decode batch")
     return ap.parse_args()
 
 
@@ -65,70 +68,66 @@ def parse():
 # clocks sampled during the timed region
 # --------------------------------------------------------------------------
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Polls SM clock, power and throttle reasons through NVML every ~10 ms
+    while the timed region runs (nvidia-smi's 100 ms loop is the fallback)."""
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, gpu_index: str):
-        self.gpu_index = gpu_index
-        self.proc = None
-        self.lines = []
+    def __init__(self, torch_device_index: int):
+        self.dev_index = torch_device_index
+        self.samples = []          # (sm_mhz, max_mhz, power_w, reason_bits)
+        self._stop = threading.Event()
         self.thread = None
+        self.nvml = None
+        self.handle = None
+        self.error = None
+
+    def _open(self):
+        import pynvml
+        pynvml.nvmlInit()
+        uuid = str(torch.cuda.get_device_properties(self.dev_index).uuid)
+        uuid = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        self.handle = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode())
+        self.nvml = pynvml
 
     def start(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu_index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except (OSError, ValueError):
-            self.proc = None
+            self._open()
+        except Exception as e:   # NVML missing or the UUID lookup failed
+            self.error = f"nvml unavailable: {e}"
             return
-        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread = threading.Thread(target=self._poll, daemon=True)
         self.thread.start()
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _poll(self):
+        n, h = self.nvml, self.handle
+        while not self._stop.is_set():
+            try:
+                sm = n.nvmlDeviceGetClockInfo(h, n.NVML_CLOCK_SM)
+                mx = n.nvmlDeviceGetMaxClockInfo(h, n.NVML_CLOCK_SM)
+                pw = n.nvmlDeviceGetPowerUsage(h) / 1000.0
+                rs = n.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((float(sm), float(mx), pw, int(rs)))
+            except Exception as e:
+                self.error = str(e)
+                return
+            time.sleep(0.01)
 
     def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except subprocess.TimeoutExpired:
-            self.proc.kill()
-        self.thread.join(timeout=5)
-        sm, smax, power, reasons = [], [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
-                power.append(float(parts[3]))
-            except ValueError:
-                continue
-            for name, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
+        self._stop.set()
+        if self.thread is not None:
+            self.thread.join(timeout=5)
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [self.error or "no samples"], "samples": 0}
+        reasons = set()
+        for *_, bits in self.samples:
+            for bit, name in self.REASONS.items():
+                if bits & bit:
                     reasons.add(name)
-        loaded = [s for s, p in zip(sm, power) if p > 300.0] or sm
-        return {"sm_mhz": statistics.median(loaded) if loaded else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm),
-                "power_w_max": max(power) if power else None}
-
-
-def physical_gpu_id(local_rank: int) -> str:
-    """nvidia-smi's id for this process's GPU (CUDA_VISIBLE_DEVICES may remap ordinals)."""
-    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").strip()
-    if vis:
-        ids = [x.strip() for x in vis.split(",") if x.strip()]
-        if local_rank < len(ids):
-            return ids[local_rank]
-    return str(local_rank)
+        loaded = [s[0] for s in self.samples if s[2] > 300.0] or [s[0] for s in self.samples]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(s[1] for s in self.samples),
+                "reasons": sorted(reasons), "samples": len(self.samples),
+                "power_w_max": round(max(s[2] for s in self.samples), 1)}
 
 
 # --------------------------------------------------------------------------
@@ -149,23 +148,45 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- inputs (per rank: its own sequences; seeds differ by rank) ----
     seed = args.seed + 1000 * rank
-    q_h, k_h, v_h = W.prefill_inputs_for(PREFILL, seed=seed, device="cpu")
-    q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
-    dq, dk, dv, dsl = W.decode_inputs_for(DECODE, seed=seed, device=dev)
+    if args.only != "decode":
+        q_h, k_h, v_h = W.prefill_inputs_for(PREFILL, seed=seed, device="cpu")
+        q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    if args.only == "prefill":
+        dshape = W.DecodeShape(DECODE.name, 1, DECODE.Hq, DECODE.Hkv, 64, DECODE.D, 64, 64)
+    elif args.decode_batch:
+        dshape = W.DecodeShape(DECODE.name + f" (first {args.decode_batch})", args.decode_batch, DECODE.Hq,
+                               DECODE.Hkv, DECODE.Lmax, DECODE.D, DECODE.seqlen_lo, DECODE.seqlen_hi)
+    else:
+        dshape = DECODE
+    if args.only == "decode":
+        q_h, k_h, v_h = W.prefill_inputs(1, PREFILL.Hq, PREFILL.Hkv, 128, 128, PREFILL.D, seed=seed)
+        q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
+    dq, dk, dv, dsl = W.decode_inputs_for(dshape, seed=seed, device=dev)
     seqlens_host = dsl.cpu()
     p_flops = RL.prefill_flops(PREFILL.B, PREFILL.Hq, PREFILL.Lq, PREFILL.Lk, PREFILL.D, PREFILL.is_causal)
-    d_bytes = RL.decode_bytes(seqlens_host.tolist(), DECODE.B, DECODE.Hq, DECODE.Hkv, DECODE.D)
+    d_bytes = RL.decode_bytes(seqlens_host.tolist(), dshape.B, dshape.Hq, dshape.Hkv, dshape.D)
     p_out = torch.empty_like(q)
     p_lse = torch.empty((PREFILL.B, PREFILL.Hq, PREFILL.Lq), dtype=torch.float32, device=dev)
     d_out = torch.empty_like(dq)
-    d_lse = torch.empty((DECODE.B, DECODE.Hq), dtype=torch.float32, device=dev)
-    ws = torch.empty(attn.decode_workspace_size(DECODE.B, DECODE.Hq, DECODE.Hkv, DECODE.Lmax, DECODE.D),
+    d_lse = torch.empty((dshape.B, dshape.Hq), dtype=torch.float32, device=dev)
+    ws = torch.empty(attn.decode_workspace_size(dshape.B, dshape.Hq, dshape.Hkv, dshape.Lmax, dshape.D),
                      dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    do_pre = args.only in (None, "prefill")
+    do_dec = args.only in (None, "decode")
+
+    def call_prefill():
+        if do_pre:
+            attn.prefill(q, k, v, is_causal=True, out=p_out, lse=p_lse, stream=stream)
+
+    def call_decode():
+        if do_dec:
+            attn.decode(dq, dk, dv, dsl, out=d_out, lse=d_lse, workspace=ws, stream=stream)
+
     def step():
-        attn.prefill(q, k, v, is_causal=True, out=p_out, lse=p_lse, stream=stream)
-        attn.decode(dq, dk, dv, dsl, out=d_out, lse=d_lse, workspace=ws, stream=stream)
+        call_prefill()
+        call_decode()
 
     def barrier():
         if dist is not None:
@@ -178,7 +199,7 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- timed region: K steps, events around each call on the launching stream ----
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    sampler = ClockSampler(physical_gpu_id(local_rank))
+    sampler = ClockSampler(local_rank)
     barrier()
     torch.cuda.synchronize()
     sampler.start()
@@ -188,9 +209,9 @@ def run_ours(args, rank, world, local_rank):
     t_start.record(stream)
     for i in range(args.steps):
         ev[i][0].record(stream)
-        attn.prefill(q, k, v, is_causal=True, out=p_out, lse=p_lse, stream=stream)
+        call_prefill()
         ev[i][1].record(stream)
-        attn.decode(dq, dk, dv, dsl, out=d_out, lse=d_lse, workspace=ws, stream=stream)
+        call_decode()
         ev[i][2].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize()
@@ -219,7 +240,7 @@ def run_ours(args, rank, world, local_rank):
     ho, hl = torch.empty_like(hq).pin_memory(), torch.empty(p_lse.shape, dtype=torch.float32).pin_memory()
     hdo, hdl = torch.empty_like(hdq).pin_memory(), torch.empty(d_lse.shape, dtype=torch.float32).pin_memory()
     e2e_pre, e2e_dec = [], []
-    for i in range(args.e2e_steps + 1):
+    for i in range(args.e2e_steps + 1 if args.only is None else 0):
         e = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
         e[0].record(stream)
         q.copy_(hq, non_blocking=True)
@@ -238,8 +259,13 @@ def run_ours(args, rank, world, local_rank):
         if i > 0:   # the first is a warm-up of the copy path
             e2e_pre.append(e[0].elapsed_time(e[1]))
             e2e_dec.append(e[1].elapsed_time(e[2]))
-    e2e_pre_ms = max_over_ranks(sum(e2e_pre) / len(e2e_pre))
-    e2e_dec_ms = max_over_ranks(sum(e2e_dec) / len(e2e_dec))
+    e2e_pre_ms = max_over_ranks(sum(e2e_pre) / max(1, len(e2e_pre)))
+    e2e_dec_ms = max_over_ranks(sum(e2e_dec) / max(1, len(e2e_dec)))
+    if args.only is not None:
+        print(json.dumps({"only": args.only, "prefill_ms": pre_avg, "decode_ms": dec_avg,
+                          "prefill_tflops": p_flops / (pre_avg * 1e-3) / 1e12 if do_pre else None,
+                          "decode_gbs": d_bytes / (dec_avg * 1e-3) / 1e9 if do_dec else None}), flush=True)
+        return None
     h2d = (hq.numel() + hk.numel() + hv.numel() + hdq.numel()) * 2
     d2h = (ho.numel() + hdo.numel()) * 2 + (hl.numel() + hdl.numel()) * 4
 

@@ -9,6 +9,7 @@ from __future__ import annotations
 
 import glob
 import os
+import re
 import shutil
 import subprocess
 import sys
@@ -40,13 +41,53 @@ def up_to_date() -> bool:
     return all(os.path.getmtime(s) <= t for s in sources())
 
 
+# The prefill kernel launches with this many registers per thread and then
+# moves registers between its warpgroups with setmaxnreg; the exchange only
+# balances if the compiled count is exactly this (see prefill_sm100.cuh).
+PREFILL_LAUNCH_REGS = 168
+
+
+def check_ptxas_report(report: str) -> dict:
+    """Parse `-Xptxas -v` output: {kernel: (registers, spill_bytes)}; enforce the prefill register count."""
+    kernels, current = {}, None
+    for line in report.splitlines():
+        m = re.search(r"Compiling entry function '([^']+)'", line)
+        if m:
+            current = m.group(1)
+            continue
+        m = re.search(r"(\d+) bytes spill stores", line)
+        if m and current:
+            kernels.setdefault(current, [0, 0])[1] = int(m.group(1))
+        m = re.search(r"Used (\d+) registers", line)
+        if m and current:
+            kernels.setdefault(current, [0, 0])[0] = int(m.group(1))
+    prefill = {k: v for k, v in kernels.items() if "attn_prefill_sm100_kernel" in k}
+    if not prefill:
+        raise RuntimeError("ptxas report has no prefill kernel entry")
+    for name, (regs, _) in prefill.items():
+        if regs != PREFILL_LAUNCH_REGS:
+            raise RuntimeError(f"{name} compiled to {regs} registers, expected exactly {PREFILL_LAUNCH_REGS}: "
+                               "the setmaxnreg exchange would not balance")
+    return {k: tuple(v) for k, v in kernels.items()}
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
     if not force and up_to_date():
         return LIB_PATH
     tmp = LIB_PATH + f".tmp{os.getpid()}"
     cmd = [_nvcc(), "-std=c++17", "-O3", "-lineinfo", *ARCH_FLAGS, "-Xcompiler", "-fPIC", "-shared",
-           "-Xptxas", "-v" if verbose else "-O3", os.path.join(CSRC, "attn_gqa.cu"), "-o", tmp]
-    subprocess.run(cmd, check=True)
+           "-Xptxas", "-v", os.path.join(CSRC, "attn_gqa.cu"), "-o", tmp]
+    res = subprocess.run(cmd, capture_output=True, text=True)
+    if res.returncode != 0:
+        raise RuntimeError(f"nvcc failed:\n{res.stdout}\n{res.stderr}")
+    try:
+        kernels = check_ptxas_report(res.stdout + res.stderr)
+    except RuntimeError:
+        os.remove(tmp)
+        raise
+    if verbose:
+        for name, (regs, spill) in sorted(kernels.items()):
+            print(f"{regs:4d} regs {spill:6d} B spill  {name}")
     os.replace(tmp, LIB_PATH)
     return LIB_PATH
 

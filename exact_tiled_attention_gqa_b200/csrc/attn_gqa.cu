@@ -205,9 +205,13 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
     return check_launch("attn_decode_combine_kernel");
 }
 
+// q/out may be null only when they are empty (B == 0 or L1 == 0); k/v only when
+// they are empty (B == 0 or L2 == 0) -- an empty tensor has no storage.
 int check_common(const void* q, const void* k, const void* v, const void* out, const float* lse, int B, int Hq,
                  int Hkv, int L1, int L2, int D, float scale, const char* l1name, const char* l2name) {
-    if (!q || !k || !v || !out) return fail(ATTN_ERR_INVALID_ARG, "null tensor pointer");
+    const bool q_empty = (B == 0 || L1 == 0), kv_empty = (B == 0 || L2 == 0);
+    if ((!q && !q_empty) || (!out && !q_empty)) return fail(ATTN_ERR_INVALID_ARG, "null q or out pointer");
+    if ((!k || !v) && !kv_empty) return fail(ATTN_ERR_INVALID_ARG, "null k or v pointer");
     if (B < 0 || L1 < 0 || L2 < 0)
         return fail(ATTN_ERR_INVALID_ARG, "negative size (B=%d %s=%d %s=%d)", B, l1name, L1, l2name, L2);
     if (Hq < 1 || Hkv < 1) return fail(ATTN_ERR_INVALID_ARG, "head counts must be >= 1 (Hq=%d Hkv=%d)", Hq, Hkv);
@@ -258,7 +262,7 @@ extern "C" int attn_decode(const void* q, const void* k_cache, const void* v_cac
                            size_t workspace_bytes, void* stream) {
     int st = check_common(q, k_cache, v_cache, out, lse, B, Hq, Hkv, Lmax, Lmax, D, scale, "Lmax", "Lmax");
     if (st != ATTN_OK) return st;
-    if (!seqlens) return fail(ATTN_ERR_INVALID_ARG, "null seqlens");
+    if (!seqlens && B > 0) return fail(ATTN_ERR_INVALID_ARG, "null seqlens");
     if (reinterpret_cast<uintptr_t>(seqlens) & 3u) return fail(ATTN_ERR_INVALID_ARG, "seqlens must be 4-byte aligned");
     if (Lmax < 1) return fail(ATTN_ERR_INVALID_ARG, "Lmax must be >= 1");
     if (Hq / Hkv > 64) return fail(ATTN_ERR_UNSUPPORTED, "decode group size G=%d > 64", Hq / Hkv);

@@ -16,11 +16,17 @@
 // position p0 + r % P), so every K/V tile staged in shared memory feeds all
 // G heads of the group and both Q tiles.
 //
-// Roles (320 threads):
+// Roles (384 threads = 3 warpgroups):
 //   warps 0-3  softmax warpgroup for Q tile 0 (thread = TMEM lane = row)
 //   warps 4-7  softmax warpgroup for Q tile 1
 //   warp  8    TMA producer: Q tiles once, then K_j, V_j into a ring of stages
 //   warp  9    TMEM allocator and single-thread tcgen05.mma issuer
+//   warps 10-11 idle
+// The block launches at 168 registers per thread (3 warps per SM sub-partition
+// x 168 x 32 = 16128 of its 16384).  The third warpgroup then gives registers
+// back (setmaxnreg.dec to 88) and the softmax warpgroups take them
+// (setmaxnreg.inc to 208): 2 x 208 + 88 = 3 x 168, so the exchange balances
+// exactly and neither side waits.
 //
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D).
 // P_q (bf16, two per column) overwrites the first 64 columns of S_q once the
@@ -45,7 +51,11 @@
 
 namespace attn {
 
-constexpr int kPrefillThreads = 320;
+constexpr int kPrefillThreads = 384;
+constexpr int kPrefillLaunchRegs = 168;    // must equal the compiled register count (checked by the build)
+constexpr int kSoftmaxRegs = 208;
+constexpr int kControlRegs = 88;
+static_assert(2 * kSoftmaxRegs + kControlRegs == 3 * kPrefillLaunchRegs, "register exchange must balance");
 constexpr int kBM = 128;               // rows per Q tile (MMA M)
 constexpr int kBN = 128;               // keys per K/V tile
 constexpr float kRescaleLog2 = 8.0f;
@@ -78,7 +88,7 @@ struct PrefillParams {
 };
 
 template <int D>
-__global__ void __maxnreg__(200)
+__global__ void __launch_bounds__(kPrefillThreads, 1)
     attn_prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                               const __grid_constant__ CUtensorMap tm_k,
                               const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
@@ -159,7 +169,9 @@ __global__ void __maxnreg__(200)
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_base_ptr;
 
-    if (warp == 8) {
+    if (warp >= 8) {
+      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
+      if (warp == 8) {
         // ================= TMA producer =================
         if (lane == 0 && n_kt > 0) {
             tma_prefetch_desc(&tm_q);
@@ -275,7 +287,9 @@ __global__ void __maxnreg__(200)
             }
         }
         __syncwarp();
+      }
     } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
         // ================= softmax warpgroups =================
         const int q = warp >> 2;                 // Q tile of this warpgroup
         const int r = threadIdx.x & 127;         // row = TMEM lane

@@ -76,7 +76,10 @@ typedef enum {
  *   B == 0 or Lq == 0: nothing to do, returns ATTN_OK.
  *   Lk == 0: every row sees no key (O = 0, LSE = -inf).
  *
- * Errors: ATTN_ERR_INVALID_ARG for null q/k/v/out, negative sizes, Hq or
+ * q and out may be NULL only when they are empty (B == 0 or Lq == 0), k and
+ * v only when they are empty (B == 0 or Lk == 0).
+ *
+ * Errors: ATTN_ERR_INVALID_ARG for a null non-empty tensor, negative sizes, Hq or
  * Hkv < 1, Hq % Hkv != 0, non-finite or non-positive scale, or a base
  * address not 16-byte aligned; ATTN_ERR_UNSUPPORTED for D outside {64, 128}
  * or G > 128; ATTN_ERR_CUDA when a launch fails.

@@ -70,6 +70,11 @@ def test_prefill_rejects(lib, bad, code):
 def test_prefill_empty_is_noop(lib):
     assert _prefill(lib, B=0) == 0
     assert _prefill(lib, Lq=0) == 0
+    # empty tensors have no storage: null is accepted for them, and only for them
+    assert _prefill(lib, B=0, q=NULL, k=NULL, v=NULL, out=NULL) == 0
+    assert _prefill(lib, Lq=0, q=NULL, out=NULL) == 0
+    assert _prefill(lib, Lq=0, q=NULL, out=NULL, k=NULL) == -1
+    assert _prefill(lib, Lk=0, k=NULL, v=NULL, q=NULL) == -1
 
 
 def _decode(lib, **kw):
@@ -92,6 +97,7 @@ def test_decode_rejects(lib, bad, code):
 
 def test_decode_empty_batch_is_noop(lib):
     assert _decode(lib, B=0) == 0
+    assert _decode(lib, B=0, q=NULL, k=NULL, v=NULL, out=NULL, sl=NULL, ws=NULL) == 0
 
 
 def test_workspace_size(lib):
