@@ -40,6 +40,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
 from exact_tiled_attention_gqa_b200 import roofline as RL          # noqa: E402
+from exact_tiled_attention_gqa_b200.multigpu import max_over_ranks as _max_over_ranks, rank_seed  # noqa: E402
 from exact_tiled_attention_gqa_b200 import workloads as W          # noqa: E402
 
 METRIC = "prefill TFLOP/s & decode HBM GB/s (frac. of roofline), Qwen3-8B GQA shapes"
@@ -147,7 +148,7 @@ def run_ours(args, rank, world, local_rank):
     peaks = RL.measured_peaks()
 
     # ---- inputs (per rank: its own sequences; seeds differ by rank) ----
-    seed = args.seed + 1000 * rank
+    seed = rank_seed(args.seed, rank)
     if args.only != "decode":
         q_h, k_h, v_h = W.prefill_inputs_for(PREFILL, seed=seed, device="cpu")
         q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
@@ -224,11 +225,7 @@ def run_ours(args, rank, world, local_rank):
     assert derr == 0, f"device error word {derr:#x} after the timed region"
 
     def max_over_ranks(x):
-        if dist is None:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return _max_over_ranks(x, device=dev)
 
     total_ms = max_over_ranks(total_ms)
     pre_avg = max_over_ranks(sum(pre_ms) / len(pre_ms))
@@ -275,7 +272,7 @@ def run_ours(args, rank, world, local_rank):
     dec_gbs = world * d_bytes / (dec_avg * 1e-3) / 1e9
     peak_t = float(peaks["bf16_tflops"])
     peak_b = float(peaks["hbm_gbs"])
-    traffic = load_traffic()
+    traffic = RL.committed_traffic()
     line = {
         "metric": METRIC,
         "value": round(pre_tflops, 2),
@@ -324,15 +321,6 @@ def run_ours(args, rank, world, local_rank):
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(args, q_h, k_h, v_h, dq.cpu(), dk, dv, seqlens_host)
     return line
-
-
-def load_traffic():
-    """Per-launch DRAM bytes from the committed ncu summary, if one matches the current kernels."""
-    path = os.path.join(ROOT, "profiles", "traffic.json")
-    if not os.path.exists(path):
-        return {}
-    with open(path) as f:
-        return json.load(f)
 
 
 # --------------------------------------------------------------------------

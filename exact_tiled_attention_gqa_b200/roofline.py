@@ -14,6 +14,8 @@ KV head) plus q, out and lse.  Split-KV partials are overhead and not credited.
 """
 from __future__ import annotations
 
+import glob
+import hashlib
 import json
 import os
 
@@ -55,3 +57,25 @@ def measured_peaks() -> dict:
         d["source"] = "measured"
         return d
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def kernel_source_hash() -> str:
+    """Hash of the CUDA sources; a DRAM-traffic figure is only valid for the hash it was taken at."""
+    h = hashlib.sha256()
+    for path in sorted(glob.glob(os.path.join(ROOT, "exact_tiled_attention_gqa_b200", "csrc", "*"))):
+        with open(path, "rb") as f:
+            h.update(os.path.basename(path).encode())
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic() -> dict:
+    """Per-launch DRAM bytes from profiles/traffic.json, only if taken at the current sources."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return {}
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("source_hash") != kernel_source_hash():
+        return {}
+    return d.get("bytes_per_launch", {})
