@@ -22,7 +22,8 @@ import torch
 from . import _native
 from ._native import AttnError
 
-__all__ = ["prefill", "decode", "decode_workspace_size", "device_error", "AttnError", "library_path"]
+__all__ = ["prefill", "decode", "decode_noalloc", "decode_workspace_size", "device_error", "AttnError",
+           "library_path"]
 
 
 def library_path() -> str:
@@ -109,6 +110,28 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, seqlen
                                        B, Hq, Hkv, Lmax, D, float(scale), _ptr(workspace), workspace.numel(),
                                        _stream_handle(stream))
     _native.check(st, "attn_decode")
+    return out, lse
+
+
+def decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, seqlens: torch.Tensor, *,
+                   scale: Optional[float] = None, out: torch.Tensor, lse: Optional[torch.Tensor] = None, stream=None):
+    """decode() for callers that cannot allocate: the split partials use the
+    library's own fixed scratch (16 MiB per GPU), and `out` (and `lse`, if
+    wanted) must be passed in.  Calls on one GPU must not overlap in time."""
+    for n, t, dt, nd in (("q", q, torch.bfloat16, 3), ("k_cache", k_cache, torch.bfloat16, 4),
+                         ("v_cache", v_cache, torch.bfloat16, 4), ("seqlens", seqlens, torch.int32, 1),
+                         ("out", out, torch.bfloat16, 3)):
+        _check_tensor(n, t, dt, nd)
+    if lse is not None:
+        _check_tensor("lse", lse, torch.float32, 2)
+    B, Hq, D = q.shape
+    Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    with torch.cuda.device(q.device):
+        st = _native.lib().attn_decode_noalloc(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(out),
+                                               _ptr(lse), B, Hq, Hkv, Lmax, D, float(scale), _stream_handle(stream))
+    _native.check(st, "attn_decode_noalloc")
     return out, lse
 
 

@@ -20,6 +20,7 @@ ATTN_ERR_WORKSPACE = -3
 ATTN_ERR_CUDA = -4
 ATTN_DEVERR_TIMEOUT = 0x1
 ATTN_DEVERR_SEQLEN = 0x2
+ATTN_DECODE_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 # name -> (restype, argtypes): every symbol the header declares
 _vp, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
@@ -27,6 +28,7 @@ SIGNATURES = {
     "attn_prefill": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp]),
     "attn_decode_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32]),
     "attn_decode": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _sz, _vp]),
+    "attn_decode_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp]),
     "attn_status_string": (ctypes.c_char_p, [_i32]),
     "attn_last_error": (ctypes.c_char_p, []),
     "attn_device_error": (_i32, [ctypes.POINTER(ctypes.c_uint), _i32]),

@@ -306,3 +306,69 @@ extern "C" int attn_device_error(unsigned int* flags, int reset) {
     }
     return ok();
 }
+
+// ---------------------------------------------------------------------------
+// attn_decode_noalloc: attn_decode whose split partials live in a scratch
+// array declared here, for callers that cannot allocate device memory.
+// ---------------------------------------------------------------------------
+namespace attn {
+namespace {
+
+static __device__ __align__(256) uint8_t g_decode_scratch[ATTN_DECODE_NOALLOC_SCRATCH_BYTES];
+
+// In host code `g_decode_scratch` only names a host-side stand-in; the device
+// address is looked up once per device, with that device current.
+void* decode_scratch_address(int* status) {
+    static std::mutex mu;
+    static void* addr[64];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        *status = fail(ATTN_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+        return nullptr;
+    }
+    if (dev < 0 || dev >= 64) {
+        *status = fail(ATTN_ERR_CUDA, "device ordinal %d out of range", dev);
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (addr[dev] == nullptr) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_decode_scratch);
+        if (e != cudaSuccess || p == nullptr) {
+            *status = fail(ATTN_ERR_CUDA, "cudaGetSymbolAddress(decode scratch): %s", cudaGetErrorString(e));
+            return nullptr;
+        }
+        addr[dev] = p;
+    }
+    *status = ATTN_OK;
+    return addr[dev];
+}
+
+}  // namespace
+}  // namespace attn
+
+extern "C" int attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,
+                                   void* out, float* lse, int B, int Hq, int Hkv, int Lmax, int D, float scale,
+                                   void* stream) {
+    int st = check_common(q, k_cache, v_cache, out, lse, B, Hq, Hkv, Lmax, Lmax, D, scale, "Lmax", "Lmax");
+    if (st != ATTN_OK) return st;
+    if (!seqlens && B > 0) return fail(ATTN_ERR_INVALID_ARG, "null seqlens");
+    if (reinterpret_cast<uintptr_t>(seqlens) & 3u) return fail(ATTN_ERR_INVALID_ARG, "seqlens must be 4-byte aligned");
+    if (Lmax < 1) return fail(ATTN_ERR_INVALID_ARG, "Lmax must be >= 1");
+    if (Hq / Hkv > 64) return fail(ATTN_ERR_UNSUPPORTED, "decode group size G=%d > 64", Hq / Hkv);
+    if (static_cast<long long>(B) * Hq > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "B*Hq too large");
+    if (B == 0) return ok();
+    const size_t need = decode_layout(B, Hq, Hkv, Lmax, D).total;
+    if (need > ATTN_DECODE_NOALLOC_SCRATCH_BYTES)
+        return fail(ATTN_ERR_WORKSPACE,
+                    "attn_decode_noalloc: these sizes need %zu bytes of split partials; the static scratch holds %u "
+                    "(use attn_decode with a caller workspace)",
+                    need, ATTN_DECODE_NOALLOC_SCRATCH_BYTES);
+    void* scratch = decode_scratch_address(&st);
+    if (st != ATTN_OK) return st;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = (D == 128) ? launch_decode<128>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, scratch, s)
+                    : launch_decode<64>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, scratch, s);
+    return st == ATTN_OK ? ok() : st;
+}

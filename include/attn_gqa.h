@@ -130,6 +130,40 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, const i
                 void* out, float* lse, int B, int Hq, int Hkv, int Lmax, int D, float scale,
                 void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * attn_decode_noalloc -- attn_decode for callers that cannot allocate device
+ * memory: the split partials live in a scratch array that the library itself
+ * declares at file scope (ATTN_DECODE_NOALLOC_SCRATCH_BYTES per GPU, reserved
+ * on every GPU that loads the library and held until the process exits).
+ *
+ * The pages have no counterpart to this call; it exists for callers whose
+ * device memory is all owned by someone else -- an inference engine that
+ * reserves nearly all of HBM for its own pool up front, or a caller that must
+ * not call cudaMalloc on its hot path because cudaMalloc can synchronise the
+ * device and stall every stream -- and who therefore cannot hand attn_decode
+ * a workspace.
+ *
+ * Arguments, layouts and results are those of attn_decode, without the
+ * workspace.  Nothing is allocated: no cudaMalloc, cudaFree or allocating
+ * library routine is called.
+ *   - Sizes whose partials need more than ATTN_DECODE_NOALLOC_SCRATCH_BYTES
+ *     (attn_decode_workspace_size(...) > the limit) are rejected with
+ *     ATTN_ERR_WORKSPACE; attn_decode with a caller workspace has no limit.
+ *   - The first call on a device looks up the scratch array's device address
+ *     (once per device, with that device current); make that first call
+ *     before any stream capture.
+ *   - Every call on a device shares the one scratch array, which keeps the
+ *     previous call's contents.  Nothing in it has to start at zero: each
+ *     call writes every partial it later reads.  Calls whose kernels overlap
+ *     on the GPU (different streams, no ordering between them) race on the
+ *     array and produce wrong results; order them on one stream or with events.
+ */
+#define ATTN_DECODE_NOALLOC_SCRATCH_BYTES (16u << 20)
+
+int attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,
+                        void* out, float* lse, int B, int Hq, int Hkv, int Lmax, int D, float scale,
+                        void* stream);
+
 /* attn_status_string -- a static name for a status code; never NULL. */
 const char* attn_status_string(int status);
 
