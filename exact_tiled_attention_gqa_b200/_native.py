@@ -29,6 +29,7 @@ SIGNATURES = {
     "attn_decode_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32]),
     "attn_decode": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _sz, _vp]),
     "attn_decode_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp]),
+    "attn_selftest_exp2": (_i32, [_vp, _vp, _i32, _vp]),
     "attn_status_string": (ctypes.c_char_p, [_i32]),
     "attn_last_error": (ctypes.c_char_p, []),
     "attn_device_error": (_i32, [ctypes.POINTER(ctypes.c_uint), _i32]),

@@ -280,6 +280,29 @@ extern "C" int attn_decode(const void* q, const void* k_cache, const void* v_cac
     return st == ATTN_OK ? ok() : st;
 }
 
+namespace attn {
+namespace {
+__global__ void exp2_fma_selftest_kernel(const float* x, float* y, int n) {
+    const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
+    if (i >= n) return;
+    const float x0 = x[i], x1 = (i + 1 < n) ? x[i + 1] : 0.0f;
+    float y0, y1;
+    f2_unpack(exp2_fma_x2(f2_pack(x0, x1)), y0, y1);
+    y[i] = y0;
+    if (i + 1 < n) y[i + 1] = y1;
+}
+}  // namespace
+}  // namespace attn
+
+extern "C" int attn_selftest_exp2(const float* x, float* y, int n, void* stream) {
+    if (n < 0 || (n > 0 && (!x || !y))) return fail(ATTN_ERR_INVALID_ARG, "bad selftest arguments");
+    if (n == 0) return ok();
+    const int threads = 256, pairs = (n + 1) / 2;
+    exp2_fma_selftest_kernel<<<(pairs + threads - 1) / threads, threads, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+    const int st = check_launch("exp2_fma_selftest_kernel");
+    return st == ATTN_OK ? ok() : st;
+}
+
 extern "C" const char* attn_status_string(int status) {
     switch (status) {
         case ATTN_OK: return "ATTN_OK";

@@ -34,9 +34,17 @@
 //
 // Per key tile j the MMA thread issues, in order:
 //   O0 += P0(j) V_j ; S0(j+1) = Q0 K_{j+1}^T ; O1 += P1(j) V_j ; S1(j+1) = Q1 K_{j+1}^T
-// so the tensor cores work on one Q tile while the other's softmax runs.
+// so the tensor cores work on one Q tile while the other's softmax runs.  The
+// softmax hands P over in two halves (keys 0-63, then 64-127), and each half of
+// O_q += P_q V_j is issued as soon as its half is in TMEM.
 // A commit after S_q(j+1) also covers O_q += P_q(j) V_j, so when the softmax
 // sees S_q(j+1) its O_q is settled and may be rescaled in place.
+//
+// The exponentials of an unmasked tile are split between the MUFU unit
+// (ex2.approx) and the FMA pipe (a cubic after range reduction, see
+// exp2_fma_x2): at 128 exponentials per row per tile the MUFU unit alone
+// would take as long as the tile's two MMAs.  Scale-and-subtract, sums and
+// O rescales use packed f32x2 instructions, maxima a 3-input max.
 //
 // Online softmax, in the log2 domain (x2 = x * scale * log2 e): per row a
 // running max m and sum l.  The max used for the exponentials is only raised
@@ -45,6 +53,8 @@
 // is the same exact quantity -- O = sum_j 2^(s2_j - m) v_j / sum_j 2^(s2_j - m)
 // holds for any m -- and the O rescale in TMEM is skipped on most tiles.
 #pragma once
+
+#include <type_traits>
 
 #include "ptx_sm100.cuh"
 #include "device_error.cuh"
@@ -59,6 +69,12 @@ static_assert(2 * kSoftmaxRegs + kControlRegs == 3 * kPrefillLaunchRegs, "regist
 constexpr int kBM = 128;               // rows per Q tile (MMA M)
 constexpr int kBN = 128;               // keys per K/V tile
 constexpr float kRescaleLog2 = 8.0f;
+// Of every 8 pairs of exponentials in an unmasked tile, this many are computed
+// on the FMA pipe (exp2_fma_x2) and the rest on the MUFU unit.
+#ifndef ATTN_EXP_FMA_PAIRS_PER_8
+#define ATTN_EXP_FMA_PAIRS_PER_8 3
+#endif
+constexpr int kExpFmaPairsPer8 = ATTN_EXP_FMA_PAIRS_PER_8;
 
 template <int D>
 struct PrefillSmem {
@@ -70,8 +86,8 @@ struct PrefillSmem {
     static constexpr int kQOff = 0;
     static constexpr int kKVOff = 2 * kQTileBytes;
     static constexpr int kBarOff = kKVOff + kStages * kKVTileBytes;
-    // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_full[2], o_done[2], drain
-    static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 1;
+    // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_half[2], p_full[2], o_done[2], drain
+    static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 2 + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;   // tmem base (u32), abort flag (int)
     static constexpr int kBytes = kMiscOff + 16;
     static constexpr int kAlloc = kBytes + 1024;              // slack to align the base to 1 KiB
@@ -101,10 +117,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // ---- work unit: heaviest (latest) position blocks first ----
-    const int bh_count = p.B * p.Hkv;
-    const int mblk = p.n_mblk - 1 - static_cast<int>(blockIdx.x) / bh_count;
-    const int bh = static_cast<int>(blockIdx.x) % bh_count;
+    // ---- work unit: one (b, KV head) group after another, so CTAs running at
+    // the same time share that group's K/V in L2; within a group the heaviest
+    // (latest) position blocks come first ----
+    const int mblk = p.n_mblk - 1 - static_cast<int>(blockIdx.x % static_cast<unsigned>(p.n_mblk));
+    const int bh = static_cast<int>(blockIdx.x / static_cast<unsigned>(p.n_mblk));
     const int b = bh / p.Hkv;
     const int g = bh % p.Hkv;
     const int P = p.P;
@@ -127,9 +144,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     auto bar_kv_full = [&](int s) { return bar0 + 8u * (1 + s); };
     auto bar_kv_empty = [&](int s) { return bar0 + 8u * (1 + L::kStages + s); };
     auto bar_s_full = [&](int q) { return bar0 + 8u * (1 + 2 * L::kStages + q); };
-    auto bar_p_full = [&](int q) { return bar0 + 8u * (3 + 2 * L::kStages + q); };
-    auto bar_o_done = [&](int q) { return bar0 + 8u * (5 + 2 * L::kStages + q); };
-    const uint32_t bar_drain = bar0 + 8u * (7 + 2 * L::kStages);
+    auto bar_p_half = [&](int q) { return bar0 + 8u * (3 + 2 * L::kStages + q); };
+    auto bar_p_full = [&](int q) { return bar0 + 8u * (5 + 2 * L::kStages + q); };
+    auto bar_o_done = [&](int q) { return bar0 + 8u * (7 + 2 * L::kStages + q); };
+    const uint32_t bar_drain = bar0 + 8u * (9 + 2 * L::kStages);
     uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
 
@@ -141,6 +159,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         }
         for (int q = 0; q < 2; ++q) {
             mbar_init(bar_s_full(q), 1);
+            mbar_init(bar_p_half(q), 128);
             mbar_init(bar_p_full(q), 128);
             mbar_init(bar_o_done(q), 1);
         }
@@ -223,24 +242,44 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             const uint32_t tO[2] = {tmem + 256u, tmem + 256u + D};
             auto slot_of = [&](int t) { return t % L::kStages; };
             auto par_of = [&](int t) { return static_cast<uint32_t>(t / L::kStages) & 1u; };
+            // Shared-memory descriptors are built once; a k-step only moves the
+            // start-address field (bits 0-13, address >> 4), so each MMA issue
+            // costs one 64-bit add.
+            const uint64_t dQ[2] = {umma_sdesc_sw128(sQ, 16, 1024), umma_sdesc_sw128(sQ + L::kQTileBytes, 16, 1024)};
+            const uint64_t dK0 = umma_sdesc_sw128(sKV, 16, 1024);
+            const uint64_t dV0 = umma_sdesc_sw128(sKV, L::kBlockBytes, 1024);
+            constexpr uint64_t kSlotStep = L::kKVTileBytes >> 4;
             // S_q = Q_q K^T : M=128, N=128, K=D in steps of 16 (32 bytes)
             auto issue_qk = [&](int q, int t) {
-                const uint32_t a0 = sQ + q * L::kQTileBytes;
-                const uint32_t b0 = sKV + slot_of(t) * L::kKVTileBytes;
+                const uint64_t b0 = dK0 + static_cast<uint64_t>(slot_of(t)) * kSlotStep;
 #pragma unroll
                 for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t koff = (kk >> 2) * L::kBlockBytes + (kk & 3) * 32;
-                    umma_ss(tS[q], umma_sdesc_sw128(a0 + koff, 16, 1024), umma_sdesc_sw128(b0 + koff, 16, 1024),
-                            kIdescQK, kk > 0 ? 1u : 0u);
+                    const uint64_t koff = static_cast<uint64_t>(((kk >> 2) * L::kBlockBytes + (kk & 3) * 32) >> 4);
+                    umma_ss(tS[q], dQ[q] + koff, b0 + koff, kIdescQK, kk > 0 ? 1u : 0u);
                 }
             };
-            // O_q += P_q V : M=128, N=D, K=128 keys in steps of 16 (8 TMEM columns of P)
-            auto issue_pv = [&](int q, int t, bool acc) {
-                const uint32_t b0 = sKV + slot_of(t) * L::kKVTileBytes;
+            // O_q += P_q V : M=128, N=D, K=128 keys in steps of 16 (8 TMEM columns of P);
+            // `half` 0 covers keys 0-63 (P columns 0-31), half 1 keys 64-127
+            auto issue_pv = [&](int q, int t, bool acc, int half) {
+                const uint64_t b0 = dV0 + static_cast<uint64_t>(slot_of(t)) * kSlotStep;
 #pragma unroll
-                for (int kk = 0; kk < kBN / 16; ++kk)
-                    umma_ts(tO[q], tS[q] + kk * 8, umma_sdesc_sw128(b0 + kk * 2048, L::kBlockBytes, 1024),
-                            kIdescPV, (acc || kk > 0) ? 1u : 0u);
+                for (int k4 = 0; k4 < kBN / 32; ++k4) {
+                    const int kk = half * (kBN / 32) + k4;
+                    umma_ts(tO[q], tS[q] + kk * 8, b0 + static_cast<uint64_t>((kk * 2048) >> 4), kIdescPV,
+                            (acc || kk > 0) ? 1u : 0u);
+                }
+            };
+            // both halves of O_q += P_q(j) V_j, each as soon as the softmax has released it
+            auto pv_tile = [&](int q, int t, int j) {
+                if (!mbar_wait(bar_p_half(q), static_cast<uint32_t>(j) & 1u, abort_flag, &g_attn_err, kDevErrTimeout))
+                    return false;
+                tc_fence_after_sync();
+                issue_pv(q, t, j > 0, 0);
+                if (!mbar_wait(bar_p_full(q), static_cast<uint32_t>(j) & 1u, abort_flag, &g_attn_err, kDevErrTimeout))
+                    return false;
+                tc_fence_after_sync();
+                issue_pv(q, t, true, 1);
+                return true;
             };
             bool ok = mbar_wait(bar_q_full, 0, abort_flag, &g_attn_err, kDevErrTimeout);
             if (ok) ok = mbar_wait(bar_kv_full(slot_of(0)), par_of(0), abort_flag, &g_attn_err, kDevErrTimeout);
@@ -256,10 +295,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 const int tv = 2 * j + 1, tk = 2 * j + 2;
                 const bool last = (j + 1 == n_kt);
                 ok = mbar_wait(bar_kv_full(slot_of(tv)), par_of(tv), abort_flag, &g_attn_err, kDevErrTimeout) &&
-                     mbar_wait(bar_p_full(0), static_cast<uint32_t>(j) & 1u, abort_flag, &g_attn_err, kDevErrTimeout);
+                     pv_tile(0, tv, j);
                 if (!ok) break;
-                tc_fence_after_sync();
-                issue_pv(0, tv, j > 0);
                 if (last) umma_commit(bar_o_done(0));
                 if (!last) {
                     ok = mbar_wait(bar_kv_full(slot_of(tk)), par_of(tk), abort_flag, &g_attn_err, kDevErrTimeout);
@@ -268,10 +305,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     issue_qk(0, tk);
                     umma_commit(bar_s_full(0));
                 }
-                ok = mbar_wait(bar_p_full(1), static_cast<uint32_t>(j) & 1u, abort_flag, &g_attn_err, kDevErrTimeout);
+                ok = pv_tile(1, tv, j);
                 if (!ok) break;
-                tc_fence_after_sync();
-                issue_pv(1, tv, j > 0);
                 if (last) umma_commit(bar_o_done(1));
                 umma_commit(bar_kv_empty(slot_of(tv)));
                 if (!last) {
@@ -325,7 +360,8 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
 #pragma unroll
             for (int c = 0; c < kBN; ++c) s[c] = __uint_as_float(sr[c]);
             const long key0 = static_cast<long>(j) * kBN;
-            if (key0 + kBN - 1 > tile_min_bound) {
+            const bool masked = key0 + kBN - 1 > tile_min_bound;
+            if (masked) {
                 // diagonal or ragged tile: mask keys beyond this row's bound
 #pragma unroll
                 for (int c = 0; c < kBN; ++c)
@@ -333,13 +369,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             }
             float mx[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) mx[i] = s[i];
+            for (int i = 0; i < 8; ++i) mx[i] = fmax3(s[i], s[8 + i], s[16 + i]);
 #pragma unroll
-            for (int c = 8; c < kBN; c += 8)
+            for (int c = 24; c < kBN - 8; c += 16)
 #pragma unroll
-                for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[c + i]);
-            float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+                for (int i = 0; i < 8; ++i) mx[i] = fmax3(mx[i], s[c + i], s[c + 8 + i]);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[kBN - 8 + i]);
+            const float tmax = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(fmax3(mx[3], mx[4], mx[5]), mx[6], mx[7]));
             const float m_tile = tmax * sl2;   // -inf stays -inf
             float factor = 1.0f;
             if (m_tile > m_run + kRescaleLog2) {
@@ -350,6 +387,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             // rescale O_q in TMEM if any row of this warp raised its max (O holds
             // the sum over tiles < j, settled: see the file comment)
             if (j > 0 && __any_sync(0xffffffffu, factor != 1.0f)) {
+                const uint64_t f2 = f2_pack(factor, factor);
 #pragma unroll 1
                 for (int c = 0; c < D; c += 32) {
                     uint32_t orr[32];
@@ -357,30 +395,58 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     tmem_wait_ld();
                     reg_fence<32>(orr);
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        orr[i] = __float_as_uint(__uint_as_float(orr[i]) * factor);
+                    for (int i = 0; i < 32; i += 2) {
+                        float a0, a1;
+                        f2_unpack(f2_mul(f2_pack(__uint_as_float(orr[i]), __uint_as_float(orr[i + 1])), f2), a0, a1);
+                        orr[i] = __float_as_uint(a0);
+                        orr[i + 1] = __float_as_uint(a1);
+                    }
                     tmem_st_32x32b_x32(tO + c, orr);
                 }
                 tmem_wait_st();
             }
+            // exponentials 2^(s * scale * log2 e - m), the row sum, and P (bf16)
+            // into TMEM in two halves, each handed to the MMA thread at once
             const float m_sub = (m_run == -INFINITY) ? 0.0f : m_run;
-            float lsum[8];
+            const uint64_t sl2x2 = f2_pack(sl2, sl2);
+            const uint64_t negm2 = f2_pack(-m_sub, -m_sub);
+            uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
+            auto exp_half = [&](auto masked_tag, int h) {
+                constexpr bool kMasked = decltype(masked_tag)::value;
+                uint32_t pk[32];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) lsum[i] = 0.0f;
-            uint32_t pk[64];
-#pragma unroll
-            for (int c = 0; c < kBN; c += 2) {
-                const float e0 = ex2_approx(fmaf(s[c], sl2, -m_sub));
-                const float e1 = ex2_approx(fmaf(s[c + 1], sl2, -m_sub));
-                lsum[(c >> 1) & 7] += e0 + e1;
-                pk[c >> 1] = pack_bf16x2(e0, e1);
+                for (int i = 0; i < 32; ++i) {
+                    const int c = h * 64 + 2 * i;
+                    const uint64_t t = f2_fma(f2_pack(s[c], s[c + 1]), sl2x2, negm2);
+                    uint64_t e;
+                    if (!kMasked && (i % 8) < kExpFmaPairsPer8) {
+                        e = exp2_fma_x2(t);
+                    } else {
+                        float t0, t1;
+                        f2_unpack(t, t0, t1);
+                        e = f2_pack(ex2_approx(t0), ex2_approx(t1));
+                    }
+                    acc2[i & 3] = f2_add(acc2[i & 3], e);
+                    float e0, e1;
+                    f2_unpack(e, e0, e1);
+                    pk[i] = pack_bf16x2(e0, e1);
+                }
+                tmem_st_32x32b_x32(tS + h * 32, pk);
+                tmem_wait_st();
+                tc_fence_before_sync();
+                mbar_arrive(h == 0 ? bar_p_half(q) : bar_p_full(q));
+            };
+            if (masked) {
+                exp_half(std::true_type{}, 0);
+                exp_half(std::true_type{}, 1);
+            } else {
+                exp_half(std::false_type{}, 0);
+                exp_half(std::false_type{}, 1);
             }
-            l_run += ((lsum[0] + lsum[1]) + (lsum[2] + lsum[3])) + ((lsum[4] + lsum[5]) + (lsum[6] + lsum[7]));
-            tmem_st_32x32b_x32(tS + 0, pk);
-            tmem_st_32x32b_x32(tS + 32, pk + 32);
-            tmem_wait_st();
-            tc_fence_before_sync();
-            mbar_arrive(bar_p_full(q));
+            float a0, a1, b0, b1;
+            f2_unpack(f2_add(acc2[0], acc2[1]), a0, a1);
+            f2_unpack(f2_add(acc2[2], acc2[3]), b0, b1);
+            l_run += (a0 + a1) + (b0 + b1);
         }
 
         // ---- epilogue: O / l -> bf16, LSE ----

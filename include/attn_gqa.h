@@ -164,6 +164,15 @@ int attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
                         void* out, float* lse, int B, int Hq, int Hkv, int Lmax, int D, float scale,
                         void* stream);
 
+/*
+ * attn_selftest_exp2 -- diagnostic: y[i] = the prefill softmax's FMA-pipe
+ * approximation of 2^x[i] (range reduction plus a minimax cubic; relative
+ * error about 7.5e-5 for x in [-125, 8], below 2e-4 for x in [-126, -125]
+ * where the result nears the subnormal range; inputs below -126 are clamped
+ * to -126).  x and y are device arrays of n floats; enqueued on `stream`.
+ */
+int attn_selftest_exp2(const float* x, float* y, int n, void* stream);
+
 /* attn_status_string -- a static name for a status code; never NULL. */
 const char* attn_status_string(int status);
 

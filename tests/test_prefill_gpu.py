@@ -113,3 +113,28 @@ def test_full_size_sampled_rows(oracle_mod, shape):
         rows = rows[:48]
     _run(oracle_mod, shape.B, shape.Hq, shape.Hkv, shape.Lq, shape.Lk, shape.D, shape.is_causal, seed=0,
          spike=shape.spike_every, rows=rows)
+
+
+def test_fma_pipe_exp2_against_cuda_exp2():
+    """The softmax's FMA-pipe 2^x (range reduction + minimax cubic) against CUDA's exp2f (via torch)."""
+    import ctypes
+    from exact_tiled_attention_gqa_b200 import _native
+    x = torch.cat([torch.linspace(-126.0, 8.0, 1_000_001), torch.linspace(-1.0, 1.0, 100_001),
+                   torch.arange(-126, 9).float()]).cuda()
+    y = torch.empty_like(x)
+    st = _native.lib().attn_selftest_exp2(ctypes.c_void_p(x.data_ptr()), ctypes.c_void_p(y.data_ptr()), x.numel(),
+                                          ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == 0
+    ref = torch.exp2(x.double())
+    rel = (y.double() - ref).abs() / ref
+    normal = x >= -125.0
+    assert rel[normal].max().item() <= 1e-4, rel[normal].max().item()
+    # within 1 of the clamp the result nears the subnormal range and may lose the implicit bit
+    assert rel[~normal].max().item() <= 2e-4, rel[~normal].max().item()
+    # below the clamp the result is the value at -126, a tiny positive number
+    z = torch.tensor([-1000.0, -127.0], device="cuda")
+    w = torch.empty_like(z)
+    _native.lib().attn_selftest_exp2(ctypes.c_void_p(z.data_ptr()), ctypes.c_void_p(w.data_ptr()), 2,
+                                     ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    torch.cuda.synchronize()
+    assert torch.all(w > 0) and torch.all(w < 2e-38)
