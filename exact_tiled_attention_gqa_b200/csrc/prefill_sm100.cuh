@@ -70,9 +70,12 @@ constexpr int kBM = 128;               // rows per Q tile (MMA M)
 constexpr int kBN = 128;               // keys per K/V tile
 constexpr float kRescaleLog2 = 8.0f;
 // Of every 8 pairs of exponentials in an unmasked tile, this many are computed
-// on the FMA pipe (exp2_fma_x2) and the rest on the MUFU unit.
+// on the FMA pipe (exp2_fma_x2) and the rest on the MUFU unit.  Measured on
+// B200: 0 is fastest for this kernel (the softmax is latency-bound, not MUFU
+// throughput-bound: each Q tile's softmax waits on its own S / P / MMA chain),
+// so the FMA-pipe exponential is built and tested but off by default.
 #ifndef ATTN_EXP_FMA_PAIRS_PER_8
-#define ATTN_EXP_FMA_PAIRS_PER_8 3
+#define ATTN_EXP_FMA_PAIRS_PER_8 0
 #endif
 constexpr int kExpFmaPairsPer8 = ATTN_EXP_FMA_PAIRS_PER_8;
 
@@ -294,14 +297,14 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             for (int j = 0; j < n_kt && ok; ++j) {
                 const int tv = 2 * j + 1, tk = 2 * j + 2;
                 const bool last = (j + 1 == n_kt);
-                ok = mbar_wait(bar_kv_full(slot_of(tv)), par_of(tv), abort_flag, &g_attn_err, kDevErrTimeout) &&
-                     pv_tile(0, tv, j);
+                // operands first (normally long landed), so only the P waits sit on the chain
+                ok = mbar_wait(bar_kv_full(slot_of(tv)), par_of(tv), abort_flag, &g_attn_err, kDevErrTimeout);
+                if (ok && !last)
+                    ok = mbar_wait(bar_kv_full(slot_of(tk)), par_of(tk), abort_flag, &g_attn_err, kDevErrTimeout);
+                ok = ok && pv_tile(0, tv, j);
                 if (!ok) break;
                 if (last) umma_commit(bar_o_done(0));
                 if (!last) {
-                    ok = mbar_wait(bar_kv_full(slot_of(tk)), par_of(tk), abort_flag, &g_attn_err, kDevErrTimeout);
-                    if (!ok) break;
-                    tc_fence_after_sync();
                     issue_qk(0, tk);
                     umma_commit(bar_s_full(0));
                 }
