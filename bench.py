@@ -62,6 +62,8 @@ def parse():
                     help="profiling aid: time one call type only (the JSON line is then partial)")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="profiling aid: use the first N sequences of the decode batch")
+    ap.add_argument("--no-sweeps", action="store_true",
+                    help="skip the other workloads (group-size decode sweep, other prefill shapes)")
     return ap.parse_args()
 
 
@@ -266,6 +268,14 @@ def run_ours(args, rank, world, local_rank):
     h2d = (hq.numel() + hk.numel() + hv.numel() + hdq.numel()) * 2
     d2h = (ho.numel() + hdo.numel()) * 2 + (hl.numel() + hdl.numel()) * 4
 
+    cpu_line = None
+    if rank == 0 and not args.no_cpu_baseline and args.only is None:
+        cpu_line = cpu_baseline(args, q_h, k_h, v_h, dq.cpu(), dk, dv, seqlens_host)
+    sweeps = None
+    if not args.no_sweeps and args.only is None:
+        del dk, dv   # make room: the group-size sweep holds up to 34 GB of cache at a time
+        torch.cuda.empty_cache()
+        sweeps = run_sweeps(attn, dev, stream, seed, max_over_ranks)
     if rank != 0:
         return None
     pre_tflops = world * p_flops / (pre_avg * 1e-3) / 1e12
@@ -316,11 +326,72 @@ def run_ours(args, rank, world, local_rank):
                 "what": "pinned host -> device inputs, attn_prefill / attn_decode, device -> host outputs; "
                         "decode KV cache resident"},
         "gpu_launches": 3 * args.steps,
+        "sweeps": sweeps,
         "clocks": clocks,
     }
-    if not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(args, q_h, k_h, v_h, dq.cpu(), dk, dv, seqlens_host)
+    if cpu_line is not None:
+        line["cpu_baseline"] = cpu_line
     return line
+
+
+_L2_FLUSH = None
+
+
+def _time_calls(fn, stream, n_warm=2, n=10, flush=False):
+    """Mean device time of fn() over n calls (CUDA events on `stream`).  With
+    flush, a 256 MB write (twice the L2) precedes every call, outside its events."""
+    global _L2_FLUSH
+    for _ in range(n_warm):
+        fn()
+    if flush and _L2_FLUSH is None:
+        _L2_FLUSH = torch.empty(256 << 20, dtype=torch.uint8, device=torch.cuda.current_device())
+    total = 0.0
+    for _ in range(n):
+        if flush:
+            _L2_FLUSH.fill_(1)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        e1.synchronize()
+        total += e0.elapsed_time(e1)
+    return total / n
+
+
+def run_sweeps(attn, dev, stream, seed, max_over_ranks):
+    """The other workloads: Qwen3-8B prefill B1 L4096, the chunked prefills, and the
+    group-size decode sweep (Hq=64, D=128, batch 8, 131072 keys, G = 1 .. 64)."""
+    peaks = RL.measured_peaks()
+    out = {"prefill": [], "decode_group_sweep": []}
+    for shape in (W.QWEN_PREFILL_4K, W.CHUNKED_16K, W.CHUNKED_32K):
+        q, k, v = (t.to(dev) for t in W.prefill_inputs_for(shape, seed=seed))
+        o = torch.empty_like(q)
+        l = torch.empty((shape.B, shape.Hq, shape.Lq), dtype=torch.float32, device=dev)
+        small = (q.numel() + 2 * k.numel()) * 2 < 126e6
+        ms = max_over_ranks(_time_calls(lambda: attn.prefill(q, k, v, scale=shape.scale, is_causal=True, out=o,
+                                                              lse=l, stream=stream), stream, n=20, flush=small))
+        fl = RL.prefill_flops(shape.B, shape.Hq, shape.Lq, shape.Lk, shape.D, True)
+        out["prefill"].append({"workload": shape.name, "ms": round(ms, 4), "tflops": round(fl / ms / 1e9, 1),
+                               "frac_of_measured_bf16": round(fl / ms / 1e9 / float(peaks["bf16_tflops"]), 4),
+                               "l2": "L2 flushed (256 MB write) before each timed call" if small else
+                                     "inputs larger than L2"})
+        del q, k, v, o, l
+    for G in W.GROUP_SWEEP:
+        shape = W.group_sweep_decode(G)
+        dq, dk, dv, dsl = W.decode_inputs_for(shape, seed=seed + G, device=dev)
+        o = torch.empty_like(dq)
+        l = torch.empty((shape.B, shape.Hq), dtype=torch.float32, device=dev)
+        ws = torch.empty(attn.decode_workspace_size(shape.B, shape.Hq, shape.Hkv, shape.Lmax, shape.D),
+                         dtype=torch.uint8, device=dev)
+        ms = max_over_ranks(_time_calls(lambda: attn.decode(dq, dk, dv, dsl, scale=shape.scale, out=o, lse=l,
+                                                             workspace=ws, stream=stream), stream, n=10))
+        by = RL.decode_bytes(dsl.cpu().tolist(), shape.B, shape.Hq, shape.Hkv, shape.D)
+        out["decode_group_sweep"].append({"G": G, "Hkv": shape.Hkv, "ms": round(ms, 4), "bytes": by,
+                                          "gbs": round(by / ms / 1e6, 1),
+                                          "frac_of_measured_hbm": round(by / ms / 1e6 / float(peaks["hbm_gbs"]), 4)})
+        del dq, dk, dv, dsl, o, l, ws
+        torch.cuda.empty_cache()
+    return out
 
 
 # --------------------------------------------------------------------------

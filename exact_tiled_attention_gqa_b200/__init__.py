@@ -6,6 +6,9 @@ Two calls, both thin wrappers over the C ABI in ``include/attn_gqa.h``:
   the bottom-right causal mask, for Q [B,Hq,Lq,D] and K/V [B,Hkv,Lk,D] bf16.
 * ``decode(q, k_cache, v_cache, seqlens)`` -- one new token per sequence
   against a KV cache [B,Hkv,Lmax,D] whose rows 0..seqlens[b]-1 are valid.
+* ``decode_mq(q, k_cache, v_cache, seqlens)`` -- Lq new tokens per sequence
+  (q [B,Hq,Lq,D]), the last Lq rows of the cache, bottom-right causal: the
+  verify step of speculative decoding.
 
 Both return ``(out, lse)``: out bf16 shaped like q, lse fp32 (natural log).
 PyTorch supplies device memory and the current stream; every step of the
@@ -22,8 +25,8 @@ import torch
 from . import _native
 from ._native import AttnError
 
-__all__ = ["prefill", "decode", "decode_noalloc", "decode_workspace_size", "device_error", "AttnError",
-           "library_path"]
+__all__ = ["prefill", "decode", "decode_mq", "decode_noalloc", "decode_workspace_size",
+           "decode_mq_workspace_size", "device_error", "AttnError", "library_path"]
 
 
 def library_path() -> str:
@@ -110,6 +113,40 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, seqlen
                                        B, Hq, Hkv, Lmax, D, float(scale), _ptr(workspace), workspace.numel(),
                                        _stream_handle(stream))
     _native.check(st, "attn_decode")
+    return out, lse
+
+
+def decode_mq_workspace_size(B: int, Hq: int, Hkv: int, Lq: int, Lmax: int, D: int) -> int:
+    return int(_native.lib().attn_decode_mq_workspace_size(B, Hq, Hkv, Lq, Lmax, D))
+
+
+def decode_mq(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, seqlens: torch.Tensor, *,
+              scale: Optional[float] = None, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+              want_lse: bool = True, workspace: Optional[torch.Tensor] = None, stream=None):
+    """Lq new tokens per sequence.  q [B,Hq,Lq,D], caches [B,Hkv,Lmax,D] bf16, seqlens int32 [B] (CUDA);
+    the new tokens are the last Lq of each sequence's seqlens[b] cached rows."""
+    _check_tensor("q", q, torch.bfloat16, 4)
+    _check_tensor("k_cache", k_cache, torch.bfloat16, 4)
+    _check_tensor("v_cache", v_cache, torch.bfloat16, 4)
+    _check_tensor("seqlens", seqlens, torch.int32, 1)
+    B, Hq, Lq, D = q.shape
+    Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
+    if k_cache.shape[0] != B or k_cache.shape[3] != D or v_cache.shape != k_cache.shape or seqlens.shape[0] != B:
+        raise ValueError("shape mismatch between q, the caches and seqlens")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    need = decode_mq_workspace_size(B, Hq, Hkv, Lq, Lmax, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    with torch.cuda.device(q.device):
+        st = _native.lib().attn_decode_mq(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(out),
+                                          _ptr(lse), B, Hq, Hkv, Lq, Lmax, D, float(scale), _ptr(workspace),
+                                          workspace.numel(), _stream_handle(stream))
+    _native.check(st, "attn_decode_mq")
     return out, lse
 
 

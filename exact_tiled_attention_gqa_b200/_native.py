@@ -28,6 +28,9 @@ SIGNATURES = {
     "attn_prefill": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp]),
     "attn_decode_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32]),
     "attn_decode": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _sz, _vp]),
+    "attn_decode_mq_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32]),
+    "attn_decode_mq": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _sz,
+                              _vp]),
     "attn_decode_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp]),
     "attn_selftest_exp2": (_i32, [_vp, _vp, _i32, _vp]),
     "attn_status_string": (ctypes.c_char_p, [_i32]),

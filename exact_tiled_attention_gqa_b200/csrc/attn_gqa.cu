@@ -146,11 +146,11 @@ struct DecodeLayout {
     size_t o_bytes, lse_off, total;
 };
 
-DecodeLayout decode_layout(int B, int Hq, int Hkv, int Lmax, int D) {
+DecodeLayout decode_layout(int B, int Hq, int Hkv, int Lmax, int D, int Lq = 1) {
     DecodeLayout d;
     d.chunk = decode_chunk(B, Hkv, Lmax);
     d.n_splits = (Lmax + d.chunk - 1) / d.chunk;
-    const size_t rows = static_cast<size_t>(B) * Hq * d.n_splits;
+    const size_t rows = static_cast<size_t>(B) * Hq * Lq * d.n_splits;
     d.o_bytes = align256(rows * D * sizeof(float));
     d.lse_off = d.o_bytes;
     d.total = d.o_bytes + align256(rows * sizeof(float));
@@ -170,8 +170,8 @@ int launch_decode_split(const CUtensorMap& tk, const CUtensorMap& tv, const Deco
 
 template <int D>
 int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* seqlens, void* out, float* lse, int B,
-                  int Hq, int Hkv, int Lmax, float scale, void* workspace, cudaStream_t stream) {
-    const DecodeLayout lay = decode_layout(B, Hq, Hkv, Lmax, D);
+                  int Hq, int Hkv, int Lmax, float scale, void* workspace, cudaStream_t stream, int Lq = 1) {
+    const DecodeLayout lay = decode_layout(B, Hq, Hkv, Lmax, D, Lq);
     CUtensorMap tk, tv;
     int st;
     if ((st = encode_bf16_3d(&tk, kc, D, Lmax, static_cast<uint64_t>(B) * Hkv, 64, kDecKT, 1, "k_cache")) != ATTN_OK)
@@ -188,19 +188,21 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
     prm.Hkv = Hkv;
     prm.Lmax = Lmax;
     prm.G = Hq / Hkv;
+    prm.Lq = Lq;
     prm.chunk = lay.chunk;
     prm.n_splits = lay.n_splits;
     prm.scale_log2 = scale * kLog2e;
     if (prm.n_splits > 65535 || Hkv > 65535 || B > 65535)
         return fail(ATTN_ERR_UNSUPPORTED, "decode grid (%d, %d, %d) exceeds launch limits", prm.n_splits, Hkv, B);
-    if (prm.G <= 16)
+    const int rows_per_group = prm.G * Lq;
+    if (rows_per_group <= 16)
         st = launch_decode_split<D, 16>(tk, tv, prm, stream);
-    else if (prm.G <= 32)
+    else if (rows_per_group <= 32)
         st = launch_decode_split<D, 32>(tk, tv, prm, stream);
     else
         st = launch_decode_split<D, 64>(tk, tv, prm, stream);
     if (st != ATTN_OK) return st;
-    const int rows = B * Hq;
+    const int rows = B * Hq * Lq;
     attn_decode_combine_kernel<D><<<(rows + 3) / 4, 128, 0, stream>>>(prm, static_cast<__nv_bfloat16*>(out), lse);
     return check_launch("attn_decode_combine_kernel");
 }
@@ -300,6 +302,40 @@ extern "C" int attn_selftest_exp2(const float* x, float* y, int n, void* stream)
     const int threads = 256, pairs = (n + 1) / 2;
     exp2_fma_selftest_kernel<<<(pairs + threads - 1) / threads, threads, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
     const int st = check_launch("exp2_fma_selftest_kernel");
+    return st == ATTN_OK ? ok() : st;
+}
+
+extern "C" size_t attn_decode_mq_workspace_size(int B, int Hq, int Hkv, int Lq, int Lmax, int D) {
+    if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Lmax < 1 || Lq < 1 || (D != 64 && D != 128) ||
+        static_cast<long long>(Hq / Hkv) * Lq > 64)
+        return 0;
+    if (B == 0) return 0;
+    return decode_layout(B, Hq, Hkv, Lmax, D, Lq).total;
+}
+
+extern "C" int attn_decode_mq(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,
+                              void* out, float* lse, int B, int Hq, int Hkv, int Lq, int Lmax, int D, float scale,
+                              void* workspace, size_t workspace_bytes, void* stream) {
+    int st = check_common(q, k_cache, v_cache, out, lse, B, Hq, Hkv, Lq, Lmax, D, scale, "Lq", "Lmax");
+    if (st != ATTN_OK) return st;
+    if (Lq < 1) return fail(ATTN_ERR_INVALID_ARG, "Lq must be >= 1");
+    if (!seqlens && B > 0) return fail(ATTN_ERR_INVALID_ARG, "null seqlens");
+    if (reinterpret_cast<uintptr_t>(seqlens) & 3u) return fail(ATTN_ERR_INVALID_ARG, "seqlens must be 4-byte aligned");
+    if (Lmax < 1) return fail(ATTN_ERR_INVALID_ARG, "Lmax must be >= 1");
+    if (static_cast<long long>(Hq / Hkv) * Lq > 64)
+        return fail(ATTN_ERR_UNSUPPORTED, "G * Lq = %lld query rows per KV head (built: up to 64)",
+                    static_cast<long long>(Hq / Hkv) * Lq);
+    if (static_cast<long long>(B) * Hq * Lq > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "B*Hq*Lq too large");
+    if (B == 0) return ok();
+    const size_t need = decode_layout(B, Hq, Hkv, Lmax, D, Lq).total;
+    if (!workspace || workspace_bytes < need)
+        return fail(ATTN_ERR_WORKSPACE, "decode workspace needs %zu bytes, got %zu", need,
+                    workspace ? workspace_bytes : static_cast<size_t>(0));
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+        return fail(ATTN_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = (D == 128) ? launch_decode<128>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s, Lq)
+                    : launch_decode<64>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s, Lq);
     return st == ATTN_OK ? ok() : st;
 }
 

@@ -1,9 +1,12 @@
 // decode_sm100.cuh -- split-KV GQA decode and its log-sum-exp combine.
 //
-// What it computes: for each sequence b and query head h, one new query row
-// against cache rows 0 .. seqlens[b]-1 of KV head h / G (no mask: the new
-// token sees every cached key -- the "use_cache" and is_causal sections of
-// the SDPA / FlashAttention selection guide).  Decode is bound by reading the
+// What it computes: for each sequence b and query head h, Lq new query rows
+// (Lq = 1: plain decode; Lq > 1: the speculative-decoding verify step or a
+// small chunk) against cache rows of KV head h / G.  The Lq new tokens are the
+// last Lq of the sequence's seqlens[b] cached rows, so new token i sees rows
+// 0 .. seqlens[b] - Lq + i (the bottom-right alignment of the is_causal
+// section of the SDPA / FlashAttention selection guide; for Lq = 1 every
+// cached row, as its "use_cache" section has it).  Decode is bound by reading the
 // cache (NVIDIA attention page, "Prefill and decode are two different
 // tasks"), so the kernel is built around streaming K and V once at full HBM
 // bandwidth:
@@ -12,13 +15,13 @@
 //                 of one (b, KV head): a producer warp streams 64-row K and V
 //                 tiles into a ring of shared-memory stages with TMA (128-byte
 //                 swizzle, so the ldmatrix reads below are conflict-free); four
-//                 compute warps multiply the G query heads of the group (as
+//                 compute warps multiply the G x Lq query rows of the group (as
 //                 the M rows of m16n8k16 tensor-core MMAs, padded to 16) with
 //                 each tile once, run an online softmax, and accumulate P V.
 //                 Warps sharing a 16-row block split the tile's keys and merge
 //                 through shared memory at the end; the CTA writes one
 //                 normalised partial output and its log2-sum-exp per row.
-//   combine       one warp per (b, h): LSE-weighted sum of that row's partials.
+//   combine       one warp per query row: LSE-weighted sum of its partials.
 //
 // Splitting the cache length and merging by log-sum-exp is the single-GPU
 // form of the KV parallelism on the NVIDIA page ("Parameter four").
@@ -49,11 +52,12 @@ struct DecodeSmem {
 };
 
 struct DecodeParams {
-    const __nv_bfloat16* q;   // [B,Hq,D]
+    const __nv_bfloat16* q;   // [B,Hq,Lq,D]
     const int* seqlens;       // [B]
-    float* o_part;            // [B,Hq,n_splits,D]
-    float* lse_part;          // [B,Hq,n_splits] (log2 domain)
+    float* o_part;            // [B,Hq,Lq,n_splits,D]
+    float* lse_part;          // [B,Hq,Lq,n_splits] (log2 domain)
     int B, Hq, Hkv, Lmax, G;
+    int Lq;                   // new query rows per sequence (1 = plain decode)
     int chunk;                // cache rows per split (multiple of 64)
     int n_splits;
     float scale_log2;
@@ -68,7 +72,9 @@ __device__ __forceinline__ int decode_seqlen(const DecodeParams& p, int b) {
     return n;
 }
 
-// KPW = cache rows of each 64-row tile handled by one compute warp (16, 32 or 64)
+// KPW = cache rows of each 64-row tile handled by one compute warp (16, 32 or 64).
+// A group's query rows are the G heads x Lq new tokens, head-major (row r = head
+// r / Lq, token r % Lq), which is also their order in q, out and lse.
 template <int D, int KPW>
 __global__ void __maxnreg__(200)
     attn_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
@@ -144,15 +150,20 @@ __global__ void __maxnreg__(200)
     const int ws = warp % kWPM;           // which slice of each tile's keys
     const int key_off = ws * KPW;
     const int grp = lane >> 2, tq = lane & 3;
-    const int h0 = g * p.G + mt * 16;     // first query head of this block
+    const int R = p.G * p.Lq;             // query rows of the group
     const int row_a = mt * 16 + grp, row_b = row_a + 8;   // rows (within the group) this thread holds
+    const size_t group_row0 = (static_cast<size_t>(b) * p.Hq + static_cast<size_t>(g) * p.G) * p.Lq;
+    // keys this thread's rows may see: below min(k_end, seqlen - Lq + token + 1)
+    const int lim_a = min(k_end, seqlen - p.Lq + row_a % p.Lq + 1);
+    const int lim_b = min(k_end, seqlen - p.Lq + row_b % p.Lq + 1);
+    const int lim_lo = min(k_end, seqlen - p.Lq + 1);   // the smallest limit of any row
 
-    // Q as m16n8k16 A fragments (rows beyond G are zero)
+    // Q as m16n8k16 A fragments (rows beyond R are zero)
     uint32_t qa[D / 16][4];
     {
-        const uint32_t* qrow_a = reinterpret_cast<const uint32_t*>(p.q + (static_cast<size_t>(b) * p.Hq + h0 + grp) * D);
-        const uint32_t* qrow_b = reinterpret_cast<const uint32_t*>(p.q + (static_cast<size_t>(b) * p.Hq + h0 + grp + 8) * D);
-        const bool va = row_a < p.G, vb = row_b < p.G;
+        const uint32_t* qrow_a = reinterpret_cast<const uint32_t*>(p.q + (group_row0 + row_a) * D);
+        const uint32_t* qrow_b = reinterpret_cast<const uint32_t*>(p.q + (group_row0 + row_b) * D);
+        const bool va = row_a < R, vb = row_b < R;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
             const int c = (kk * 16 + 2 * tq) >> 1;   // bf16x2 index
@@ -177,7 +188,8 @@ __global__ void __maxnreg__(200)
         const uint32_t kbase = ring + s * L::kStageBytes;
         const uint32_t vbase = kbase + L::kTileBytes;
         const int tile_key0 = k_begin + t * kDecKT + key_off;   // absolute row of this warp's first key
-        const bool tail = (k_begin + (t + 1) * kDecKT > k_end);
+        const bool tail = (k_begin + (t + 1) * kDecKT > k_end);            // rows past the valid length
+        const bool masked = (k_begin + (t + 1) * kDecKT > lim_lo);        // keys some row may not see
 
         // ---- S = Q K^T over this warp's KPW keys ----
         float sacc[kNT][4];
@@ -199,13 +211,15 @@ __global__ void __maxnreg__(200)
                 mma_bf16_16816(sacc[2 * np + 1], qa[kk], r2, r3);
             }
         }
-        // ---- mask rows beyond the valid length (only the last tile) ----
-        if (tail) {
+        // ---- mask keys a row may not see (only in the last tiles of a sequence) ----
+        if (masked) {
 #pragma unroll
             for (int nt = 0; nt < kNT; ++nt) {
                 const int key = tile_key0 + nt * 8 + 2 * tq;
-                if (key >= k_end) sacc[nt][0] = sacc[nt][2] = -INFINITY;
-                if (key + 1 >= k_end) sacc[nt][1] = sacc[nt][3] = -INFINITY;
+                if (key >= lim_a) sacc[nt][0] = -INFINITY;
+                if (key + 1 >= lim_a) sacc[nt][1] = -INFINITY;
+                if (key >= lim_b) sacc[nt][2] = -INFINITY;
+                if (key + 1 >= lim_b) sacc[nt][3] = -INFINITY;
             }
         }
         // ---- online softmax (log2 domain), rows a and b ----
@@ -309,7 +323,7 @@ __global__ void __maxnreg__(200)
     }
     asm volatile("bar.sync 1, 128;" ::: "memory");
     if (!ok) return;
-    for (int idx = threadIdx.x; idx < p.G * D; idx += 128) {
+    for (int idx = threadIdx.x; idx < R * D; idx += 128) {
         const int row = idx / D, d = idx % D;
         const int blk = row >> 4, rr = row & 15;
         float M = -INFINITY;
@@ -324,21 +338,20 @@ __global__ void __maxnreg__(200)
             Lsum += sm_l[ww * 16 + rr] * sc;
             acc += sm_o[(ww * 16 + rr) * D + d] * sc;
         }
-        const int h = g * p.G + row;
-        const size_t prow = (static_cast<size_t>(b) * p.Hq + h) * p.n_splits + split;
+        const size_t prow = (group_row0 + row) * p.n_splits + split;
         p.o_part[prow * D + d] = (Lsum > 0.0f) ? acc / Lsum : 0.0f;
         if (d == 0) p.lse_part[prow] = (Lsum > 0.0f) ? M + __log2f(Lsum) : -INFINITY;
     }
 }
 
-// One warp per (b, h): out = sum_s 2^(lse_s - lse) O_s,  lse = log2 sum_s 2^lse_s.
+// One warp per query row: out = sum_s 2^(lse_s - lse) O_s,  lse = log2 sum_s 2^lse_s.
 template <int D>
 __global__ void __launch_bounds__(128)
     attn_decode_combine_kernel(const DecodeParams p, __nv_bfloat16* out, float* lse) {
     const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
-    if (row >= p.B * p.Hq) return;
-    const int b = row / p.Hq;
+    if (row >= p.B * p.Hq * p.Lq) return;
+    const int b = row / (p.Hq * p.Lq);
     const int seqlen = decode_seqlen(p, b);
     const int n_valid = (seqlen + p.chunk - 1) / p.chunk;
     const float* lp = p.lse_part + static_cast<size_t>(row) * p.n_splits;

@@ -131,6 +131,38 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, const i
                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * attn_decode_mq_workspace_size -- bytes of scratch attn_decode_mq needs for
+ * these sizes.  Depends only on the arguments; 0 for sizes it would reject.
+ */
+size_t attn_decode_mq_workspace_size(int B, int Hq, int Hkv, int Lq, int Lmax, int D);
+
+/*
+ * attn_decode_mq -- Lq >= 1 new tokens per sequence against a KV cache: the
+ * verify step of speculative decoding, or a small chunk of new tokens.
+ *
+ * The SDPA / FlashAttention selection guide's is_causal section works this
+ * case out for two queries (its L = 2 rows: "the verify step of speculative
+ * decoding or chunked prefill"): the new tokens' K/V are already the last Lq
+ * rows of the cache, and the mask must be aligned bottom-right.  So with
+ * n = seqlens[b], new token i (0-based) of sequence b sees cache rows
+ * 0 .. n - Lq + i; a token that sees no row (n < Lq - i) gets O = 0 and
+ * LSE = -inf.  Lq = 1 is exactly attn_decode.
+ *
+ *   q        [B, Hq, Lq, D]      bf16, read
+ *   k_cache, v_cache, seqlens    as attn_decode (rows >= seqlens[b] unused)
+ *   out      [B, Hq, Lq, D]      bf16, written
+ *   lse      [B, Hq, Lq]         fp32, written; may be NULL
+ *   workspace: at least attn_decode_mq_workspace_size(...) bytes, as attn_decode
+ *   D: 64 or 128.  G * Lq <= 64 (G = Hq / Hkv).
+ *
+ * Errors: as attn_decode, plus ATTN_ERR_INVALID_ARG for Lq < 1 and
+ * ATTN_ERR_UNSUPPORTED for G * Lq > 64.
+ */
+int attn_decode_mq(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,
+                   void* out, float* lse, int B, int Hq, int Hkv, int Lq, int Lmax, int D, float scale,
+                   void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * attn_decode_noalloc -- attn_decode for callers that cannot allocate device
  * memory: the split partials live in a scratch array that the library itself
  * declares at file scope (ATTN_DECODE_NOALLOC_SCRATCH_BYTES per GPU, reserved

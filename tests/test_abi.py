@@ -119,3 +119,28 @@ def test_missing_library_raises(monkeypatch, tmp_path):
     monkeypatch.setattr(_native, "LIB_PATH", str(tmp_path / "absent.so"))
     with pytest.raises(RuntimeError, match="no fallback"):
         _native.lib()
+
+
+def _decode_mq(lib, **kw):
+    args = dict(q=A, k=A, v=A, sl=A, out=A, lse=NULL, B=2, Hq=8, Hkv=2, Lq=4, Lmax=64, D=128, scale=0.1, ws=A,
+                wsb=1 << 30)
+    args.update(kw)
+    return lib.attn_decode_mq(args["q"], args["k"], args["v"], args["sl"], args["out"], args["lse"], args["B"],
+                              args["Hq"], args["Hkv"], args["Lq"], args["Lmax"], args["D"], args["scale"], args["ws"],
+                              args["wsb"], None)
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(Lq=0), -1), (dict(Lq=-2), -1), (dict(sl=NULL), -1), (dict(Hq=6, Hkv=4), -1), (dict(D=80), -2),
+    (dict(Lq=17), -2), (dict(Hq=64, Hkv=1, Lq=2), -2), (dict(ws=NULL), -3), (dict(wsb=100), -3),
+])
+def test_decode_mq_rejects(lib, bad, code):
+    assert _decode_mq(lib, **bad) == code
+
+
+def test_decode_mq_workspace(lib):
+    f = lib.attn_decode_mq_workspace_size
+    assert f(2, 8, 2, 0, 64, 128) == 0
+    assert f(2, 8, 2, 17, 64, 128) == 0          # G * Lq > 64
+    assert f(2, 8, 2, 1, 1000, 128) == lib.attn_decode_workspace_size(2, 8, 2, 1000, 128)
+    assert f(2, 8, 2, 4, 1000, 128) >= 4 * lib.attn_decode_workspace_size(2, 8, 2, 1000, 128) - 1024
