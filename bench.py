@@ -376,6 +376,37 @@ def run_sweeps(attn, dev, stream, seed, max_over_ranks):
                                "l2": "L2 flushed (256 MB write) before each timed call" if small else
                                      "inputs larger than L2"})
         del q, k, v, o, l
+    # the Qwen3-8B decode batch again, its cache in 128-row pages handed out in shuffled order
+    shape = DECODE
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed + 77)
+    gcpu = torch.Generator().manual_seed(seed)
+    sl = torch.randint(shape.seqlen_lo, shape.seqlen_hi + 1, (shape.B,), generator=gcpu).to(torch.int32)
+    page = 128
+    per = [-(-int(n) // page) for n in sl]
+    n_pages = sum(per)
+    kp = torch.randn((n_pages, shape.Hkv, page, shape.D), generator=g, device=dev).to(torch.bfloat16)
+    vp = torch.randn((n_pages, shape.Hkv, page, shape.D), generator=g, device=dev).to(torch.bfloat16)
+    perm = torch.randperm(n_pages, generator=gcpu).to(torch.int32)
+    table = torch.zeros((shape.B, max(per)), dtype=torch.int32)
+    o0 = 0
+    for b_, n_ in enumerate(per):
+        table[b_, :n_] = perm[o0:o0 + n_]
+        o0 += n_
+    table, sl_d = table.to(dev), sl.to(dev)
+    dq = torch.randn((shape.B, shape.Hq, 1, shape.D), generator=g, device=dev).to(torch.bfloat16)
+    o = torch.empty_like(dq)
+    l = torch.empty((shape.B, shape.Hq, 1), dtype=torch.float32, device=dev)
+    ws = torch.empty(attn.decode_workspace_size(shape.B, shape.Hq, shape.Hkv, page * table.shape[1], shape.D) + 4096,
+                     dtype=torch.uint8, device=dev)
+    ms = max_over_ranks(_time_calls(lambda: attn.decode_paged(dq, kp, vp, table, sl_d, scale=shape.scale, out=o, lse=l,
+                                                               workspace=ws, stream=stream), stream, n=10))
+    by = RL.decode_bytes(sl.tolist(), shape.B, shape.Hq, shape.Hkv, shape.D)
+    out["decode_paged"] = {"workload": shape.name + ", 128-row pages in shuffled order", "ms": round(ms, 4),
+                           "gbs": round(by / ms / 1e6, 1),
+                           "frac_of_measured_hbm": round(by / ms / 1e6 / float(peaks["hbm_gbs"]), 4)}
+    del kp, vp, dq, o, l, ws, table
+    torch.cuda.empty_cache()
     for G in W.GROUP_SWEEP:
         shape = W.group_sweep_decode(G)
         dq, dk, dv, dsl = W.decode_inputs_for(shape, seed=seed + G, device=dev)

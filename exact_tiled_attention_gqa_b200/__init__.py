@@ -9,6 +9,8 @@ Two calls, both thin wrappers over the C ABI in ``include/attn_gqa.h``:
 * ``decode_mq(q, k_cache, v_cache, seqlens)`` -- Lq new tokens per sequence
   (q [B,Hq,Lq,D]), the last Lq rows of the cache, bottom-right causal: the
   verify step of speculative decoding.
+* ``decode_paged(q, k_pages, v_pages, block_table, seqlens)`` -- decode_mq over
+  a paged cache: pools [n_pages,Hkv,page_size,D] and a block table [B,max_pages].
 
 Both return ``(out, lse)``: out bf16 shaped like q, lse fp32 (natural log).
 PyTorch supplies device memory and the current stream; every step of the
@@ -25,7 +27,7 @@ import torch
 from . import _native
 from ._native import AttnError
 
-__all__ = ["prefill", "decode", "decode_mq", "decode_noalloc", "decode_workspace_size",
+__all__ = ["prefill", "decode", "decode_mq", "decode_paged", "decode_noalloc", "decode_workspace_size",
            "decode_mq_workspace_size", "device_error", "AttnError", "library_path"]
 
 
@@ -147,6 +149,47 @@ def decode_mq(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, seq
                                           _ptr(lse), B, Hq, Hkv, Lq, Lmax, D, float(scale), _ptr(workspace),
                                           workspace.numel(), _stream_handle(stream))
     _native.check(st, "attn_decode_mq")
+    return out, lse
+
+
+def decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, block_table: torch.Tensor,
+                 seqlens: torch.Tensor, *, scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                 lse: Optional[torch.Tensor] = None, want_lse: bool = True, workspace: Optional[torch.Tensor] = None,
+                 stream=None):
+    """Paged-cache decode.  q [B,Hq,Lq,D] (or [B,Hq,D] for Lq = 1), pools [n_pages,Hkv,page_size,D],
+    block_table int32 [B,max_pages], seqlens int32 [B], all on one CUDA device."""
+    squeeze = q.dim() == 3
+    if squeeze:
+        q = q.unsqueeze(2)
+    _check_tensor("q", q, torch.bfloat16, 4)
+    _check_tensor("k_pages", k_pages, torch.bfloat16, 4)
+    _check_tensor("v_pages", v_pages, torch.bfloat16, 4)
+    _check_tensor("block_table", block_table, torch.int32, 2)
+    _check_tensor("seqlens", seqlens, torch.int32, 1)
+    B, Hq, Lq, D = q.shape
+    n_pages, Hkv, page_size = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
+    max_pages = block_table.shape[1]
+    if (k_pages.shape[3] != D or v_pages.shape != k_pages.shape or block_table.shape[0] != B
+            or seqlens.shape[0] != B):
+        raise ValueError("shape mismatch between q, the page pools, block_table and seqlens")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    need = int(_native.lib().attn_decode_paged_workspace_size(B, Hq, Hkv, Lq, page_size, max_pages, D))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    with torch.cuda.device(q.device):
+        st = _native.lib().attn_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table),
+                                             _ptr(seqlens), _ptr(out), _ptr(lse), B, Hq, Hkv, Lq, n_pages, page_size,
+                                             max_pages, D, float(scale), _ptr(workspace), workspace.numel(),
+                                             _stream_handle(stream))
+    _native.check(st, "attn_decode_paged")
+    if squeeze:
+        out = out.squeeze(2)
+        lse = None if lse is None else lse.squeeze(2)
     return out, lse
 
 

@@ -20,6 +20,7 @@ ATTN_ERR_WORKSPACE = -3
 ATTN_ERR_CUDA = -4
 ATTN_DEVERR_TIMEOUT = 0x1
 ATTN_DEVERR_SEQLEN = 0x2
+ATTN_DEVERR_PAGE = 0x4
 ATTN_DECODE_NOALLOC_SCRATCH_BYTES = 16 << 20
 
 # name -> (restype, argtypes): every symbol the header declares
@@ -31,6 +32,9 @@ SIGNATURES = {
     "attn_decode_mq_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32]),
     "attn_decode_mq": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _sz,
                               _vp]),
+    "attn_decode_paged_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32, _i32]),
+    "attn_decode_paged": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
+                                 _f32, _vp, _sz, _vp]),
     "attn_decode_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp]),
     "attn_selftest_exp2": (_i32, [_vp, _vp, _i32, _vp]),
     "attn_status_string": (ctypes.c_char_p, [_i32]),

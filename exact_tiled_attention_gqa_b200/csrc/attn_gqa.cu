@@ -168,16 +168,25 @@ int launch_decode_split(const CUtensorMap& tk, const CUtensorMap& tv, const Deco
     return check_launch("attn_decode_split_kernel");
 }
 
+// Paged cache description (block_table == nullptr: the contiguous layout).
+struct PagedKV {
+    const int32_t* block_table = nullptr;
+    int page_size = 0, max_pages = 0, n_pages = 0;
+};
+
 template <int D>
 int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* seqlens, void* out, float* lse, int B,
-                  int Hq, int Hkv, int Lmax, float scale, void* workspace, cudaStream_t stream, int Lq = 1) {
+                  int Hq, int Hkv, int Lmax, float scale, void* workspace, cudaStream_t stream, int Lq = 1,
+                  PagedKV paged = PagedKV()) {
     const DecodeLayout lay = decode_layout(B, Hq, Hkv, Lmax, D, Lq);
     CUtensorMap tk, tv;
     int st;
-    if ((st = encode_bf16_3d(&tk, kc, D, Lmax, static_cast<uint64_t>(B) * Hkv, 64, kDecKT, 1, "k_cache")) != ATTN_OK)
-        return st;
-    if ((st = encode_bf16_3d(&tv, vc, D, Lmax, static_cast<uint64_t>(B) * Hkv, 64, kDecKT, 1, "v_cache")) != ATTN_OK)
-        return st;
+    // the [outer, rows, D] view TMA reads boxes of 64 rows from
+    const uint64_t view_rows = paged.block_table ? static_cast<uint64_t>(paged.page_size) : static_cast<uint64_t>(Lmax);
+    const uint64_t view_outer = paged.block_table ? static_cast<uint64_t>(paged.n_pages) * Hkv
+                                                  : static_cast<uint64_t>(B) * Hkv;
+    if ((st = encode_bf16_3d(&tk, kc, D, view_rows, view_outer, 64, kDecKT, 1, "k_cache")) != ATTN_OK) return st;
+    if ((st = encode_bf16_3d(&tv, vc, D, view_rows, view_outer, 64, kDecKT, 1, "v_cache")) != ATTN_OK) return st;
     DecodeParams prm;
     prm.q = static_cast<const __nv_bfloat16*>(q);
     prm.seqlens = seqlens;
@@ -189,6 +198,10 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
     prm.Lmax = Lmax;
     prm.G = Hq / Hkv;
     prm.Lq = Lq;
+    prm.block_table = paged.block_table;
+    prm.page_size = paged.page_size;
+    prm.max_pages = paged.max_pages;
+    prm.n_pages = paged.n_pages;
     prm.chunk = lay.chunk;
     prm.n_splits = lay.n_splits;
     prm.scale_log2 = scale * kLog2e;
@@ -336,6 +349,54 @@ extern "C" int attn_decode_mq(const void* q, const void* k_cache, const void* v_
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     st = (D == 128) ? launch_decode<128>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s, Lq)
                     : launch_decode<64>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s, Lq);
+    return st == ATTN_OK ? ok() : st;
+}
+
+extern "C" size_t attn_decode_paged_workspace_size(int B, int Hq, int Hkv, int Lq, int page_size, int max_pages,
+                                                    int D) {
+    if (page_size < 64 || page_size % 64 != 0 || max_pages < 1 ||
+        static_cast<long long>(page_size) * max_pages > 0x7fffffffLL)
+        return 0;
+    return attn_decode_mq_workspace_size(B, Hq, Hkv, Lq, page_size * max_pages, D);
+}
+
+extern "C" int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
+                                 const int32_t* seqlens, void* out, float* lse, int B, int Hq, int Hkv, int Lq,
+                                 int n_pages, int page_size, int max_pages, int D, float scale, void* workspace,
+                                 size_t workspace_bytes, void* stream) {
+    if (page_size < 64 || page_size % 64 != 0)
+        return fail(ATTN_ERR_INVALID_ARG, "page_size=%d must be a positive multiple of 64", page_size);
+    if (n_pages < 1 || max_pages < 1) return fail(ATTN_ERR_INVALID_ARG, "n_pages and max_pages must be >= 1");
+    if (static_cast<long long>(page_size) * max_pages > 0x7fffffffLL ||
+        static_cast<long long>(n_pages) * Hkv > 0x7fffffffLL)
+        return fail(ATTN_ERR_UNSUPPORTED, "page pool too large");
+    const int Lmax = page_size * max_pages;   // the longest sequence the block table can describe
+    int st = check_common(q, k_pages, v_pages, out, lse, B, Hq, Hkv, Lq, Lmax, D, scale, "Lq", "Lmax");
+    if (st != ATTN_OK) return st;
+    if (Lq < 1) return fail(ATTN_ERR_INVALID_ARG, "Lq must be >= 1");
+    if (B > 0 && (!seqlens || !block_table)) return fail(ATTN_ERR_INVALID_ARG, "null seqlens or block_table");
+    if ((reinterpret_cast<uintptr_t>(seqlens) | reinterpret_cast<uintptr_t>(block_table)) & 3u)
+        return fail(ATTN_ERR_INVALID_ARG, "seqlens and block_table must be 4-byte aligned");
+    if (static_cast<long long>(Hq / Hkv) * Lq > 64)
+        return fail(ATTN_ERR_UNSUPPORTED, "G * Lq = %lld query rows per KV head (built: up to 64)",
+                    static_cast<long long>(Hq / Hkv) * Lq);
+    if (static_cast<long long>(B) * Hq * Lq > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "B*Hq*Lq too large");
+    if (B == 0) return ok();
+    const size_t need = decode_layout(B, Hq, Hkv, Lmax, D, Lq).total;
+    if (!workspace || workspace_bytes < need)
+        return fail(ATTN_ERR_WORKSPACE, "decode workspace needs %zu bytes, got %zu", need,
+                    workspace ? workspace_bytes : static_cast<size_t>(0));
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+        return fail(ATTN_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    PagedKV pg;
+    pg.block_table = block_table;
+    pg.page_size = page_size;
+    pg.max_pages = max_pages;
+    pg.n_pages = n_pages;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    st = (D == 128)
+             ? launch_decode<128>(q, k_pages, v_pages, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s, Lq, pg)
+             : launch_decode<64>(q, k_pages, v_pages, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s, Lq, pg);
     return st == ATTN_OK ? ok() : st;
 }
 

@@ -25,6 +25,16 @@
 //
 // Splitting the cache length and merging by log-sum-exp is the single-GPU
 // form of the KV parallelism on the NVIDIA page ("Parameter four").
+//
+// Two cache layouts share these kernels:
+//   contiguous  K/V [B, Hkv, Lmax, D]; a tile of rows r .. r+63 of (b, g) is
+//               TMA box (0/64, r, b * Hkv + g) of the [B*Hkv, Lmax, D] view.
+//   paged       K/V pools [n_pages, Hkv, page_size, D] and a block table
+//               [B, max_pages]: logical row r of sequence b lives in page
+//               block_table[b][r / page_size] at row r % page_size.  page_size
+//               is a multiple of 64, so a tile never straddles two pages; the
+//               box is (0/64, r % page_size, page * Hkv + g) of the
+//               [n_pages*Hkv, page_size, D] view.
 #pragma once
 
 #include "ptx_sm100.cuh"
@@ -58,6 +68,8 @@ struct DecodeParams {
     float* lse_part;          // [B,Hq,Lq,n_splits] (log2 domain)
     int B, Hq, Hkv, Lmax, G;
     int Lq;                   // new query rows per sequence (1 = plain decode)
+    const int* block_table;   // [B, max_pages] for the paged layout, nullptr for the contiguous one
+    int page_size, max_pages, n_pages;
     int chunk;                // cache rows per split (multiple of 64)
     int n_splits;
     float scale_log2;
@@ -116,18 +128,28 @@ __global__ void __maxnreg__(200)
         if (lane == 0) {
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
-            const int kv_row = b * p.Hkv + g;
             int issued = 0;
             for (int t = 0; t < n_tiles; ++t) {
                 const int s = t % L::kStages;
                 const uint32_t round = static_cast<uint32_t>(t / L::kStages);
+                // where rows k_begin + 64 t .. + 63 of (b, g) live
+                const int key0 = k_begin + t * kDecKT;
+                int row = key0, outer = b * p.Hkv + g;
+                if (p.block_table != nullptr) {
+                    int page = __ldg(p.block_table + static_cast<size_t>(b) * p.max_pages + key0 / p.page_size);
+                    if (page < 0 || page >= p.n_pages) {   // the tile would read another tenant's rows
+                        atomicOr(&g_attn_err, kDevErrPage);
+                        page = 0;
+                    }
+                    row = key0 % p.page_size;
+                    outer = page * p.Hkv + g;
+                }
                 if (!mbar_wait(bar_empty(s), (round & 1u) ^ 1u, abort_flag, &g_attn_err, kDevErrTimeout)) break;
                 mbar_arrive_expect_tx(bar_full(s), L::kStageBytes);
                 const uint32_t dst = ring + s * L::kStageBytes;
                 for (int kb = 0; kb < L::kKB; ++kb) {
-                    tma_load_3d(dst + kb * L::kBlockBytes, &tm_k, bar_full(s), kb * 64, k_begin + t * kDecKT, kv_row);
-                    tma_load_3d(dst + L::kTileBytes + kb * L::kBlockBytes, &tm_v, bar_full(s), kb * 64,
-                                k_begin + t * kDecKT, kv_row);
+                    tma_load_3d(dst + kb * L::kBlockBytes, &tm_k, bar_full(s), kb * 64, row, outer);
+                    tma_load_3d(dst + L::kTileBytes + kb * L::kBlockBytes, &tm_v, bar_full(s), kb * 64, row, outer);
                 }
                 issued = t + 1;
             }

@@ -163,6 +163,42 @@ int attn_decode_mq(const void* q, const void* k_cache, const void* v_cache, cons
                    void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * attn_decode_paged_workspace_size -- bytes of scratch attn_decode_paged needs;
+ * 0 for sizes it would reject.
+ */
+size_t attn_decode_paged_workspace_size(int B, int Hq, int Hkv, int Lq, int page_size, int max_pages, int D);
+
+/*
+ * attn_decode_paged -- attn_decode_mq over a paged KV cache: the cache lives
+ * in fixed-size pages of a shared pool, and a block table says which pages
+ * hold each sequence (the layout serving engines use so that sequences can
+ * grow without copying).  The arithmetic is that of attn_decode_mq; only
+ * where cache row r of sequence b is read from changes:
+ *
+ *   row r of sequence b, KV head g  =  k_pages[block_table[b][r / page_size], g, r % page_size, :]
+ *
+ *   q            [B, Hq, Lq, D]                  bf16, read
+ *   k_pages      [n_pages, Hkv, page_size, D]    bf16, read (pages not in use may hold anything)
+ *   v_pages      [n_pages, Hkv, page_size, D]    bf16, read
+ *   block_table  [B, max_pages]                  int32 in device memory; entries for the pages
+ *                                                a sequence uses must lie in [0, n_pages); one
+ *                                                outside is replaced by page 0 and flags
+ *                                                ATTN_DEVERR_PAGE
+ *   seqlens      [B]                             int32 in device memory, each in
+ *                                                [0, page_size * max_pages]
+ *   out          [B, Hq, Lq, D] bf16;  lse [B, Hq, Lq] fp32 or NULL
+ *   page_size: a positive multiple of 64.  D: 64 or 128.  G * Lq <= 64.
+ *
+ * Errors: as attn_decode_mq, plus ATTN_ERR_INVALID_ARG for a page_size that
+ * is not a positive multiple of 64, n_pages or max_pages < 1, or a null
+ * block_table.
+ */
+int attn_decode_paged(const void* q, const void* k_pages, const void* v_pages, const int32_t* block_table,
+                      const int32_t* seqlens, void* out, float* lse, int B, int Hq, int Hkv, int Lq, int n_pages,
+                      int page_size, int max_pages, int D, float scale, void* workspace, size_t workspace_bytes,
+                      void* stream);
+
+/*
  * attn_decode_noalloc -- attn_decode for callers that cannot allocate device
  * memory: the split partials live in a scratch array that the library itself
  * declares at file scope (ATTN_DECODE_NOALLOC_SCRATCH_BYTES per GPU, reserved
@@ -219,6 +255,7 @@ const char* attn_last_error(void);
  */
 #define ATTN_DEVERR_TIMEOUT 0x1u  /* a pipeline wait gave up after ~2 s */
 #define ATTN_DEVERR_SEQLEN  0x2u  /* a seqlens value was outside [0, Lmax] */
+#define ATTN_DEVERR_PAGE    0x4u  /* a block_table entry was outside [0, n_pages) */
 
 /*
  * attn_device_error -- synchronise the current device, copy its error word

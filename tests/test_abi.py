@@ -144,3 +144,16 @@ def test_decode_mq_workspace(lib):
     assert f(2, 8, 2, 17, 64, 128) == 0          # G * Lq > 64
     assert f(2, 8, 2, 1, 1000, 128) == lib.attn_decode_workspace_size(2, 8, 2, 1000, 128)
     assert f(2, 8, 2, 4, 1000, 128) >= 4 * lib.attn_decode_workspace_size(2, 8, 2, 1000, 128) - 1024
+
+
+def test_decode_paged_rejects(lib):
+    f = lambda **kw: lib.attn_decode_paged(
+        kw.get("q", A), A, A, kw.get("bt", A), A, A, None, 2, 8, 2, kw.get("Lq", 1), kw.get("n_pages", 16),
+        kw.get("ps", 128), kw.get("mp", 8), 128, 0.1, A, 1 << 30, None)
+    assert f(ps=96) == -1 and f(ps=0) == -1 and f(ps=-64) == -1
+    assert f(n_pages=0) == -1 and f(mp=0) == -1
+    assert f(bt=NULL) == -1
+    assert f(Lq=0) == -1
+    assert lib.attn_decode_paged_workspace_size(2, 8, 2, 1, 96, 8, 128) == 0
+    assert lib.attn_decode_paged_workspace_size(2, 8, 2, 1, 128, 8, 128) == \
+        lib.attn_decode_mq_workspace_size(2, 8, 2, 1, 1024, 128)
