@@ -15,6 +15,7 @@
 
 #include "../../include/attn_gqa.h"
 #include "decode_sm100.cuh"
+#include "decode_tc_sm100.cuh"
 #include "prefill_sm100.cuh"
 
 namespace attn {
@@ -208,7 +209,19 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
     if (prm.n_splits > 65535 || Hkv > 65535 || B > 65535)
         return fail(ATTN_ERR_UNSUPPORTED, "decode grid (%d, %d, %d) exceeds launch limits", prm.n_splits, Hkv, B);
     const int rows_per_group = prm.G * Lq;
-    if (rows_per_group <= 16)
+    if (rows_per_group > 16) {
+        // many query rows per cache row: the tcgen05 split kernel (decode_tc_sm100.cuh)
+        static int smem_done_tc[64];
+        using LT = DecodeTcSmem<D>;
+        CUtensorMap tq;
+        if ((st = encode_bf16_3d(&tq, q, D, static_cast<uint64_t>(B) * Hq * Lq, 1, 64, rows_per_group, 1, "q")) !=
+            ATTN_OK)
+            return st;
+        if ((st = ensure_smem(attn_decode_tc_kernel<D>, LT::kAlloc, smem_done_tc)) != ATTN_OK) return st;
+        dim3 grid(prm.n_splits, prm.Hkv, prm.B);
+        attn_decode_tc_kernel<D><<<grid, kDtcThreads, LT::kAlloc, stream>>>(tq, tk, tv, prm);
+        st = check_launch("attn_decode_tc_kernel");
+    } else if (rows_per_group <= 16)
         st = launch_decode_split<D, 16>(tk, tv, prm, stream);
     else if (rows_per_group <= 32)
         st = launch_decode_split<D, 32>(tk, tv, prm, stream);
@@ -266,7 +279,7 @@ extern "C" int attn_prefill(const void* q, const void* k, const void* v, void* o
 }
 
 extern "C" size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int D) {
-    if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Lmax < 1 || (D != 64 && D != 128) || Hq / Hkv > 64)
+    if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Lmax < 1 || (D != 64 && D != 128) || Hq / Hkv > 128)
         return 0;
     if (B == 0) return 0;
     return decode_layout(B, Hq, Hkv, Lmax, D).total;
@@ -280,7 +293,7 @@ extern "C" int attn_decode(const void* q, const void* k_cache, const void* v_cac
     if (!seqlens && B > 0) return fail(ATTN_ERR_INVALID_ARG, "null seqlens");
     if (reinterpret_cast<uintptr_t>(seqlens) & 3u) return fail(ATTN_ERR_INVALID_ARG, "seqlens must be 4-byte aligned");
     if (Lmax < 1) return fail(ATTN_ERR_INVALID_ARG, "Lmax must be >= 1");
-    if (Hq / Hkv > 64) return fail(ATTN_ERR_UNSUPPORTED, "decode group size G=%d > 64", Hq / Hkv);
+    if (Hq / Hkv > 128) return fail(ATTN_ERR_UNSUPPORTED, "decode group size G=%d > 128", Hq / Hkv);
     if (static_cast<long long>(B) * Hq > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "B*Hq too large");
     if (B == 0) return ok();
     const size_t need = decode_layout(B, Hq, Hkv, Lmax, D).total;
@@ -320,7 +333,7 @@ extern "C" int attn_selftest_exp2(const float* x, float* y, int n, void* stream)
 
 extern "C" size_t attn_decode_mq_workspace_size(int B, int Hq, int Hkv, int Lq, int Lmax, int D) {
     if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Lmax < 1 || Lq < 1 || (D != 64 && D != 128) ||
-        static_cast<long long>(Hq / Hkv) * Lq > 64)
+        static_cast<long long>(Hq / Hkv) * Lq > 128)
         return 0;
     if (B == 0) return 0;
     return decode_layout(B, Hq, Hkv, Lmax, D, Lq).total;
@@ -335,8 +348,8 @@ extern "C" int attn_decode_mq(const void* q, const void* k_cache, const void* v_
     if (!seqlens && B > 0) return fail(ATTN_ERR_INVALID_ARG, "null seqlens");
     if (reinterpret_cast<uintptr_t>(seqlens) & 3u) return fail(ATTN_ERR_INVALID_ARG, "seqlens must be 4-byte aligned");
     if (Lmax < 1) return fail(ATTN_ERR_INVALID_ARG, "Lmax must be >= 1");
-    if (static_cast<long long>(Hq / Hkv) * Lq > 64)
-        return fail(ATTN_ERR_UNSUPPORTED, "G * Lq = %lld query rows per KV head (built: up to 64)",
+    if (static_cast<long long>(Hq / Hkv) * Lq > 128)
+        return fail(ATTN_ERR_UNSUPPORTED, "G * Lq = %lld query rows per KV head (built: up to 128)",
                     static_cast<long long>(Hq / Hkv) * Lq);
     if (static_cast<long long>(B) * Hq * Lq > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "B*Hq*Lq too large");
     if (B == 0) return ok();
@@ -377,8 +390,8 @@ extern "C" int attn_decode_paged(const void* q, const void* k_pages, const void*
     if (B > 0 && (!seqlens || !block_table)) return fail(ATTN_ERR_INVALID_ARG, "null seqlens or block_table");
     if ((reinterpret_cast<uintptr_t>(seqlens) | reinterpret_cast<uintptr_t>(block_table)) & 3u)
         return fail(ATTN_ERR_INVALID_ARG, "seqlens and block_table must be 4-byte aligned");
-    if (static_cast<long long>(Hq / Hkv) * Lq > 64)
-        return fail(ATTN_ERR_UNSUPPORTED, "G * Lq = %lld query rows per KV head (built: up to 64)",
+    if (static_cast<long long>(Hq / Hkv) * Lq > 128)
+        return fail(ATTN_ERR_UNSUPPORTED, "G * Lq = %lld query rows per KV head (built: up to 128)",
                     static_cast<long long>(Hq / Hkv) * Lq);
     if (static_cast<long long>(B) * Hq * Lq > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "B*Hq*Lq too large");
     if (B == 0) return ok();
@@ -476,7 +489,7 @@ extern "C" int attn_decode_noalloc(const void* q, const void* k_cache, const voi
     if (!seqlens && B > 0) return fail(ATTN_ERR_INVALID_ARG, "null seqlens");
     if (reinterpret_cast<uintptr_t>(seqlens) & 3u) return fail(ATTN_ERR_INVALID_ARG, "seqlens must be 4-byte aligned");
     if (Lmax < 1) return fail(ATTN_ERR_INVALID_ARG, "Lmax must be >= 1");
-    if (Hq / Hkv > 64) return fail(ATTN_ERR_UNSUPPORTED, "decode group size G=%d > 64", Hq / Hkv);
+    if (Hq / Hkv > 128) return fail(ATTN_ERR_UNSUPPORTED, "decode group size G=%d > 128", Hq / Hkv);
     if (static_cast<long long>(B) * Hq > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "B*Hq too large");
     if (B == 0) return ok();
     const size_t need = decode_layout(B, Hq, Hkv, Lmax, D).total;

@@ -121,7 +121,7 @@ size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int D);
  *              bytes, 256-byte aligned, owned by the caller; its contents on
  *              entry do not matter and on return are unspecified.  Two calls
  *              in flight at once must not share one workspace.
- *   D: 64 or 128.  G = Hq / Hkv: 1 .. 64.  B == 0 returns ATTN_OK.
+ *   D: 64 or 128.  G = Hq / Hkv: 1 .. 128.  B == 0 returns ATTN_OK.
  *
  * Errors: as attn_prefill, plus ATTN_ERR_WORKSPACE for a null or too small
  * workspace.
@@ -153,10 +153,10 @@ size_t attn_decode_mq_workspace_size(int B, int Hq, int Hkv, int Lq, int Lmax, i
  *   out      [B, Hq, Lq, D]      bf16, written
  *   lse      [B, Hq, Lq]         fp32, written; may be NULL
  *   workspace: at least attn_decode_mq_workspace_size(...) bytes, as attn_decode
- *   D: 64 or 128.  G * Lq <= 64 (G = Hq / Hkv).
+ *   D: 64 or 128.  G * Lq <= 128 (G = Hq / Hkv).
  *
  * Errors: as attn_decode, plus ATTN_ERR_INVALID_ARG for Lq < 1 and
- * ATTN_ERR_UNSUPPORTED for G * Lq > 64.
+ * ATTN_ERR_UNSUPPORTED for G * Lq > 128.
  */
 int attn_decode_mq(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,
                    void* out, float* lse, int B, int Hq, int Hkv, int Lq, int Lmax, int D, float scale,
@@ -187,7 +187,7 @@ size_t attn_decode_paged_workspace_size(int B, int Hq, int Hkv, int Lq, int page
  *   seqlens      [B]                             int32 in device memory, each in
  *                                                [0, page_size * max_pages]
  *   out          [B, Hq, Lq, D] bf16;  lse [B, Hq, Lq] fp32 or NULL
- *   page_size: a positive multiple of 64.  D: 64 or 128.  G * Lq <= 64.
+ *   page_size: a positive multiple of 64.  D: 64 or 128.  G * Lq <= 128.
  *
  * Errors: as attn_decode_mq, plus ATTN_ERR_INVALID_ARG for a page_size that
  * is not a positive multiple of 64, n_pages or max_pages < 1, or a null

@@ -88,7 +88,7 @@ def _decode(lib, **kw):
 
 @pytest.mark.parametrize("bad,code", [
     (dict(sl=NULL), -1), (dict(sl=ctypes.c_void_p(0x10001)), -1), (dict(Lmax=0), -1), (dict(Hq=5, Hkv=2), -1),
-    (dict(k=NULL), -1), (dict(D=32), -2), (dict(Hq=128, Hkv=1), -2), (dict(ws=NULL), -3), (dict(wsb=16), -3),
+    (dict(k=NULL), -1), (dict(D=32), -2), (dict(Hq=256, Hkv=1), -2), (dict(ws=NULL), -3), (dict(wsb=16), -3),
     (dict(ws=ctypes.c_void_p(0x10010)), -1),
 ])
 def test_decode_rejects(lib, bad, code):
@@ -106,7 +106,7 @@ def test_workspace_size(lib):
     assert f(2, 8, 3, 64, 128) == 0        # Hq % Hkv
     assert f(2, 8, 2, 64, 96) == 0         # D
     assert f(2, 8, 2, 0, 128) == 0         # Lmax
-    assert f(1, 128, 1, 64, 128) == 0      # G > 64
+    assert f(1, 256, 1, 64, 128) == 0      # G > 128
     a = f(2, 8, 2, 1000, 128)
     assert a > 0 and a % 256 == 0
     assert f(2, 8, 2, 100000, 128) >= a
@@ -132,7 +132,7 @@ def _decode_mq(lib, **kw):
 
 @pytest.mark.parametrize("bad,code", [
     (dict(Lq=0), -1), (dict(Lq=-2), -1), (dict(sl=NULL), -1), (dict(Hq=6, Hkv=4), -1), (dict(D=80), -2),
-    (dict(Lq=17), -2), (dict(Hq=64, Hkv=1, Lq=2), -2), (dict(ws=NULL), -3), (dict(wsb=100), -3),
+    (dict(Lq=33), -2), (dict(Hq=64, Hkv=1, Lq=3), -2), (dict(ws=NULL), -3), (dict(wsb=100), -3),
 ])
 def test_decode_mq_rejects(lib, bad, code):
     assert _decode_mq(lib, **bad) == code
@@ -141,7 +141,7 @@ def test_decode_mq_rejects(lib, bad, code):
 def test_decode_mq_workspace(lib):
     f = lib.attn_decode_mq_workspace_size
     assert f(2, 8, 2, 0, 64, 128) == 0
-    assert f(2, 8, 2, 17, 64, 128) == 0          # G * Lq > 64
+    assert f(2, 8, 2, 33, 64, 128) == 0          # G * Lq > 128
     assert f(2, 8, 2, 1, 1000, 128) == lib.attn_decode_workspace_size(2, 8, 2, 1000, 128)
     assert f(2, 8, 2, 4, 1000, 128) >= 4 * lib.attn_decode_workspace_size(2, 8, 2, 1000, 128) - 1024
 

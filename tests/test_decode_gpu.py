@@ -47,10 +47,10 @@ def _check(oracle_mod, q, k, v, sl, what):
 
 
 @pytest.mark.parametrize("D", [64, 128])
-@pytest.mark.parametrize("G", [1, 2, 4, 8, 16, 32, 64, 3, 12, 24, 48])
+@pytest.mark.parametrize("G", [1, 2, 4, 8, 16, 32, 64, 128, 3, 12, 17, 24, 48, 96])
 def test_group_sizes(oracle_mod, D, G):
-    Hkv = 2
-    seqlens = [700, 1, 333, 64, 65]
+    Hkv = 2 if G <= 64 else 1
+    seqlens = [700, 1, 333, 64, 65, 129, 128, 127]
     q, k, v, sl = _inputs(len(seqlens), G * Hkv, Hkv, 700, D, seqlens, seed=G * 10 + D)
     _check(oracle_mod, q, k, v, sl, f"G{G} D{D}")
 
