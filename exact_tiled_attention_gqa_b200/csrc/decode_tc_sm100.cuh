@@ -243,11 +243,20 @@ __global__ void __launch_bounds__(kDtcThreads, 2)
         const float sl2 = p.scale_log2;
         const uint64_t sl2x2 = f2_pack(sl2, sl2);
         float m_run = -INFINITY, l_run = 0.0f;
+        // A warp whose 32 rows are all padding (row >= R) only keeps the pipeline
+        // moving: its P rows are never read into a real output row (the MMA keeps
+        // rows apart), so it skips the softmax and just signals.
+        const bool idle_warp = warp * 32 >= R;
         bool ok = true;
         for (int j = 0; j < n_tiles; ++j) {
             ok = mbar_wait(bar_s_full, static_cast<uint32_t>(j) & 1u, abort_flag, &g_attn_err, kDevErrTimeout);
             if (!ok) break;
             tc_fence_after_sync();
+            if (idle_warp) {
+                tc_fence_before_sync();
+                mbar_arrive(bar_p_full);
+                continue;
+            }
             const int key0 = k_begin + j * kDtcBN;
             const bool masked = key0 + kDtcBN > lim_lo;
             // pass 1: the row max of this tile
