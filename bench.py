@@ -62,6 +62,8 @@ def parse():
                     help="profiling aid: time one call type only (the JSON line is then partial)")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="profiling aid: use the first N sequences of the decode batch")
+    ap.add_argument("--decode-group", type=int, default=None,
+                    help="profiling aid: with --only decode, use the group-size sweep shape with this G")
     ap.add_argument("--no-sweeps", action="store_true",
                     help="skip the other workloads (group-size decode sweep, other prefill shapes)")
     return ap.parse_args()
@@ -156,6 +158,8 @@ def run_ours(args, rank, world, local_rank):
         q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
     if args.only == "prefill":
         dshape = W.DecodeShape(DECODE.name, 1, DECODE.Hq, DECODE.Hkv, 64, DECODE.D, 64, 64)
+    elif args.decode_group:
+        dshape = W.group_sweep_decode(args.decode_group)
     elif args.decode_batch:
         dshape = W.DecodeShape(DECODE.name + f" (first {args.decode_batch})", args.decode_batch, DECODE.Hq,
                                DECODE.Hkv, DECODE.Lmax, DECODE.D, DECODE.seqlen_lo, DECODE.seqlen_hi)
@@ -165,6 +169,8 @@ def run_ours(args, rank, world, local_rank):
         q_h, k_h, v_h = W.prefill_inputs(1, PREFILL.Hq, PREFILL.Hkv, 128, 128, PREFILL.D, seed=seed)
         q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
     dq, dk, dv, dsl = W.decode_inputs_for(dshape, seed=seed, device=dev)
+    if args.only is not None:
+        print(json.dumps({"profiling_workload": dshape.name if args.only == "decode" else PREFILL.name}), flush=True)
     seqlens_host = dsl.cpu()
     p_flops = RL.prefill_flops(PREFILL.B, PREFILL.Hq, PREFILL.Lq, PREFILL.Lk, PREFILL.D, PREFILL.is_causal)
     d_bytes = RL.decode_bytes(seqlens_host.tolist(), dshape.B, dshape.Hq, dshape.Hkv, dshape.D)
