@@ -365,11 +365,12 @@ def _time_calls(fn, stream, n_warm=2, n=10, flush=False):
 
 
 def run_sweeps(attn, dev, stream, seed, max_over_ranks):
-    """The other workloads: Qwen3-8B prefill B1 L4096, the chunked prefills, and the
-    group-size decode sweep (Hq=64, D=128, batch 8, 131072 keys, G = 1 .. 64)."""
+    """The other workloads: Qwen3-8B prefill B1 L4096, the chunked prefills, head dim
+    256 prefill and decode, the paged decode, and the group-size decode sweep
+    (Hq=64, D=128, batch 8, 131072 keys, G = 1 .. 64)."""
     peaks = RL.measured_peaks()
     out = {"prefill": [], "decode_group_sweep": []}
-    for shape in (W.QWEN_PREFILL_4K, W.CHUNKED_16K, W.CHUNKED_32K):
+    for shape in (W.QWEN_PREFILL_4K, W.CHUNKED_16K, W.CHUNKED_32K, W.HD256_PREFILL):
         q, k, v = (t.to(dev) for t in W.prefill_inputs_for(shape, seed=seed))
         o = torch.empty_like(q)
         l = torch.empty((shape.B, shape.Hq, shape.Lq), dtype=torch.float32, device=dev)
@@ -412,6 +413,19 @@ def run_sweeps(attn, dev, stream, seed, max_over_ranks):
                            "gbs": round(by / ms / 1e6, 1),
                            "frac_of_measured_hbm": round(by / ms / 1e6 / float(peaks["hbm_gbs"]), 4)}
     del kp, vp, dq, o, l, ws, table
+    torch.cuda.empty_cache()
+    shape = W.HD256_DECODE
+    dq, dk, dv, dsl = W.decode_inputs_for(shape, seed=seed + 256, device=dev)
+    o = torch.empty_like(dq)
+    l = torch.empty((shape.B, shape.Hq), dtype=torch.float32, device=dev)
+    ws = torch.empty(attn.decode_workspace_size(shape.B, shape.Hq, shape.Hkv, shape.Lmax, shape.D),
+                     dtype=torch.uint8, device=dev)
+    ms = max_over_ranks(_time_calls(lambda: attn.decode(dq, dk, dv, dsl, scale=shape.scale, out=o, lse=l,
+                                                         workspace=ws, stream=stream), stream, n=10))
+    by = RL.decode_bytes(dsl.cpu().tolist(), shape.B, shape.Hq, shape.Hkv, shape.D)
+    out["decode_hd256"] = {"workload": shape.name, "ms": round(ms, 4), "gbs": round(by / ms / 1e6, 1),
+                           "frac_of_measured_hbm": round(by / ms / 1e6 / float(peaks["hbm_gbs"]), 4)}
+    del dq, dk, dv, dsl, o, l, ws
     torch.cuda.empty_cache()
     for G in W.GROUP_SWEEP:
         shape = W.group_sweep_decode(G)

@@ -104,6 +104,7 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
                    int Lq, int Lk, float scale, int is_causal, cudaStream_t stream) {
     static int smem_done[64];
     using L = PrefillSmem<D>;
+    constexpr int NQ = L::kNQ;
     const int G = Hq / Hkv;
     const int P = kBM / G;
     CUtensorMap tq, tk, tv;
@@ -111,7 +112,7 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
     if ((st = encode_bf16_3d(&tq, q, D, Lq, static_cast<uint64_t>(B) * Hq, 64, P, G, "q")) != ATTN_OK) return st;
     if ((st = encode_bf16_3d(&tk, k, D, Lk, static_cast<uint64_t>(B) * Hkv, 64, kBN, 1, "k")) != ATTN_OK) return st;
     if ((st = encode_bf16_3d(&tv, v, D, Lk, static_cast<uint64_t>(B) * Hkv, 64, kBN, 1, "v")) != ATTN_OK) return st;
-    if ((st = ensure_smem(attn_prefill_sm100_kernel<D>, L::kAlloc, smem_done)) != ATTN_OK) return st;
+    if ((st = ensure_smem(attn_prefill_sm100_kernel<D, NQ>, L::kAlloc, smem_done)) != ATTN_OK) return st;
     PrefillParams prm;
     prm.out = out;
     prm.lse = lse;
@@ -122,12 +123,13 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
     prm.Lk = Lk;
     prm.G = G;
     prm.P = P;
-    prm.n_mblk = (Lq + 2 * P - 1) / (2 * P);
+    prm.n_mblk = (Lq + NQ * P - 1) / (NQ * P);
     prm.is_causal = is_causal ? 1 : 0;
     prm.scale_log2 = scale * kLog2e;
     const long long grid = static_cast<long long>(B) * Hkv * prm.n_mblk;
     if (grid > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "prefill grid too large (%lld CTAs)", grid);
-    attn_prefill_sm100_kernel<D><<<static_cast<unsigned>(grid), kPrefillThreads, L::kAlloc, stream>>>(tq, tk, tv, prm);
+    attn_prefill_sm100_kernel<D, NQ>
+        <<<static_cast<unsigned>(grid), prefill_threads<NQ>(), L::kAlloc, stream>>>(tq, tk, tv, prm);
     return check_launch("attn_prefill_sm100_kernel");
 }
 
@@ -140,9 +142,13 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
 #ifndef ATTN_TC_MIN_CHUNK
 #define ATTN_TC_MIN_CHUNK 2048
 #endif
-int decode_chunk(int B, int Hkv, int Lmax, int rows_per_group = 1) {
+// D = 256 always takes the tcgen05 kernel: a 256-wide O per row does not fit
+// the mma.sync kernel's registers.
+bool decode_uses_tc(int D, int rows_per_group) { return D == 256 || rows_per_group > 16; }
+
+int decode_chunk(int B, int Hkv, int Lmax, bool tc_path) {
     const long long target = 148LL * 2 * 4;
-    const int min_chunk = rows_per_group > 16 ? ATTN_TC_MIN_CHUNK : 256;
+    const int min_chunk = tc_path ? ATTN_TC_MIN_CHUNK : 256;
     int chunk = 4096;
     while (chunk > min_chunk && static_cast<long long>(B) * Hkv * ((Lmax + chunk - 1) / chunk) < target) chunk >>= 1;
     return chunk;
@@ -157,7 +163,7 @@ struct DecodeLayout {
 
 DecodeLayout decode_layout(int B, int Hq, int Hkv, int Lmax, int D, int Lq = 1) {
     DecodeLayout d;
-    d.chunk = decode_chunk(B, Hkv, Lmax, (Hq / Hkv) * Lq);
+    d.chunk = decode_chunk(B, Hkv, Lmax, decode_uses_tc(D, (Hq / Hkv) * Lq));
     d.n_splits = (Lmax + d.chunk - 1) / d.chunk;
     const size_t rows = static_cast<size_t>(B) * Hq * Lq * d.n_splits;
     d.o_bytes = align256(rows * D * sizeof(float));
@@ -217,7 +223,7 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
     if (prm.n_splits > 65535 || Hkv > 65535 || B > 65535)
         return fail(ATTN_ERR_UNSUPPORTED, "decode grid (%d, %d, %d) exceeds launch limits", prm.n_splits, Hkv, B);
     const int rows_per_group = prm.G * Lq;
-    if (rows_per_group > 16) {
+    if (decode_uses_tc(D, rows_per_group)) {
         // many query rows per cache row: the tcgen05 split kernel (decode_tc_sm100.cuh)
         static int smem_done_tc[64];
         using LT = DecodeTcSmem<D>;
@@ -229,6 +235,8 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
         dim3 grid(prm.n_splits, prm.Hkv, prm.B);
         attn_decode_tc_kernel<D><<<grid, kDtcThreads, LT::kAlloc, stream>>>(tq, tk, tv, prm);
         st = check_launch("attn_decode_tc_kernel");
+    } else if constexpr (D == 256) {
+        st = fail(ATTN_ERR_UNSUPPORTED, "unreachable");   // D = 256 always takes the branch above
     } else if (rows_per_group <= 16)
         st = launch_decode_split<D, 16>(tk, tv, prm, stream);
     else if (rows_per_group <= 32)
@@ -257,7 +265,7 @@ int check_common(const void* q, const void* k, const void* v, const void* out, c
         return fail(ATTN_ERR_INVALID_ARG, "tensor base addresses must be 16-byte aligned");
     if (lse && (reinterpret_cast<uintptr_t>(lse) & 3u))
         return fail(ATTN_ERR_INVALID_ARG, "lse must be 4-byte aligned");
-    if (D != 64 && D != 128) return fail(ATTN_ERR_UNSUPPORTED, "head dim D=%d (built: 64, 128)", D);
+    if (D != 64 && D != 128 && D != 256) return fail(ATTN_ERR_UNSUPPORTED, "head dim D=%d (built: 64, 128, 256)", D);
     return ATTN_OK;
 }
 
@@ -281,13 +289,14 @@ extern "C" int attn_prefill(const void* q, const void* k, const void* v, void* o
         st = check_launch("fill_no_key_rows_kernel");
         return st == ATTN_OK ? ok() : st;
     }
-    st = (D == 128) ? launch_prefill<128>(q, k, v, out, lse, B, Hq, Hkv, Lq, Lk, scale, is_causal, s)
-                    : launch_prefill<64>(q, k, v, out, lse, B, Hq, Hkv, Lq, Lk, scale, is_causal, s);
+    st = (D == 256)   ? launch_prefill<256>(q, k, v, out, lse, B, Hq, Hkv, Lq, Lk, scale, is_causal, s)
+         : (D == 128) ? launch_prefill<128>(q, k, v, out, lse, B, Hq, Hkv, Lq, Lk, scale, is_causal, s)
+                      : launch_prefill<64>(q, k, v, out, lse, B, Hq, Hkv, Lq, Lk, scale, is_causal, s);
     return st == ATTN_OK ? ok() : st;
 }
 
 extern "C" size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int D) {
-    if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Lmax < 1 || (D != 64 && D != 128) || Hq / Hkv > 128)
+    if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Lmax < 1 || (D != 64 && D != 128 && D != 256) || Hq / Hkv > 128)
         return 0;
     if (B == 0) return 0;
     return decode_layout(B, Hq, Hkv, Lmax, D).total;
@@ -311,8 +320,9 @@ extern "C" int attn_decode(const void* q, const void* k_cache, const void* v_cac
     if (reinterpret_cast<uintptr_t>(workspace) & 255u)
         return fail(ATTN_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    st = (D == 128) ? launch_decode<128>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s)
-                    : launch_decode<64>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s);
+    st = (D == 256)   ? launch_decode<256>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s)
+         : (D == 128) ? launch_decode<128>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s)
+                      : launch_decode<64>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s);
     return st == ATTN_OK ? ok() : st;
 }
 
@@ -340,7 +350,7 @@ extern "C" int attn_selftest_exp2(const float* x, float* y, int n, void* stream)
 }
 
 extern "C" size_t attn_decode_mq_workspace_size(int B, int Hq, int Hkv, int Lq, int Lmax, int D) {
-    if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Lmax < 1 || Lq < 1 || (D != 64 && D != 128) ||
+    if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Lmax < 1 || Lq < 1 || (D != 64 && D != 128 && D != 256) ||
         static_cast<long long>(Hq / Hkv) * Lq > 128)
         return 0;
     if (B == 0) return 0;
@@ -368,8 +378,11 @@ extern "C" int attn_decode_mq(const void* q, const void* k_cache, const void* v_
     if (reinterpret_cast<uintptr_t>(workspace) & 255u)
         return fail(ATTN_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    st = (D == 128) ? launch_decode<128>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s, Lq)
-                    : launch_decode<64>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s, Lq);
+    st = (D == 256)
+             ? launch_decode<256>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s, Lq)
+         : (D == 128)
+             ? launch_decode<128>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s, Lq)
+             : launch_decode<64>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s, Lq);
     return st == ATTN_OK ? ok() : st;
 }
 
@@ -415,7 +428,9 @@ extern "C" int attn_decode_paged(const void* q, const void* k_pages, const void*
     pg.max_pages = max_pages;
     pg.n_pages = n_pages;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    st = (D == 128)
+    st = (D == 256)
+             ? launch_decode<256>(q, k_pages, v_pages, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s, Lq, pg)
+         : (D == 128)
              ? launch_decode<128>(q, k_pages, v_pages, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s, Lq, pg)
              : launch_decode<64>(q, k_pages, v_pages, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s, Lq, pg);
     return st == ATTN_OK ? ok() : st;
@@ -509,7 +524,8 @@ extern "C" int attn_decode_noalloc(const void* q, const void* k_cache, const voi
     void* scratch = decode_scratch_address(&st);
     if (st != ATTN_OK) return st;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    st = (D == 128) ? launch_decode<128>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, scratch, s)
-                    : launch_decode<64>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, scratch, s);
+    st = (D == 256)   ? launch_decode<256>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, scratch, s)
+         : (D == 128) ? launch_decode<128>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, scratch, s)
+                      : launch_decode<64>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, scratch, s);
     return st == ATTN_OK ? ok() : st;
 }

@@ -53,8 +53,8 @@ struct DecodeSmem {
     static constexpr int kStageBytes = 2 * kTileBytes;      // K then V
     static constexpr int kStages = (D == 128) ? 3 : 6;
     static constexpr int kRingBytes = kStages * kStageBytes;
-    // end-of-CTA merge area (reuses the ring): m[4][16], l[4][16], O[4][16][D]
-    static constexpr int kMergeBytes = 4 * 16 * 4 * 2 + 4 * 16 * D * 4;
+    // end-of-CTA merge area (reuses the ring): m[4][16], l[4][16], l_exact[4][16], O[4][16][D]
+    static constexpr int kMergeBytes = 4 * 16 * 4 * 3 + 4 * 16 * D * 4;
     static_assert(kMergeBytes <= kRingBytes, "merge area must fit in the ring");
     static constexpr int kBarOff = kRingBytes;
     static constexpr int kBytes = kBarOff + 2 * kStages * 8 + 16;
@@ -199,7 +199,9 @@ __global__ void __maxnreg__(200)
     float oacc[D / 8][4];
 #pragma unroll
     for (int i = 0; i < D / 8; ++i) oacc[i][0] = oacc[i][1] = oacc[i][2] = oacc[i][3] = 0.0f;
-    float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.0f, l_b = 0.0f;
+    // l: row sum of P as rounded to bf16 (the weights P.V applies; normalises O);
+    // le: row sum of the unrounded exponentials (for the log-sum-exp)
+    float m_a = -INFINITY, m_b = -INFINITY, l_a = 0.0f, l_b = 0.0f, le_a = 0.0f, le_b = 0.0f;
     const float sl2 = p.scale_log2;
     bool ok = true;
 
@@ -262,18 +264,26 @@ __global__ void __maxnreg__(200)
         const float ms_b = (mn_b == -INFINITY) ? 0.0f : mn_b;
         m_a = mn_a;
         m_b = mn_b;
-        float ps_a = 0.0f, ps_b = 0.0f;
+        float ps_a = 0.0f, ps_b = 0.0f, pe_a = 0.0f, pe_b = 0.0f;
 #pragma unroll
         for (int nt = 0; nt < kNT; ++nt) {
             sacc[nt][0] = ex2_approx(fmaf(sacc[nt][0], sl2, -ms_a));
             sacc[nt][1] = ex2_approx(fmaf(sacc[nt][1], sl2, -ms_a));
             sacc[nt][2] = ex2_approx(fmaf(sacc[nt][2], sl2, -ms_b));
             sacc[nt][3] = ex2_approx(fmaf(sacc[nt][3], sl2, -ms_b));
+            pe_a += sacc[nt][0] + sacc[nt][1];
+            pe_b += sacc[nt][2] + sacc[nt][3];
+            // round P to bf16 here, as the MMA will see it, so the row sum
+            // matches the weights actually applied to V
+            f2_unpack(bf16x2_to_f2(pack_bf16x2(sacc[nt][0], sacc[nt][1])), sacc[nt][0], sacc[nt][1]);
+            f2_unpack(bf16x2_to_f2(pack_bf16x2(sacc[nt][2], sacc[nt][3])), sacc[nt][2], sacc[nt][3]);
             ps_a += sacc[nt][0] + sacc[nt][1];
             ps_b += sacc[nt][2] + sacc[nt][3];
         }
         l_a = l_a * f_a + ps_a;
         l_b = l_b * f_b + ps_b;
+        le_a = le_a * f_a + pe_a;
+        le_b = le_b * f_b + pe_b;
 #pragma unroll
         for (int i = 0; i < D / 8; ++i) {
             oacc[i][0] *= f_a;
@@ -323,15 +333,22 @@ __global__ void __maxnreg__(200)
     l_a += __shfl_xor_sync(0xffffffffu, l_a, 2);
     l_b += __shfl_xor_sync(0xffffffffu, l_b, 1);
     l_b += __shfl_xor_sync(0xffffffffu, l_b, 2);
+    le_a += __shfl_xor_sync(0xffffffffu, le_a, 1);
+    le_a += __shfl_xor_sync(0xffffffffu, le_a, 2);
+    le_b += __shfl_xor_sync(0xffffffffu, le_b, 1);
+    le_b += __shfl_xor_sync(0xffffffffu, le_b, 2);
     asm volatile("bar.sync 1, 128;" ::: "memory");   // every compute warp is done with the ring
     float* sm_m = reinterpret_cast<float*>(smem);
     float* sm_l = sm_m + 4 * 16;
-    float* sm_o = sm_l + 4 * 16;
+    float* sm_le = sm_l + 4 * 16;
+    float* sm_o = sm_le + 4 * 16;
     if (tq == 0) {
         sm_m[warp * 16 + grp] = m_a;
         sm_m[warp * 16 + grp + 8] = m_b;
         sm_l[warp * 16 + grp] = l_a;
         sm_l[warp * 16 + grp + 8] = l_b;
+        sm_le[warp * 16 + grp] = le_a;
+        sm_le[warp * 16 + grp + 8] = le_b;
     }
 #pragma unroll
     for (int nt = 0; nt < D / 8; ++nt) {
@@ -351,18 +368,19 @@ __global__ void __maxnreg__(200)
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < kWPM; ++w) M = fmaxf(M, sm_m[(blk * kWPM + w) * 16 + rr]);
-        float Lsum = 0.0f, acc = 0.0f;
+        float Lsum = 0.0f, Lexact = 0.0f, acc = 0.0f;
 #pragma unroll
         for (int w = 0; w < kWPM; ++w) {
             const int ww = blk * kWPM + w;
             const float mw = sm_m[ww * 16 + rr];
             const float sc = (mw == -INFINITY) ? 0.0f : ex2_approx(mw - M);
             Lsum += sm_l[ww * 16 + rr] * sc;
+            Lexact += sm_le[ww * 16 + rr] * sc;
             acc += sm_o[(ww * 16 + rr) * D + d] * sc;
         }
         const size_t prow = (group_row0 + row) * p.n_splits + split;
         p.o_part[prow * D + d] = (Lsum > 0.0f) ? acc / Lsum : 0.0f;
-        if (d == 0) p.lse_part[prow] = (Lsum > 0.0f) ? M + __log2f(Lsum) : -INFINITY;
+        if (d == 0) p.lse_part[prow] = (Lexact > 0.0f) ? M + __log2f(Lexact) : -INFINITY;
     }
 }
 

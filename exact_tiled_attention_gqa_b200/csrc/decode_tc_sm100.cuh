@@ -56,6 +56,7 @@ struct DecodeTcSmem {
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem base, abort flag
     static constexpr int kBytes = kMiscOff + 16;
     static constexpr int kAlloc = kBytes + 1024;
+    static constexpr uint32_t kTmemCols = (128 + D <= 256) ? 256u : 512u;   // S + O, rounded up
 };
 
 template <int D>
@@ -115,7 +116,7 @@ __global__ void __launch_bounds__(kDtcThreads, 2)
         fence_proxy_async_smem();
     }
     if (warp == kDtcMmaWarp) {
-        tmem_alloc(smem_u32(tmem_base_ptr), 256);
+        tmem_alloc(smem_u32(tmem_base_ptr), L::kTmemCols);
         tmem_relinquish();
     }
     tc_fence_before_sync();
@@ -242,7 +243,9 @@ __global__ void __launch_bounds__(kDtcThreads, 2)
         const int lim_lo = min(k_end, seqlen - p.Lq + 1);
         const float sl2 = p.scale_log2;
         const uint64_t sl2x2 = f2_pack(sl2, sl2);
-        float m_run = -INFINITY, l_run = 0.0f;
+        // l_run: row sum of P as rounded to bf16 (normalises O); l_exact: of the
+        // unrounded exponentials (for the log-sum-exp)
+        float m_run = -INFINITY, l_run = 0.0f, l_exact = 0.0f;
         // A warp whose 32 rows are all padding (row >= R) only keeps the pipeline
         // moving: its P rows are never read into a real output row (the MMA keeps
         // rows apart), so it skips the softmax and just signals.
@@ -286,6 +289,7 @@ __global__ void __launch_bounds__(kDtcThreads, 2)
                 factor = (m_run == -INFINITY) ? 0.0f : ex2_approx(m_run - m_tile);
                 m_run = m_tile;
                 l_run *= factor;
+                l_exact *= factor;
             }
             // O holds the sum over tiles < j (S(j) was issued after O += P(j-1) V_{j-1})
             if (j > 0 && __any_sync(0xffffffffu, factor != 1.0f)) {
@@ -310,7 +314,7 @@ __global__ void __launch_bounds__(kDtcThreads, 2)
             // pass 2: exponentials, row sum, P (bf16) over the S columns already read
             const float m_sub = (m_run == -INFINITY) ? 0.0f : m_run;
             const uint64_t negm2 = f2_pack(-m_sub, -m_sub);
-            uint64_t acc0 = 0ull, acc1 = 0ull;
+            uint64_t acc_r = 0ull, acc_e = 0ull;
 #pragma unroll 1
             for (int c = 0; c < kDtcBN; c += 32) {
                 uint32_t v[32];
@@ -330,20 +334,20 @@ __global__ void __launch_bounds__(kDtcThreads, 2)
                     float t0, t1;
                     f2_unpack(t, t0, t1);
                     const float e0 = ex2_approx(t0), e1 = ex2_approx(t1);
-                    if (i & 1)
-                        acc1 = f2_add(acc1, f2_pack(e0, e1));
-                    else
-                        acc0 = f2_add(acc0, f2_pack(e0, e1));
                     pk[i] = pack_bf16x2(e0, e1);
+                    acc_e = f2_add(acc_e, f2_pack(e0, e1));
+                    acc_r = f2_add(acc_r, bf16x2_to_f2(pk[i]));   // P as the MMA sees it
                 }
                 tmem_st_32x32b_x16(tS + c / 2, pk);
             }
             tmem_wait_st();
             tc_fence_before_sync();
             mbar_arrive(bar_p_full);
-            float a0, a1;
-            f2_unpack(f2_add(acc0, acc1), a0, a1);
+            float a0, a1, e0, e1;
+            f2_unpack(acc_r, a0, a1);
+            f2_unpack(acc_e, e0, e1);
             l_run += a0 + a1;
+            l_exact += e0 + e1;
         }
         // ---- this split's partial: O / l (fp32) and m + log2 l per row ----
         bool have_o = ok && n_tiles > 0;
@@ -374,7 +378,7 @@ __global__ void __launch_bounds__(kDtcThreads, 2)
                                     __uint_as_float(o[i + 2]) * inv_l, __uint_as_float(o[i + 3]) * inv_l);
             }
         }
-        if (row_valid) p.lse_part[prow] = (l_run > 0.0f) ? m_run + __log2f(l_run) : -INFINITY;
+        if (row_valid) p.lse_part[prow] = (l_exact > 0.0f) ? m_run + __log2f(l_exact) : -INFINITY;
     }
 
     // ---- teardown ----
@@ -382,7 +386,7 @@ __global__ void __launch_bounds__(kDtcThreads, 2)
     __syncthreads();
     if (warp == kDtcMmaWarp) {
         tc_fence_after_sync();
-        tmem_dealloc(tmem, 256);
+        tmem_dealloc(tmem, L::kTmemCols);
     }
 }
 

@@ -10,13 +10,16 @@
 // and the NVIDIA attention page ("Parameter one: group size": G query heads
 // share one KV head).
 //
-// Work unit (one CTA): one batch b, one KV head g, and 2*P consecutive query
-// positions, as two "Q tiles" of M = 128 rows.  A Q tile packs the G query
+// Work unit (one CTA): one batch b, one KV head g, and NQ*P consecutive query
+// positions, as NQ "Q tiles" of M = 128 rows (NQ = 2 for D <= 128; NQ = 1 for
+// D = 256, whose O accumulator alone takes 256 TMEM columns).  A Q tile packs the G query
 // heads of the group with P = 128 / G positions each (row r = head r / P,
 // position p0 + r % P), so every K/V tile staged in shared memory feeds all
 // G heads of the group and both Q tiles.
 //
-// Roles (384 threads = 3 warpgroups):
+// Roles for NQ = 2 (384 threads = 3 warpgroups; for NQ = 1 the second softmax
+// warpgroup is absent, warps 4 and 5 are producer and MMA issuer, 256 threads,
+// and no registers are exchanged):
 //   warps 0-3  softmax warpgroup for Q tile 0 (thread = TMEM lane = row)
 //   warps 4-7  softmax warpgroup for Q tile 1
 //   warp  8    TMA producer: Q tiles once, then K_j, V_j into a ring of stages
@@ -28,9 +31,12 @@
 // (setmaxnreg.inc to 208): 2 x 208 + 88 = 3 x 168, so the exchange balances
 // exactly and neither side waits.
 //
-// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D).
-// P_q (bf16, two per column) overwrites the first 64 columns of S_q once the
-// softmax has read S_q, and feeds O_q += P_q V_j as the TMEM A operand.
+// TMEM (512 columns): two S buffers at [0,128) and [128,256), then O.  For
+// NQ = 2 buffer q holds S_q and O_q sits at [256 + D q, 256 + D q + D).  For
+// NQ = 1 (D = 256) the two buffers alternate between key tiles (S(j) in buffer
+// j mod 2) and O takes [256, 512).  P (bf16, two per column) overwrites the
+// first 64 columns of its S buffer once the softmax has read S, and feeds
+// O += P V_j as the TMEM A operand.
 //
 // Per key tile j the MMA thread issues, in order:
 //   O0 += P0(j) V_j ; S0(j+1) = Q0 K_{j+1}^T ; O1 += P1(j) V_j ; S1(j+1) = Q1 K_{j+1}^T
@@ -40,11 +46,20 @@
 // A commit after S_q(j+1) also covers O_q += P_q(j) V_j, so when the softmax
 // sees S_q(j+1) its O_q is settled and may be rescaled in place.
 //
-// The exponentials of an unmasked tile are split between the MUFU unit
+// NQ = 1 (D = 256): one Q tile, so the overlap comes from the second S buffer:
+//   S(0) ; S(1) ; then per j:  O += P(j) V_j ; S(j+2) = Q K_{j+2}^T
+// The tensor cores compute S(j+1) while the softmax works on S(j).  Here the
+// commit after S(j+1) does not cover O += P(j-1) V_{j-1}, so each P.V gets its
+// own commit (o_ready) and the softmax waits on it only when it rescales O.
+// The K/V ring holds half tiles (128 keys x 128 columns, 32 KB): K and V each
+// arrive in two halves, in the order the MMAs use them (K0 K1 V0 K2 V1 ...),
+// and the P.V product is issued as two N = 128 halves of O.
+//
+// The exponentials of an unmasked tile can be split between the MUFU unit
 // (ex2.approx) and the FMA pipe (a cubic after range reduction, see
-// exp2_fma_x2): at 128 exponentials per row per tile the MUFU unit alone
-// would take as long as the tile's two MMAs.  Scale-and-subtract, sums and
-// O rescales use packed f32x2 instructions, maxima a 3-input max.
+// exp2_fma_x2; kExpFmaPairsPer8 below, off by default as measured).
+// Scale-and-subtract, sums and O rescales use packed f32x2 instructions,
+// maxima a 3-input max.
 //
 // Online softmax, in the log2 domain (x2 = x * scale * log2 e): per row a
 // running max m and sum l.  The max used for the exponentials is only raised
@@ -61,7 +76,9 @@
 
 namespace attn {
 
-constexpr int kPrefillThreads = 384;
+template <int NQ>
+__host__ __device__ constexpr int prefill_threads() { return 32 * (4 * NQ + 4); }
+__host__ __device__ constexpr int prefill_nq(int D) { return D == 256 ? 1 : 2; }
 constexpr int kPrefillLaunchRegs = 168;    // must equal the compiled register count (checked by the build)
 constexpr int kSoftmaxRegs = 208;
 constexpr int kControlRegs = 88;
@@ -85,33 +102,72 @@ struct PrefillSmem {
     static constexpr int kQTileBytes = kBM * D * 2;      // one Q tile
     static constexpr int kKVTileBytes = kBN * D * 2;     // one K or V tile
     static constexpr int kBlockBytes = 128 * 128;        // one 128-row x 128-byte block
-    static constexpr int kStages = (D == 128) ? 4 : 8;
+    static constexpr int kNQ = prefill_nq(D);
+    // ring entries: whole K or V tiles, or half tiles (32 KB each) for D = 256
+    static constexpr int kItemsPerTile = (D == 256) ? 2 : 1;
+    static constexpr int kItemBytes = kKVTileBytes / kItemsPerTile;
+    static constexpr int kItemKB = kKB / kItemsPerTile;   // 128-byte column blocks per entry
+    static constexpr int kStages = (D == 256) ? 5 : (D == 128) ? 4 : 8;
     static constexpr int kQOff = 0;
-    static constexpr int kKVOff = 2 * kQTileBytes;
-    static constexpr int kBarOff = kKVOff + kStages * kKVTileBytes;
+    static constexpr int kKVOff = kNQ * kQTileBytes;
+    static constexpr int kBarOff = kKVOff + kStages * kItemBytes;
     // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_half[2], p_full[2], o_done[2], drain
     static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 2 + 1;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;   // tmem base (u32), abort flag (int)
     static constexpr int kBytes = kMiscOff + 16;
     static constexpr int kAlloc = kBytes + 1024;              // slack to align the base to 1 KiB
+    static_assert(kAlloc <= 232448, "dynamic shared memory per CTA");
 };
+
+// Ring order of the K/V entries.  NQ = 2: K_0 V_0 K_1 V_1 ...  NQ = 1:
+// K_0 K_1 V_0 K_2 V_1 K_3 V_2 ... V_{n-1}, each tile as kItemsPerTile entries.
+// Position (in tiles) of K_j and V_j, and the inverse map.
+template <int NQ>
+__device__ __forceinline__ int ring_pos_k(int j) { return NQ == 2 ? 2 * j : (j == 0 ? 0 : 2 * j - 1); }
+template <int NQ>
+__device__ __forceinline__ int ring_pos_v(int j, int n_kt) {
+    return NQ == 2 ? 2 * j + 1 : (j + 1 < n_kt ? 2 * j + 2 : 2 * n_kt - 1);
+}
+template <int NQ>
+__device__ __forceinline__ void ring_tile(int pos, int n_kt, bool& is_v, int& j) {
+    if (NQ == 2) {
+        is_v = pos & 1;
+        j = pos >> 1;
+    } else if (pos == 0) {
+        is_v = false;
+        j = 0;
+    } else if (pos == 2 * n_kt - 1) {
+        is_v = true;
+        j = n_kt - 1;
+    } else if (pos & 1) {
+        is_v = false;
+        j = (pos + 1) >> 1;
+    } else {
+        is_v = true;
+        j = (pos - 2) >> 1;
+    }
+}
 
 struct PrefillParams {
     void* out;          // [B,Hq,Lq,D] bf16
     float* lse;         // [B,Hq,Lq] or nullptr
     int B, Hq, Hkv, Lq, Lk;
     int G, P;           // group size, positions per Q tile (P = 128 / G)
-    int n_mblk;         // ceil(Lq / (2P))
+    int n_mblk;         // ceil(Lq / (NQ P))
     int is_causal;
     float scale_log2;   // scale * log2(e)
 };
 
-template <int D>
-__global__ void __launch_bounds__(kPrefillThreads, 1)
+template <int D, int NQ>
+__global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
     attn_prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                               const __grid_constant__ CUtensorMap tm_k,
                               const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
     using L = PrefillSmem<D>;
+    static_assert(L::kNQ == NQ, "Q tiles per CTA follow from D");
+    constexpr int kThreads = prefill_threads<NQ>();
+    constexpr int kProducerWarp = 4 * NQ;
+    constexpr int kMmaWarp = 4 * NQ + 1;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     const uint32_t base = (raw_base + 1023u) & ~1023u;
@@ -129,11 +185,11 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     const int g = bh % p.Hkv;
     const int P = p.P;
     const int rows_used = p.G * P;
-    const int p_begin = mblk * 2 * P;
+    const int p_begin = mblk * NQ * P;
     const long off = static_cast<long>(p.Lk) - static_cast<long>(p.Lq);
     int n_kt;
     {
-        const int p_last = min(p_begin + 2 * P, p.Lq) - 1;
+        const int p_last = min(p_begin + NQ * P, p.Lq) - 1;
         const long last_key = p.is_causal ? min(static_cast<long>(p_last) + off, static_cast<long>(p.Lk) - 1)
                                           : static_cast<long>(p.Lk) - 1;
         n_kt = last_key < 0 ? 0 : static_cast<int>(last_key / kBN) + 1;
@@ -160,7 +216,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             mbar_init(bar_kv_full(s), 1);
             mbar_init(bar_kv_empty(s), 1);
         }
-        for (int q = 0; q < 2; ++q) {
+        for (int q = 0; q < 2; ++q) {   // per Q tile (NQ = 2) or per S buffer (NQ = 1)
             mbar_init(bar_s_full(q), 1);
             mbar_init(bar_p_half(q), 128);
             mbar_init(bar_p_full(q), 128);
@@ -174,15 +230,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // finite values: zero them through the generic proxy, then hand them over.
     if (rows_used < kBM) {
         const int pad_bytes_per_block = (kBM - rows_used) * 128;
-        for (int q = 0; q < 2; ++q)
+        for (int q = 0; q < NQ; ++q)
             for (int kb = 0; kb < L::kKB; ++kb) {
                 uint8_t* blk = smem + L::kQOff + q * L::kQTileBytes + kb * L::kBlockBytes + rows_used * 128;
-                for (int i = threadIdx.x * 16; i < pad_bytes_per_block; i += kPrefillThreads * 16)
+                for (int i = threadIdx.x * 16; i < pad_bytes_per_block; i += kThreads * 16)
                     *reinterpret_cast<uint4*>(blk + i) = make_uint4(0, 0, 0, 0);
             }
         fence_proxy_async_smem();
     }
-    if (warp == 9) {
+    if (warp == kMmaWarp) {
         tmem_alloc(smem_u32(tmem_base_ptr), 512);
         tmem_relinquish();
     }
@@ -191,33 +247,36 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_base_ptr;
 
-    if (warp >= 8) {
-      asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
-      if (warp == 8) {
+    if (warp >= kProducerWarp) {
+      if constexpr (NQ == 2) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
+      if (warp == kProducerWarp) {
         // ================= TMA producer =================
         if (lane == 0 && n_kt > 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
             const int q_head0 = b * p.Hq + g * p.G;
-            mbar_arrive_expect_tx(bar_q_full, 2u * L::kKB * rows_used * 128u);
-            for (int q = 0; q < 2; ++q)
+            mbar_arrive_expect_tx(bar_q_full, static_cast<uint32_t>(NQ * L::kKB * rows_used * 128));
+            for (int q = 0; q < NQ; ++q)
                 for (int kb = 0; kb < L::kKB; ++kb)
                     tma_load_3d(sQ + q * L::kQTileBytes + kb * L::kBlockBytes, &tm_q, bar_q_full, kb * 64,
                                 p_begin + q * P, q_head0);
             const int kv_row = b * p.Hkv + g;
             int issued = 0;
             bool ok = true;
-            for (int t = 0; t < 2 * n_kt && ok; ++t) {
+            for (int t = 0; t < 2 * n_kt * L::kItemsPerTile && ok; ++t) {
                 const int s = t % L::kStages;
                 const uint32_t round = static_cast<uint32_t>(t / L::kStages);
                 ok = mbar_wait(bar_kv_empty(s), (round & 1u) ^ 1u, abort_flag, &g_attn_err, kDevErrTimeout);
                 if (!ok) break;
-                mbar_arrive_expect_tx(bar_kv_full(s), L::kKVTileBytes);
-                const CUtensorMap* map = (t & 1) ? &tm_v : &tm_k;
-                const int j = t >> 1;
-                for (int kb = 0; kb < L::kKB; ++kb)
-                    tma_load_3d(sKV + s * L::kKVTileBytes + kb * L::kBlockBytes, map, bar_kv_full(s), kb * 64,
+                mbar_arrive_expect_tx(bar_kv_full(s), L::kItemBytes);
+                bool is_v;
+                int j;
+                ring_tile<NQ>(t / L::kItemsPerTile, n_kt, is_v, j);
+                const int kb0 = (t % L::kItemsPerTile) * L::kItemKB;
+                const CUtensorMap* map = is_v ? &tm_v : &tm_k;
+                for (int kb = 0; kb < L::kItemKB; ++kb)
+                    tma_load_3d(sKV + s * L::kItemBytes + kb * L::kBlockBytes, map, bar_kv_full(s), (kb0 + kb) * 64,
                                 j * kBN, kv_row);
                 issued = t + 1;
             }
@@ -236,7 +295,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             }
         }
         __syncwarp();
-    } else if (warp == 9) {
+    } else if (warp == kMmaWarp) {
         // ================= MMA issuer =================
         if (lane == 0 && n_kt > 0) {
             constexpr uint32_t kIdescQK = umma_idesc_bf16_f32(kBM, kBN, false);
@@ -251,7 +310,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             const uint64_t dQ[2] = {umma_sdesc_sw128(sQ, 16, 1024), umma_sdesc_sw128(sQ + L::kQTileBytes, 16, 1024)};
             const uint64_t dK0 = umma_sdesc_sw128(sKV, 16, 1024);
             const uint64_t dV0 = umma_sdesc_sw128(sKV, L::kBlockBytes, 1024);
-            constexpr uint64_t kSlotStep = L::kKVTileBytes >> 4;
+            constexpr uint64_t kSlotStep = L::kItemBytes >> 4;
             // S_q = Q_q K^T : M=128, N=128, K=D in steps of 16 (32 bytes)
             auto issue_qk = [&](int q, int t) {
                 const uint64_t b0 = dK0 + static_cast<uint64_t>(slot_of(t)) * kSlotStep;
@@ -285,13 +344,16 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 return true;
             };
             bool ok = mbar_wait(bar_q_full, 0, abort_flag, &g_attn_err, kDevErrTimeout);
+          if constexpr (NQ == 2) {
             if (ok) ok = mbar_wait(bar_kv_full(slot_of(0)), par_of(0), abort_flag, &g_attn_err, kDevErrTimeout);
             if (ok) {
                 tc_fence_after_sync();
                 issue_qk(0, 0);
                 umma_commit(bar_s_full(0));
-                issue_qk(1, 0);
-                umma_commit(bar_s_full(1));
+                if constexpr (NQ == 2) {
+                    issue_qk(1, 0);
+                    umma_commit(bar_s_full(1));
+                }
                 umma_commit(bar_kv_empty(slot_of(0)));
             }
             for (int j = 0; j < n_kt && ok; ++j) {
@@ -308,16 +370,83 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                     issue_qk(0, tk);
                     umma_commit(bar_s_full(0));
                 }
-                ok = pv_tile(1, tv, j);
-                if (!ok) break;
-                if (last) umma_commit(bar_o_done(1));
+                if constexpr (NQ == 2) {
+                    ok = pv_tile(1, tv, j);
+                    if (!ok) break;
+                    if (last) umma_commit(bar_o_done(1));
+                }
                 umma_commit(bar_kv_empty(slot_of(tv)));
                 if (!last) {
-                    issue_qk(1, tk);
-                    umma_commit(bar_s_full(1));
+                    if constexpr (NQ == 2) {
+                        issue_qk(1, tk);
+                        umma_commit(bar_s_full(1));
+                    }
                     umma_commit(bar_kv_empty(slot_of(tk)));
                 }
             }
+          } else {
+            // ---- one Q tile, S double-buffered (D = 256) ----
+            constexpr uint32_t kIdescPVh = umma_idesc_bf16_f32(kBM, 128, true);
+            const uint32_t tOq = tmem + 256u;
+            auto wait_item = [&](int it) {
+                return mbar_wait(bar_kv_full(slot_of(it)), par_of(it), abort_flag, &g_attn_err, kDevErrTimeout);
+            };
+            // S(j) into buffer j % 2, K_j in two half entries (columns 0-127, 128-255)
+            auto qk = [&](int j) {
+                const int it0 = L::kItemsPerTile * ring_pos_k<NQ>(j);
+                const uint32_t tSb = tS[j & 1];
+                for (int hh = 0; hh < 2; ++hh) {
+                    if (!wait_item(it0 + hh)) return false;
+                    tc_fence_after_sync();
+                    const uint64_t b0 = dK0 + static_cast<uint64_t>(slot_of(it0 + hh)) * kSlotStep;
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const int kq = hh * 8 + kk;
+                        const uint64_t koff = static_cast<uint64_t>(((kk >> 2) * L::kBlockBytes + (kk & 3) * 32) >> 4);
+                        const uint64_t qoff = static_cast<uint64_t>(((kq >> 2) * L::kBlockBytes + (kq & 3) * 32) >> 4);
+                        umma_ss(tSb, dQ[0] + qoff, b0 + koff, kIdescQK, kq > 0 ? 1u : 0u);
+                    }
+                    umma_commit(bar_kv_empty(slot_of(it0 + hh)));
+                }
+                umma_commit(bar_s_full(j & 1));
+                return true;
+            };
+            // O[:, 128 hv .. +128) += P(j)[:, keys of `half`] V_j^(hv)
+            auto pv_part = [&](int j, int itv, int half) {
+                const uint32_t tSb = tS[j & 1];
+#pragma unroll
+                for (int hv = 0; hv < 2; ++hv) {
+                    const uint64_t b0 = dV0 + static_cast<uint64_t>(slot_of(itv + hv)) * kSlotStep;
+#pragma unroll
+                    for (int k4 = 0; k4 < kBN / 32; ++k4) {
+                        const int kk = half * (kBN / 32) + k4;
+                        umma_ts(tOq + 128u * hv, tSb + kk * 8, b0 + static_cast<uint64_t>((kk * 2048) >> 4),
+                                kIdescPVh, (j > 0 || kk > 0) ? 1u : 0u);
+                    }
+                }
+            };
+            if (ok) ok = qk(0);
+            if (ok && n_kt > 1) ok = qk(1);
+            for (int j = 0; j < n_kt && ok; ++j) {
+                const int buf = j & 1;
+                const uint32_t ph = static_cast<uint32_t>(j >> 1) & 1u;
+                const int itv = L::kItemsPerTile * ring_pos_v<NQ>(j, n_kt);
+                ok = wait_item(itv) && wait_item(itv + 1);
+                ok = ok && mbar_wait(bar_p_half(buf), ph, abort_flag, &g_attn_err, kDevErrTimeout);
+                if (!ok) break;
+                tc_fence_after_sync();
+                pv_part(j, itv, 0);
+                ok = mbar_wait(bar_p_full(buf), ph, abort_flag, &g_attn_err, kDevErrTimeout);
+                if (!ok) break;
+                tc_fence_after_sync();
+                pv_part(j, itv, 1);
+                umma_commit(bar_o_done(1));              // o_ready: O holds tiles 0..j
+                if (j + 1 == n_kt) umma_commit(bar_o_done(0));
+                umma_commit(bar_kv_empty(slot_of(itv)));
+                umma_commit(bar_kv_empty(slot_of(itv + 1)));
+                if (j + 2 < n_kt) ok = qk(j + 2);
+            }
+          }
             // Drain: no MMA may still be running when TMEM is released.
             umma_commit(bar_drain);
             const uint64_t t0 = global_timer_ns();
@@ -327,12 +456,12 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         __syncwarp();
       }
     } else {
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+        if constexpr (NQ == 2) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
         // ================= softmax warpgroups =================
         const int q = warp >> 2;                 // Q tile of this warpgroup
         const int r = threadIdx.x & 127;         // row = TMEM lane
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t tS = tmem + (q ? 128u : 0u) + lane_off;
+        const uint32_t tS_q = tmem + (q ? 128u : 0u) + lane_off;
         const uint32_t tO = tmem + 256u + (q ? static_cast<uint32_t>(D) : 0u) + lane_off;
         const int head_local = r / P;
         const int pos = p_begin + q * P + (r % P);
@@ -346,10 +475,15 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
         const float sl2 = p.scale_log2;
 
         float m_run = -INFINITY;   // running max used for the exponentials (log2 domain)
-        float l_run = 0.0f;        // running sum of exponentials
+        float l_run = 0.0f;        // running sum of P as rounded to bf16 (normalises O)
+        float l_exact = 0.0f;      // running sum of the unrounded exponentials (for the LSE)
         bool ok = true;
         for (int j = 0; j < n_kt; ++j) {
-            ok = mbar_wait(bar_s_full(q), static_cast<uint32_t>(j) & 1u, abort_flag, &g_attn_err, kDevErrTimeout);
+            // S buffer of this tile, and the phase of its barriers
+            const int buf = (NQ == 2) ? q : (j & 1);
+            const uint32_t ph = static_cast<uint32_t>(NQ == 2 ? j : (j >> 1)) & 1u;
+            const uint32_t tS = (NQ == 2) ? tS_q : tS_q + (static_cast<uint32_t>(j & 1) << 7);
+            ok = mbar_wait(bar_s_full(buf), ph, abort_flag, &g_attn_err, kDevErrTimeout);
             if (!ok) break;
             tc_fence_after_sync();
             uint32_t sr[128];
@@ -386,10 +520,20 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 factor = (m_run == -INFINITY) ? 0.0f : ex2_approx(m_run - m_tile);
                 m_run = m_tile;
                 l_run *= factor;
+                l_exact *= factor;
             }
             // rescale O_q in TMEM if any row of this warp raised its max (O holds
             // the sum over tiles < j, settled: see the file comment)
             if (j > 0 && __any_sync(0xffffffffu, factor != 1.0f)) {
+                if constexpr (NQ == 1) {
+                    // O += P(j-1) V_{j-1} must have landed (at most one P.V is outstanding)
+                    if (!mbar_wait(bar_o_done(1), static_cast<uint32_t>(j - 1) & 1u, abort_flag, &g_attn_err,
+                                   kDevErrTimeout)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after_sync();
+                }
                 const uint64_t f2 = f2_pack(factor, factor);
 #pragma unroll 1
                 for (int c = 0; c < D; c += 32) {
@@ -413,7 +557,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             const float m_sub = (m_run == -INFINITY) ? 0.0f : m_run;
             const uint64_t sl2x2 = f2_pack(sl2, sl2);
             const uint64_t negm2 = f2_pack(-m_sub, -m_sub);
-            uint64_t acc2[4] = {0ull, 0ull, 0ull, 0ull};
+            uint64_t acc_r[2] = {0ull, 0ull}, acc_e[2] = {0ull, 0ull};
             auto exp_half = [&](auto masked_tag, int h) {
                 constexpr bool kMasked = decltype(masked_tag)::value;
                 uint32_t pk[32];
@@ -429,15 +573,19 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                         f2_unpack(t, t0, t1);
                         e = f2_pack(ex2_approx(t0), ex2_approx(t1));
                     }
-                    acc2[i & 3] = f2_add(acc2[i & 3], e);
                     float e0, e1;
                     f2_unpack(e, e0, e1);
                     pk[i] = pack_bf16x2(e0, e1);
+                    // O is normalised by the sum of P as the MMA sees it (bf16), so
+                    // the rounding of a dominant weight cancels in O / l; the LSE
+                    // takes the unrounded sum
+                    acc_e[i & 1] = f2_add(acc_e[i & 1], e);
+                    acc_r[i & 1] = f2_add(acc_r[i & 1], bf16x2_to_f2(pk[i]));
                 }
                 tmem_st_32x32b_x32(tS + h * 32, pk);
                 tmem_wait_st();
                 tc_fence_before_sync();
-                mbar_arrive(h == 0 ? bar_p_half(q) : bar_p_full(q));
+                mbar_arrive(h == 0 ? bar_p_half(buf) : bar_p_full(buf));
             };
             if (masked) {
                 exp_half(std::true_type{}, 0);
@@ -447,9 +595,10 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
                 exp_half(std::false_type{}, 1);
             }
             float a0, a1, b0, b1;
-            f2_unpack(f2_add(acc2[0], acc2[1]), a0, a1);
-            f2_unpack(f2_add(acc2[2], acc2[3]), b0, b1);
-            l_run += (a0 + a1) + (b0 + b1);
+            f2_unpack(f2_add(acc_r[0], acc_r[1]), a0, a1);
+            f2_unpack(f2_add(acc_e[0], acc_e[1]), b0, b1);
+            l_run += a0 + a1;
+            l_exact += b0 + b1;
         }
 
         // ---- epilogue: O / l -> bf16, LSE ----
@@ -483,7 +632,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
             }
         }
         if (row_valid && p.lse != nullptr) {
-            const float lse = (l_run > 0.0f) ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
+            const float lse = (l_exact > 0.0f) ? (m_run + __log2f(l_exact)) * kLn2 : -INFINITY;
             p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.Lq + pos] = lse;
         }
     }
@@ -491,7 +640,7 @@ __global__ void __launch_bounds__(kPrefillThreads, 1)
     // ---- teardown ----
     tc_fence_before_sync();
     __syncthreads();
-    if (warp == 9) {
+    if (warp == kMmaWarp) {
         tc_fence_after_sync();
         tmem_dealloc(tmem, 512);
     }

@@ -318,6 +318,11 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return r;
 }
 
+// packed bf16x2 -> the two values as fp32, packed f32x2 (exact)
+__device__ __forceinline__ uint64_t bf16x2_to_f2(uint32_t u) {
+    return f2_pack(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+
 // -------------------------------------------------------------------------
 // warp-level tensor-core path (decode): ldmatrix + mma.sync m16n8k16 bf16
 // -------------------------------------------------------------------------

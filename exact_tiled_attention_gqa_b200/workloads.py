@@ -79,6 +79,11 @@ CHUNKED_16K = PrefillShape("chunked prefill Lq2048 onto Lk16384 (bottom-right)",
 CHUNKED_32K = PrefillShape("chunked prefill Lq2048 onto Lk32768 (bottom-right)", 1, 32, 8, 2048, 32768,
                            128, True, 97, 8.0)
 QWEN_DECODE = DecodeShape("Qwen3-8B decode B64 seqlen U[1024,32768]", 64, 32, 8, 32768, 128, 1024, 32768)
+# Head dim 256, the other width the NVIDIA attention page recommends ("Parameter
+# two: head dimension"), at group size 8.
+HD256_PREFILL = PrefillShape("head-dim-256 causal prefill B2 Hq16 Hkv2 L8192 D256", 2, 16, 2, 8192, 8192, 256)
+HD256_DECODE = DecodeShape("head-dim-256 decode B32 Hq16 Hkv2 seqlen U[1024,32768] D256", 32, 16, 2, 32768, 256,
+                           1024, 32768)
 
 
 def group_sweep_decode(G: int) -> DecodeShape:

@@ -49,7 +49,7 @@ extern "C" {
 typedef enum {
     ATTN_OK = 0,
     ATTN_ERR_INVALID_ARG = -1, /* null pointer, bad size, Hq % Hkv != 0, bad scale, misalignment */
-    ATTN_ERR_UNSUPPORTED = -2, /* valid but not built: D not in {64, 128}, group size too large */
+    ATTN_ERR_UNSUPPORTED = -2, /* valid but not built: D not in {64, 128, 256}, group size too large */
     ATTN_ERR_WORKSPACE = -3,   /* decode workspace missing or smaller than required */
     ATTN_ERR_CUDA = -4         /* a CUDA runtime call or kernel launch failed */
 } attn_status_t;
@@ -72,7 +72,8 @@ typedef enum {
  *   out  [B, Hq,  Lq, D]  bf16, written
  *   lse  [B, Hq,  Lq]     fp32, written; may be NULL (not written)
  *   scale: finite and > 0 (usually 1/sqrt(D))
- *   D: 64 or 128.  G = Hq / Hkv: 1 .. 128.
+ *   D: 64, 128 or 256 (the head dims the NVIDIA attention page recommends,
+ *   "Parameter two: head dimension", plus 64).  G = Hq / Hkv: 1 .. 128.
  *   B == 0 or Lq == 0: nothing to do, returns ATTN_OK.
  *   Lk == 0: every row sees no key (O = 0, LSE = -inf).
  *
@@ -81,7 +82,7 @@ typedef enum {
  *
  * Errors: ATTN_ERR_INVALID_ARG for a null non-empty tensor, negative sizes, Hq or
  * Hkv < 1, Hq % Hkv != 0, non-finite or non-positive scale, or a base
- * address not 16-byte aligned; ATTN_ERR_UNSUPPORTED for D outside {64, 128}
+ * address not 16-byte aligned; ATTN_ERR_UNSUPPORTED for D outside {64, 128, 256}
  * or G > 128; ATTN_ERR_CUDA when a launch fails.
  */
 int attn_prefill(const void* q, const void* k, const void* v, void* out, float* lse,
@@ -121,7 +122,7 @@ size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int D);
  *              bytes, 256-byte aligned, owned by the caller; its contents on
  *              entry do not matter and on return are unspecified.  Two calls
  *              in flight at once must not share one workspace.
- *   D: 64 or 128.  G = Hq / Hkv: 1 .. 128.  B == 0 returns ATTN_OK.
+ *   D: 64, 128 or 256.  G = Hq / Hkv: 1 .. 128.  B == 0 returns ATTN_OK.
  *
  * Errors: as attn_prefill, plus ATTN_ERR_WORKSPACE for a null or too small
  * workspace.
@@ -153,7 +154,7 @@ size_t attn_decode_mq_workspace_size(int B, int Hq, int Hkv, int Lq, int Lmax, i
  *   out      [B, Hq, Lq, D]      bf16, written
  *   lse      [B, Hq, Lq]         fp32, written; may be NULL
  *   workspace: at least attn_decode_mq_workspace_size(...) bytes, as attn_decode
- *   D: 64 or 128.  G * Lq <= 128 (G = Hq / Hkv).
+ *   D: 64, 128 or 256.  G * Lq <= 128 (G = Hq / Hkv).
  *
  * Errors: as attn_decode, plus ATTN_ERR_INVALID_ARG for Lq < 1 and
  * ATTN_ERR_UNSUPPORTED for G * Lq > 128.
@@ -187,7 +188,7 @@ size_t attn_decode_paged_workspace_size(int B, int Hq, int Hkv, int Lq, int page
  *   seqlens      [B]                             int32 in device memory, each in
  *                                                [0, page_size * max_pages]
  *   out          [B, Hq, Lq, D] bf16;  lse [B, Hq, Lq] fp32 or NULL
- *   page_size: a positive multiple of 64.  D: 64 or 128.  G * Lq <= 128.
+ *   page_size: a positive multiple of 64.  D: 64, 128 or 256.  G * Lq <= 128.
  *
  * Errors: as attn_decode_mq, plus ATTN_ERR_INVALID_ARG for a page_size that
  * is not a positive multiple of 64, n_pages or max_pages < 1, or a null

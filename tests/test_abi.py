@@ -60,7 +60,7 @@ def _prefill(lib, **kw):
     (dict(Hq=0), -1), (dict(Hkv=0), -1), (dict(Hq=6, Hkv=4), -1), (dict(scale=0.0), -1),
     (dict(scale=-1.0), -1), (dict(scale=float("nan")), -1), (dict(scale=float("inf")), -1),
     (dict(q=ctypes.c_void_p(0x10008)), -1), (dict(lse=ctypes.c_void_p(0x10002)), -1),
-    (dict(D=96), -2), (dict(D=256), -2), (dict(Hq=256, Hkv=1), -2),
+    (dict(D=96), -2), (dict(D=512), -2), (dict(Hq=256, Hkv=1), -2),
 ])
 def test_prefill_rejects(lib, bad, code):
     assert _prefill(lib, **bad) == code
@@ -105,6 +105,8 @@ def test_workspace_size(lib):
     assert f(0, 8, 2, 64, 128) == 0
     assert f(2, 8, 3, 64, 128) == 0        # Hq % Hkv
     assert f(2, 8, 2, 64, 96) == 0         # D
+    assert f(2, 8, 2, 64, 512) == 0
+    assert f(2, 8, 2, 64, 256) > 0
     assert f(2, 8, 2, 0, 128) == 0         # Lmax
     assert f(1, 256, 1, 64, 128) == 0      # G > 128
     a = f(2, 8, 2, 1000, 128)

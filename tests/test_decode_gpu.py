@@ -46,7 +46,7 @@ def _check(oracle_mod, q, k, v, sl, what):
     return assert_close(out, lse, ref_o, ref_l, what)
 
 
-@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("D", [64, 128, 256])
 @pytest.mark.parametrize("G", [1, 2, 4, 8, 16, 32, 64, 128, 3, 12, 17, 24, 48, 96])
 def test_group_sizes(oracle_mod, D, G):
     Hkv = 2 if G <= 64 else 1
@@ -60,6 +60,12 @@ def test_group_sizes(oracle_mod, D, G):
 def test_split_edges(oracle_mod, Lmax, seqlens):
     q, k, v, sl = _inputs(len(seqlens), 8, 2, Lmax, 128, seqlens, seed=Lmax)
     _check(oracle_mod, q, k, v, sl, f"Lmax{Lmax}")
+
+
+@pytest.mark.parametrize("Lmax,seqlens", [(5000, [5000, 4097, 4096, 4095, 1, 2500]), (9000, [0, 9000, 2049])])
+def test_split_edges_d256(oracle_mod, Lmax, seqlens):
+    q, k, v, sl = _inputs(len(seqlens), 8, 2, Lmax, 256, seqlens, seed=Lmax + 1)
+    _check(oracle_mod, q, k, v, sl, f"D256 Lmax{Lmax}")
 
 
 def test_zero_length_sequence(oracle_mod):

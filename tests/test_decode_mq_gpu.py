@@ -47,7 +47,7 @@ def _oracle(oracle_mod, q, k, v, seqlens, scale):
     return np.stack(outs), np.stack(lses)
 
 
-@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("D", [64, 128, 256])
 @pytest.mark.parametrize("G,Lq", [(4, 1), (4, 2), (4, 4), (4, 8), (4, 16), (1, 16), (8, 8), (2, 5), (3, 7), (16, 4),
                                   (32, 2), (64, 1), (4, 32), (8, 16), (64, 2), (3, 40)])
 def test_multi_query_against_oracle(oracle_mod, D, G, Lq):

@@ -54,7 +54,8 @@ def _paged_inputs(seqlens, Hq, Hkv, Lq, D, page_size, seed, spare_pages=3):
 
 
 @pytest.mark.parametrize("page_size", [64, 128, 256])
-@pytest.mark.parametrize("G,Lq,D", [(4, 1, 128), (4, 4, 128), (8, 2, 64), (1, 1, 128), (16, 4, 128)])
+@pytest.mark.parametrize("G,Lq,D", [(4, 1, 128), (4, 4, 128), (8, 2, 64), (1, 1, 128), (16, 4, 128), (4, 2, 256),
+                                    (32, 1, 256)])
 def test_paged_against_oracle(oracle_mod, page_size, G, Lq, D):
     Hkv = 2
     seqlens = [1000, 1, 0, 257, 64, 3000]

@@ -43,7 +43,7 @@ def test_tiny_config(oracle_mod):
     _run(oracle_mod, s.B, s.Hq, s.Hkv, s.Lq, s.Lk, s.D, True)
 
 
-@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("D", [64, 128, 256])
 @pytest.mark.parametrize("causal", [True, False])
 @pytest.mark.parametrize("Hq,Hkv", [(4, 4), (8, 4), (8, 2), (16, 2), (6, 2), (32, 1), (5, 5)])
 def test_ragged_multi_tile(oracle_mod, D, causal, Hq, Hkv):
@@ -59,6 +59,35 @@ def test_chunked_bottom_right(oracle_mod, Lq, Lk):
 def test_group_of_128_and_64(oracle_mod):
     _run(oracle_mod, 1, 128, 1, 40, 300, 128, True, seed=5)
     _run(oracle_mod, 1, 64, 1, 70, 200, 64, True, seed=6)
+    _run(oracle_mod, 1, 128, 1, 20, 300, 256, True, seed=7)
+
+
+@pytest.mark.parametrize("Lq,Lk", [(77, 500), (1, 500), (128, 640), (250, 129), (1, 1), (200, 130), (513, 513),
+                                   (1000, 1700)])
+def test_d256_chunked_and_long(oracle_mod, Lq, Lk):
+    """D = 256 runs one Q tile per CTA with two S buffers in TMEM and a ring of
+    half tiles; these cover 1 to 14 key tiles, so the ring and the buffers wrap."""
+    _run(oracle_mod, 1, 8, 2, Lq, Lk, 256, True, seed=Lq + 3 * Lk, spike=97)
+
+
+@pytest.mark.parametrize("D", [128, 256])
+def test_rescale_on_every_tile(oracle_mod, D):
+    """Keys whose scores climb by more than 2^8 (log2) per 128-key tile: the
+    running max moves on every tile, so O is rescaled in TMEM each time (at
+    D = 256 while the previous P.V product may still be in flight)."""
+    B, Hq, Hkv, L = 1, 8, 2, 1400
+    q, k, v = W.prefill_inputs(B, Hq, Hkv, L, L, D, seed=21)
+    # q ~ ones / sqrt(D), k_j = noise + r_j ones: score * scale * log2 e ~ r_j log2 e,
+    # with r_j stepping by 12 / log2 e per tile (a rise of about 2^12 per tile)
+    ramp = (torch.arange(L, dtype=torch.float32) // 128) * (12.0 / math.log2(math.e))
+    q = (1.0 / math.sqrt(D) + 0.1 * q.float()).to(torch.bfloat16)
+    k = (0.5 * k.float() + ramp[None, None, :, None]).to(torch.bfloat16)
+    scale = 1.0 / math.sqrt(D)
+    out, lse = prefill(q.cuda(), k.cuda(), v.cuda(), scale=scale, is_causal=True)
+    torch.cuda.synchronize()
+    ref_o, ref_l = oracle_mod.attention_prefill(q, k, v, scale, True)
+    assert device_error(reset=True) == 0
+    assert_close(out, lse, ref_o, ref_l, f"rescale D{D}")
 
 
 def test_no_keys_and_empty(oracle_mod):
