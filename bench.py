@@ -414,6 +414,23 @@ def run_sweeps(attn, dev, stream, seed, max_over_ranks):
                            "frac_of_measured_hbm": round(by / ms / 1e6 / float(peaks["hbm_gbs"]), 4)}
     del kp, vp, dq, o, l, ws, table
     torch.cuda.empty_cache()
+    out["decode_kv8"] = []
+    for fmt, shape in ((W.KV_E4M3, W.QWEN_DECODE_E4M3), (W.KV_Q8_0, W.QWEN_DECODE_Q8_0)):
+        dq, dk, dv, dks, dvs, dsl = W.decode_inputs_kv8(shape.B, shape.Hq, shape.Hkv, shape.Lmax, shape.D,
+                                                        shape.seqlen_lo, shape.seqlen_hi, fmt, seed=seed,
+                                                        device=dev)
+        o = torch.empty_like(dq)
+        l = torch.empty((shape.B, shape.Hq, 1), dtype=torch.float32, device=dev)
+        ws = torch.empty(attn.decode_kv8_workspace_size(shape.B, shape.Hq, shape.Hkv, 1, shape.Lmax, shape.D),
+                         dtype=torch.uint8, device=dev)
+        ms = max_over_ranks(_time_calls(lambda: attn.decode_kv8(dq, dk, dv, dks, dvs, dsl, scale=shape.scale, out=o,
+                                                                 lse=l, workspace=ws, stream=stream), stream, n=10))
+        by = RL.decode_kv8_bytes(dsl.cpu().tolist(), shape.B, shape.Hq, shape.Hkv, shape.D, fmt == W.KV_Q8_0)
+        out["decode_kv8"].append({"workload": shape.name, "ms": round(ms, 4), "bytes": by,
+                                  "gbs": round(by / ms / 1e6, 1),
+                                  "frac_of_measured_hbm": round(by / ms / 1e6 / float(peaks["hbm_gbs"]), 4)})
+        del dq, dk, dv, dks, dvs, dsl, o, l, ws
+        torch.cuda.empty_cache()
     shape = W.HD256_DECODE
     dq, dk, dv, dsl = W.decode_inputs_for(shape, seed=seed + 256, device=dev)
     o = torch.empty_like(dq)

@@ -27,8 +27,8 @@ import torch
 from . import _native
 from ._native import AttnError
 
-__all__ = ["prefill", "decode", "decode_mq", "decode_paged", "decode_noalloc", "decode_workspace_size",
-           "decode_mq_workspace_size", "device_error", "AttnError", "library_path"]
+__all__ = ["prefill", "decode", "decode_mq", "decode_paged", "decode_noalloc", "decode_kv8", "decode_workspace_size",
+           "decode_mq_workspace_size", "decode_kv8_workspace_size", "device_error", "AttnError", "library_path"]
 
 
 def library_path() -> str:
@@ -152,6 +152,59 @@ def decode_mq(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, seq
     return out, lse
 
 
+def decode_kv8_workspace_size(B: int, Hq: int, Hkv: int, Lq: int, Lmax: int, D: int) -> int:
+    return int(_native.lib().attn_decode_kv8_workspace_size(B, Hq, Hkv, Lq, Lmax, D))
+
+
+def decode_kv8(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, k_scale: torch.Tensor,
+               v_scale: torch.Tensor, seqlens: torch.Tensor, *, scale: Optional[float] = None,
+               out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None, want_lse: bool = True,
+               workspace: Optional[torch.Tensor] = None, stream=None):
+    """Decode against an 8-bit cache.  q [B,Hq,Lq,D] (or [B,Hq,D]) bf16; caches [B,Hkv,Lmax,D] of
+    torch.float8_e4m3fn (E4M3; k_scale / v_scale float32 [Hkv]) or torch.int8 (Q8_0; k_scale / v_scale
+    float16 [B,Hkv,Lmax,D/32]); seqlens int32 [B]; all on one CUDA device."""
+    squeeze = q.dim() == 3
+    if squeeze:
+        q = q.unsqueeze(2)
+    _check_tensor("q", q, torch.bfloat16, 4)
+    if k_cache.dtype == torch.float8_e4m3fn:
+        fmt, sdt, sdim = _native.ATTN_KV_E4M3, torch.float32, 1
+    elif k_cache.dtype == torch.int8:
+        fmt, sdt, sdim = _native.ATTN_KV_Q8_0, torch.float16, 4
+    else:
+        raise TypeError(f"k_cache must be torch.float8_e4m3fn or torch.int8, got {k_cache.dtype}")
+    _check_tensor("k_cache", k_cache, k_cache.dtype, 4)
+    _check_tensor("v_cache", v_cache, k_cache.dtype, 4)
+    _check_tensor("k_scale", k_scale, sdt, sdim)
+    _check_tensor("v_scale", v_scale, sdt, sdim)
+    _check_tensor("seqlens", seqlens, torch.int32, 1)
+    B, Hq, Lq, D = q.shape
+    Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
+    if k_cache.shape[0] != B or k_cache.shape[3] != D or v_cache.shape != k_cache.shape or seqlens.shape[0] != B:
+        raise ValueError("shape mismatch between q, the caches and seqlens")
+    want_scale = (Hkv,) if fmt == _native.ATTN_KV_E4M3 else (B, Hkv, Lmax, D // 32)
+    if tuple(k_scale.shape) != want_scale or tuple(v_scale.shape) != want_scale:
+        raise ValueError(f"k_scale / v_scale must have shape {want_scale}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    need = decode_kv8_workspace_size(B, Hq, Hkv, Lq, Lmax, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    with torch.cuda.device(q.device):
+        st = _native.lib().attn_decode_kv8(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), fmt,
+                                           _ptr(seqlens), _ptr(out), _ptr(lse), B, Hq, Hkv, Lq, Lmax, D,
+                                           float(scale), _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    _native.check(st, "attn_decode_kv8")
+    if squeeze:
+        out = out.squeeze(2) if out.dim() == 4 else out
+        lse = None if lse is None else (lse.squeeze(2) if lse.dim() == 3 else lse)
+    return out, lse
+
+
 def decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, block_table: torch.Tensor,
                  seqlens: torch.Tensor, *, scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
                  lse: Optional[torch.Tensor] = None, want_lse: bool = True, workspace: Optional[torch.Tensor] = None,
@@ -188,8 +241,8 @@ def decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, 
                                              _stream_handle(stream))
     _native.check(st, "attn_decode_paged")
     if squeeze:
-        out = out.squeeze(2)
-        lse = None if lse is None else lse.squeeze(2)
+        out = out.squeeze(2) if out.dim() == 4 else out
+        lse = None if lse is None else (lse.squeeze(2) if lse.dim() == 3 else lse)
     return out, lse
 
 

@@ -22,6 +22,8 @@ ATTN_DEVERR_TIMEOUT = 0x1
 ATTN_DEVERR_SEQLEN = 0x2
 ATTN_DEVERR_PAGE = 0x4
 ATTN_DECODE_NOALLOC_SCRATCH_BYTES = 16 << 20
+ATTN_KV_E4M3 = 1
+ATTN_KV_Q8_0 = 2
 
 # name -> (restype, argtypes): every symbol the header declares
 _vp, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
@@ -36,6 +38,10 @@ SIGNATURES = {
     "attn_decode_paged": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32,
                                  _f32, _vp, _sz, _vp]),
     "attn_decode_noalloc": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp]),
+    "attn_decode_kv8_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32]),
+    "attn_decode_kv8": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
+                               _f32, _vp, _sz, _vp]),
+    "attn_selftest_kv8_convert": (_i32, [_vp, _vp, _i32, _i32, _vp]),
     "attn_selftest_exp2": (_i32, [_vp, _vp, _i32, _vp]),
     "attn_status_string": (ctypes.c_char_p, [_i32]),
     "attn_last_error": (ctypes.c_char_p, []),

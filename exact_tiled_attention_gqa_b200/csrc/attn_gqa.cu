@@ -14,6 +14,7 @@
 #include <mutex>
 
 #include "../../include/attn_gqa.h"
+#include "decode_kv8_sm100.cuh"
 #include "decode_sm100.cuh"
 #include "decode_tc_sm100.cuh"
 #include "prefill_sm100.cuh"
@@ -64,6 +65,39 @@ int encode_bf16_3d(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t d1, 
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for %s", (int)r, what);
+    return ATTN_OK;
+}
+
+// An 8-bit [d2][d1][d0] tensor (d0 bytes innermost) read in boxes of
+// (box0, box1, 1), swizzled to match the box's row length (128 or 64 bytes).
+int encode_u8_3d(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t d1, uint64_t d2, uint32_t box0,
+                 uint32_t box1, const char* what) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the CUDA driver");
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {d0, d0 * d1};
+    cuuint32_t box[3] = {box0, box1, 1};
+    cuuint32_t estr[3] = {1, 1, 1};
+    const CUtensorMapSwizzle swz = (box0 == 128) ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for %s", (int)r, what);
+    return ATTN_OK;
+}
+
+// A 16-bit [d1][d0] tensor read in boxes of (box0, 1), unswizzled.
+int encode_u16_2d(CUtensorMap* map, const void* ptr, uint64_t d0, uint64_t d1, uint32_t box0, const char* what) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the CUDA driver");
+    cuuint64_t dims[2] = {d0, d1};
+    cuuint64_t strides[1] = {d0 * 2};
+    cuuint32_t box[2] = {box0, 1};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(ATTN_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d) for %s", (int)r, what);
     return ATTN_OK;
@@ -161,9 +195,9 @@ struct DecodeLayout {
     size_t o_bytes, lse_off, total;
 };
 
-DecodeLayout decode_layout(int B, int Hq, int Hkv, int Lmax, int D, int Lq = 1) {
+DecodeLayout decode_layout(int B, int Hq, int Hkv, int Lmax, int D, int Lq = 1, bool kv8 = false) {
     DecodeLayout d;
-    d.chunk = decode_chunk(B, Hkv, Lmax, decode_uses_tc(D, (Hq / Hkv) * Lq));
+    d.chunk = decode_chunk(B, Hkv, Lmax, !kv8 && decode_uses_tc(D, (Hq / Hkv) * Lq));
     d.n_splits = (Lmax + d.chunk - 1) / d.chunk;
     const size_t rows = static_cast<size_t>(B) * Hq * Lq * d.n_splits;
     d.o_bytes = align256(rows * D * sizeof(float));
@@ -181,6 +215,71 @@ int launch_decode_split(const CUtensorMap& tk, const CUtensorMap& tv, const Deco
     dim3 grid(prm.n_splits, prm.Hkv, prm.B);
     attn_decode_split_kernel<D, KPW><<<grid, kDecThreads, L::kAlloc, stream>>>(tk, tv, prm);
     return check_launch("attn_decode_split_kernel");
+}
+
+template <int D, int KPW, int FMT>
+int launch_decode_kv8_split(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tks,
+                            const CUtensorMap& tvs, const DecodeParams& prm, cudaStream_t stream) {
+    static int smem_done[64];
+    using L = DecodeKv8Smem<D, FMT>;
+    int st;
+    if ((st = ensure_smem(attn_decode_kv8_kernel<D, KPW, FMT>, L::kAlloc, smem_done)) != ATTN_OK) return st;
+    dim3 grid(prm.n_splits, prm.Hkv, prm.B);
+    attn_decode_kv8_kernel<D, KPW, FMT><<<grid, kDecThreads, L::kAlloc, stream>>>(tk, tv, tks, tvs, prm);
+    return check_launch("attn_decode_kv8_kernel");
+}
+
+template <int D, int FMT>
+int launch_decode_kv8(const void* q, const void* kc, const void* vc, const void* k_scale, const void* v_scale,
+                      const int32_t* seqlens, void* out, float* lse, int B, int Hq, int Hkv, int Lq, int Lmax,
+                      float scale, void* workspace, cudaStream_t stream) {
+    const DecodeLayout lay = decode_layout(B, Hq, Hkv, Lmax, D, Lq, true);
+    CUtensorMap tk, tv, tks, tvs;
+    int st;
+    const uint64_t outer = static_cast<uint64_t>(B) * Hkv;
+    if ((st = encode_u8_3d(&tk, kc, D, static_cast<uint64_t>(Lmax), outer, D, kDecKT, "k_cache")) != ATTN_OK) return st;
+    if ((st = encode_u8_3d(&tv, vc, D, static_cast<uint64_t>(Lmax), outer, D, kDecKT, "v_cache")) != ATTN_OK) return st;
+    if (FMT == kKvFmtQ8_0) {
+        const uint64_t per_row = D / 32;
+        if ((st = encode_u16_2d(&tks, k_scale, per_row * Lmax, outer, kDecKT * (D / 32), "k_scale")) != ATTN_OK)
+            return st;
+        if ((st = encode_u16_2d(&tvs, v_scale, per_row * Lmax, outer, kDecKT * (D / 32), "v_scale")) != ATTN_OK)
+            return st;
+    } else {
+        tks = tk;   // unused
+        tvs = tv;
+    }
+    DecodeParams prm;
+    prm.q = static_cast<const __nv_bfloat16*>(q);
+    prm.seqlens = seqlens;
+    prm.o_part = static_cast<float*>(workspace);
+    prm.lse_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + lay.lse_off);
+    prm.B = B;
+    prm.Hq = Hq;
+    prm.Hkv = Hkv;
+    prm.Lmax = Lmax;
+    prm.G = Hq / Hkv;
+    prm.Lq = Lq;
+    prm.block_table = nullptr;
+    prm.page_size = prm.max_pages = prm.n_pages = 0;
+    prm.chunk = lay.chunk;
+    prm.n_splits = lay.n_splits;
+    prm.scale_log2 = scale * kLog2e;
+    prm.k_scale = (FMT == kKvFmtE4M3) ? static_cast<const float*>(k_scale) : nullptr;
+    prm.v_scale = (FMT == kKvFmtE4M3) ? static_cast<const float*>(v_scale) : nullptr;
+    if (prm.n_splits > 65535 || Hkv > 65535 || B > 65535)
+        return fail(ATTN_ERR_UNSUPPORTED, "decode grid (%d, %d, %d) exceeds launch limits", prm.n_splits, Hkv, B);
+    const int rows = prm.G * Lq;
+    if (rows <= 16)
+        st = launch_decode_kv8_split<D, 16, FMT>(tk, tv, tks, tvs, prm, stream);
+    else if (rows <= 32)
+        st = launch_decode_kv8_split<D, 32, FMT>(tk, tv, tks, tvs, prm, stream);
+    else
+        st = launch_decode_kv8_split<D, 64, FMT>(tk, tv, tks, tvs, prm, stream);
+    if (st != ATTN_OK) return st;
+    const int n_rows = B * Hq * Lq;
+    attn_decode_combine_kernel<D><<<(n_rows + 3) / 4, 128, 0, stream>>>(prm, static_cast<__nv_bfloat16*>(out), lse);
+    return check_launch("attn_decode_combine_kernel");
 }
 
 // Paged cache description (block_table == nullptr: the contiguous layout).
@@ -527,5 +626,80 @@ extern "C" int attn_decode_noalloc(const void* q, const void* k_cache, const voi
     st = (D == 256)   ? launch_decode<256>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, scratch, s)
          : (D == 128) ? launch_decode<128>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, scratch, s)
                       : launch_decode<64>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, scratch, s);
+    return st == ATTN_OK ? ok() : st;
+}
+
+extern "C" size_t attn_decode_kv8_workspace_size(int B, int Hq, int Hkv, int Lq, int Lmax, int D) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Lmax < 1 || Lq < 1 || (D != 64 && D != 128) ||
+        static_cast<long long>(Hq / Hkv) * Lq > 64)
+        return 0;
+    return decode_layout(B, Hq, Hkv, Lmax, D, Lq, true).total;
+}
+
+extern "C" int attn_decode_kv8(const void* q, const void* k_cache, const void* v_cache, const void* k_scale,
+                               const void* v_scale, int kv_format, const int32_t* seqlens, void* out, float* lse,
+                               int B, int Hq, int Hkv, int Lq, int Lmax, int D, float scale, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+    int st = check_common(q, k_cache, v_cache, out, lse, B, Hq, Hkv, Lq, Lmax, D, scale, "Lq", "Lmax");
+    if (st != ATTN_OK) return st;
+    if (kv_format != ATTN_KV_E4M3 && kv_format != ATTN_KV_Q8_0)
+        return fail(ATTN_ERR_INVALID_ARG, "kv_format %d (E4M3 = %d, Q8_0 = %d)", kv_format, ATTN_KV_E4M3,
+                    ATTN_KV_Q8_0);
+    if (Lq < 1) return fail(ATTN_ERR_INVALID_ARG, "Lq must be >= 1");
+    if (Lmax < 1) return fail(ATTN_ERR_INVALID_ARG, "Lmax must be >= 1");
+    if (!seqlens && B > 0) return fail(ATTN_ERR_INVALID_ARG, "null seqlens");
+    if (reinterpret_cast<uintptr_t>(seqlens) & 3u) return fail(ATTN_ERR_INVALID_ARG, "seqlens must be 4-byte aligned");
+    if (B > 0 && (!k_scale || !v_scale)) return fail(ATTN_ERR_INVALID_ARG, "null k_scale or v_scale");
+    if (kv_format == ATTN_KV_E4M3 && ((reinterpret_cast<uintptr_t>(k_scale) | reinterpret_cast<uintptr_t>(v_scale)) & 3u))
+        return fail(ATTN_ERR_INVALID_ARG, "E4M3 scales must be 4-byte aligned");
+    if (kv_format == ATTN_KV_Q8_0) {
+        if (!aligned16(k_scale) || !aligned16(v_scale))
+            return fail(ATTN_ERR_INVALID_ARG, "Q8_0 scale planes must be 16-byte aligned");
+        if (Lmax % 4 != 0) return fail(ATTN_ERR_INVALID_ARG, "Q8_0 caches need Lmax %% 4 == 0 (got %d)", Lmax);
+    }
+    if (D != 64 && D != 128) return fail(ATTN_ERR_UNSUPPORTED, "8-bit cache head dim D=%d (built: 64, 128)", D);
+    if (static_cast<long long>(Hq / Hkv) * Lq > 64)
+        return fail(ATTN_ERR_UNSUPPORTED, "G * Lq = %lld query rows per KV head (8-bit cache: up to 64)",
+                    static_cast<long long>(Hq / Hkv) * Lq);
+    if (static_cast<long long>(B) * Hq * Lq > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "B*Hq*Lq too large");
+    if (B == 0) return ok();
+    const size_t need = decode_layout(B, Hq, Hkv, Lmax, D, Lq, true).total;
+    if (!workspace || workspace_bytes < need)
+        return fail(ATTN_ERR_WORKSPACE, "decode workspace needs %zu bytes, got %zu", need,
+                    workspace ? workspace_bytes : static_cast<size_t>(0));
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+        return fail(ATTN_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (kv_format == ATTN_KV_E4M3)
+        st = (D == 128) ? launch_decode_kv8<128, kKvFmtE4M3>(q, k_cache, v_cache, k_scale, v_scale, seqlens, out, lse,
+                                                              B, Hq, Hkv, Lq, Lmax, scale, workspace, s)
+                        : launch_decode_kv8<64, kKvFmtE4M3>(q, k_cache, v_cache, k_scale, v_scale, seqlens, out, lse,
+                                                             B, Hq, Hkv, Lq, Lmax, scale, workspace, s);
+    else
+        st = (D == 128) ? launch_decode_kv8<128, kKvFmtQ8_0>(q, k_cache, v_cache, k_scale, v_scale, seqlens, out, lse,
+                                                              B, Hq, Hkv, Lq, Lmax, scale, workspace, s)
+                        : launch_decode_kv8<64, kKvFmtQ8_0>(q, k_cache, v_cache, k_scale, v_scale, seqlens, out, lse,
+                                                             B, Hq, Hkv, Lq, Lmax, scale, workspace, s);
+    return st == ATTN_OK ? ok() : st;
+}
+
+namespace attn {
+namespace {
+__global__ void kv8_convert_selftest_kernel(const uint16_t* codes, uint32_t* out, int n, int fmt) {
+    const int i = blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    const uint32_t x = codes[i];
+    out[i] = (fmt == kKvFmtE4M3) ? e4m3x2_to_f16x2(x) : int8x2_to_f16x2(x);
+}
+}  // namespace
+}  // namespace attn
+
+extern "C" int attn_selftest_kv8_convert(const uint16_t* codes, uint32_t* out, int n, int kv_format, void* stream) {
+    if (n < 0 || (n > 0 && (!codes || !out)) || (kv_format != ATTN_KV_E4M3 && kv_format != ATTN_KV_Q8_0))
+        return fail(ATTN_ERR_INVALID_ARG, "bad selftest arguments");
+    if (n == 0) return ok();
+    kv8_convert_selftest_kernel<<<(n + 255) / 256, 256, 0, static_cast<cudaStream_t>(stream)>>>(codes, out, n,
+                                                                                                 kv_format);
+    const int st = check_launch("kv8_convert_selftest_kernel");
     return st == ATTN_OK ? ok() : st;
 }

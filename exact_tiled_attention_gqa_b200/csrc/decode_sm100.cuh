@@ -73,6 +73,8 @@ struct DecodeParams {
     int chunk;                // cache rows per split (multiple of 64)
     int n_splits;
     float scale_log2;
+    const float* k_scale = nullptr;   // 8-bit E4M3 cache: per-KV-head scales [Hkv] (decode_kv8_sm100.cuh)
+    const float* v_scale = nullptr;
 };
 
 __device__ __forceinline__ int decode_seqlen(const DecodeParams& p, int b) {

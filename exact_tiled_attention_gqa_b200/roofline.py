@@ -48,6 +48,14 @@ def decode_bytes(seqlens, B: int, Hq: int, Hkv: int, D: int) -> int:
     return kv + B * Hq * D * 2 * 2 + B * Hq * 4
 
 
+def decode_kv8_bytes(seqlens, B: int, Hq: int, Hkv: int, D: int, q8_0: bool, Lq: int = 1) -> int:
+    """Algorithmic bytes of an 8-bit-cache decode: every valid K and V row once
+    (one byte per element, plus one fp16 scale per 32 values for q8_0), q, out, lse."""
+    per_row = D + (D // 32) * 2 if q8_0 else D
+    kv = sum(int(s) for s in seqlens) * Hkv * per_row * 2
+    return kv + B * Hq * Lq * (D * 2 * 2 + 4)
+
+
 def measured_peaks() -> dict:
     """MEASURED_PEAKS.json if present, else the pool's earlier measurement."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")

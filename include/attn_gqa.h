@@ -234,6 +234,78 @@ int attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache,
                         void* stream);
 
 /*
+ * 8-bit KV cache element formats (attn_decode_kv8).
+ *
+ * The page "Attention Slack" (llama.cpp serving Gemma 4 on one RTX 3090)
+ * runs its server with 8-bit K and V caches (the q8_0 cache type, in its
+ * server configuration); the NVIDIA attention page ("Prefill and decode are
+ * two different tasks") has decode bound by reading the cache, so one byte
+ * per element halves the bytes a token costs.  The pages define neither
+ * format; these are the two this library reads:
+ *
+ *   ATTN_KV_E4M3  OCP FP8 E4M3 codes (1 sign, 4 exponent bits with bias 7,
+ *                 3 mantissa bits; exponent 0 is subnormal; no infinities;
+ *                 S.1111.111 is NaN; largest finite value 448).  Scales:
+ *                 k_scale and v_scale are `const float*` arrays [Hkv] in
+ *                 device memory; element = scale[g] * value(code).
+ *   ATTN_KV_Q8_0  int8 codes (two's complement), one fp16 scale per 32
+ *                 consecutive values of a cache row, as q8_0 blocks are.
+ *                 The codes and the scales are two planes (not interleaved
+ *                 34-byte blocks) so both are TMA-aligned: k_scale and
+ *                 v_scale point to fp16 arrays [B, Hkv, Lmax, D / 32];
+ *                 element [b, g, r, d] = scale[b, g, r, d / 32] * code.
+ */
+#define ATTN_KV_E4M3 1
+#define ATTN_KV_Q8_0 2
+
+/*
+ * attn_decode_kv8_workspace_size -- bytes of scratch attn_decode_kv8 needs
+ * for these sizes.  Returns 0 for sizes attn_decode_kv8 would reject or B == 0.
+ */
+size_t attn_decode_kv8_workspace_size(int B, int Hq, int Hkv, int Lq, int Lmax, int D);
+
+/*
+ * attn_decode_kv8 -- attn_decode_mq (Lq >= 1 new query rows per sequence,
+ * bottom-right against the cache) with an 8-bit K/V cache.
+ *
+ * The result is the exact attention over the dequantised cache: with K and V
+ * replaced by their element values (above), the same O and LSE as
+ * attn_decode_mq.  The MMAs run in f16 with fp32 sums: every E4M3 value and
+ * every int8 value is exact in f16, Q is brought into f16 range by a power of
+ * two per row (exact), and P is rounded to f16.
+ *
+ *   q          [B, Hq, Lq, D]     bf16, read
+ *   k_cache    [B, Hkv, Lmax, D]  8-bit codes (uint8 storage), read; rows at
+ *   v_cache    [B, Hkv, Lmax, D]  or past seqlens[b] are never used (NaN
+ *                                 codes there have no effect)
+ *   k_scale, v_scale              per kv_format (above), read
+ *   kv_format  ATTN_KV_E4M3 or ATTN_KV_Q8_0
+ *   seqlens    [B] int32, read; 0 <= seqlens[b] <= Lmax
+ *   out        [B, Hq, Lq, D] bf16, written;  lse [B, Hq, Lq] fp32 or NULL
+ *   workspace  attn_decode_kv8_workspace_size(...) bytes, 256-byte aligned
+ *   D: 64 or 128.  G * Lq <= 64.  ATTN_KV_Q8_0 needs Lmax % 4 == 0 and
+ *   16-byte aligned scale planes; ATTN_KV_E4M3 4-byte aligned scale arrays.
+ *
+ * Errors: ATTN_ERR_INVALID_ARG (null or misaligned pointers, unknown
+ * kv_format, Lq < 1, Lmax < 1, Q8_0 with Lmax % 4 != 0, Hq % Hkv != 0, bad
+ * scale), ATTN_ERR_UNSUPPORTED (D not 64 or 128, G * Lq > 64),
+ * ATTN_ERR_WORKSPACE, ATTN_ERR_CUDA.  B == 0 returns ATTN_OK.
+ */
+int attn_decode_kv8(const void* q, const void* k_cache, const void* v_cache, const void* k_scale,
+                    const void* v_scale, int kv_format, const int32_t* seqlens, void* out, float* lse,
+                    int B, int Hq, int Hkv, int Lq, int Lmax, int D, float scale, void* workspace,
+                    size_t workspace_bytes, void* stream);
+
+/*
+ * attn_selftest_kv8_convert -- diagnostic: out[i] = the f16x2 (two f16 bit
+ * patterns, code byte 0 in bits 0-15) that attn_decode_kv8 feeds its MMAs for
+ * the two 8-bit codes in codes[i] (byte 0 in bits 0-7), for kv_format
+ * ATTN_KV_E4M3 (the code's value) or ATTN_KV_Q8_0 (the int8 value, unscaled).
+ * Device arrays of n elements; enqueued on `stream`.
+ */
+int attn_selftest_kv8_convert(const uint16_t* codes, uint32_t* out, int n, int kv_format, void* stream);
+
+/*
  * attn_selftest_exp2 -- diagnostic: y[i] = the prefill softmax's FMA-pipe
  * approximation of 2^x[i] (range reduction plus a minimax cubic; relative
  * error about 7.5e-5 for x in [-125, 8], below 2e-4 for x in [-126, -125]

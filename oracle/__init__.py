@@ -62,6 +62,14 @@ def _load():
                 vp, vp, vp, i32, vp, i32, i32, i32, i32, i32, f64, vp, vp, i32]
             lib.oracle_num_threads.restype = i32
             lib.oracle_num_threads.argtypes = [i32]
+            lib.oracle_e4m3_value.restype = f64
+            lib.oracle_e4m3_value.argtypes = [ctypes.c_uint8]
+            lib.oracle_f16_value.restype = f64
+            lib.oracle_f16_value.argtypes = [ctypes.c_uint16]
+            lib.oracle_dequant_kv8.restype = i32
+            lib.oracle_dequant_kv8.argtypes = [vp, i32, vp, i32, i32, i32, i32, vp]
+            lib.oracle_widen.restype = i32
+            lib.oracle_widen.argtypes = [vp, i32, ctypes.c_size_t, vp]
             _lib = lib
     return _lib
 
@@ -160,3 +168,100 @@ def attention_decode(q, k_cache, v_cache, seqlens, scale: float, nthreads: int =
     if rc != 0:
         raise ValueError(f"oracle_attn_decode failed with code {rc}")
     return out, lse
+
+
+KV_E4M3, KV_Q8_0 = 1, 2
+
+
+def e4m3_value(code: int) -> float:
+    """Value of one FP8 E4M3 code (OCP definition; NaN for S.1111.111)."""
+    return float(_load().oracle_e4m3_value(int(code) & 0xFF))
+
+
+def f16_value(bits: int) -> float:
+    """Value of one IEEE binary16 bit pattern."""
+    return float(_load().oracle_f16_value(int(bits) & 0xFFFF))
+
+
+def _raw_bytes(x) -> np.ndarray:
+    """8-bit codes (torch float8 / int8 / uint8 tensor or numpy array) as a uint8 array."""
+    try:
+        import torch  # plumbing only: viewing a CPU tensor's bytes
+        if isinstance(x, torch.Tensor):
+            x = x.detach().cpu().contiguous().view(torch.uint8).numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    x = np.ascontiguousarray(x)
+    if x.dtype.itemsize != 1:
+        raise TypeError("8-bit codes expected")
+    return x.view(np.uint8)
+
+
+def dequantize_kv8(codes, fmt: int, scales) -> np.ndarray:
+    """codes [B,Hkv,L,D] -> fp64 element values.
+
+    fmt KV_E4M3: scales fp32 [Hkv], element = scales[g] * value(code).
+    fmt KV_Q8_0: scales fp16 [B,Hkv,L,D/32], element = scales[b,g,r,d//32] * int8(code).
+    """
+    c = _raw_bytes(codes)
+    if c.ndim != 4:
+        raise ValueError("codes must be [B,Hkv,L,D]")
+    B, Hkv, L, D = c.shape
+    try:
+        import torch
+        if isinstance(scales, torch.Tensor):
+            scales = scales.detach().cpu().contiguous()
+            scales = scales.view(torch.int16).numpy().view(np.uint16) if scales.dtype == torch.float16 \
+                else scales.numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    sc = np.ascontiguousarray(scales)
+    if fmt == KV_E4M3:
+        sc = np.ascontiguousarray(sc, dtype=np.float32)
+        if sc.shape != (Hkv,):
+            raise ValueError("E4M3 scales must be [Hkv]")
+    elif fmt == KV_Q8_0:
+        if sc.dtype == np.float16:
+            sc = sc.view(np.uint16)
+        if sc.dtype != np.uint16 or sc.shape != (B, Hkv, L, D // 32):
+            raise ValueError("Q8_0 scales must be fp16 [B,Hkv,L,D/32]")
+    else:
+        raise ValueError("unknown 8-bit format")
+    out = np.zeros((B, Hkv, L, D), dtype=np.float64)
+    rc = _load().oracle_dequant_kv8(_ptr(c), int(fmt), _ptr(sc), B, Hkv, L, D, _ptr(out))
+    if rc != 0:
+        raise ValueError(f"oracle_dequant_kv8 failed with code {rc}")
+    return out
+
+
+def widen(x) -> np.ndarray:
+    """fp64, fp32 or bf16 input -> fp64 array of the same shape (exact)."""
+    a, dt = _as_input(x)
+    out = np.zeros(a.shape, dtype=np.float64)
+    rc = _load().oracle_widen(_ptr(a), dt, a.size, _ptr(out))
+    if rc != 0:
+        raise ValueError("oracle_widen failed")
+    return out
+
+
+def attention_decode_kv8(q, k_codes, v_codes, fmt: int, k_scale, v_scale, seqlens, scale: float,
+                         nthreads: int = 0):
+    """Lq new query rows per sequence against an 8-bit cache, exactly: the
+    cache is dequantised to fp64 and the rows are the last Lq of sequence b's
+    seqlens[b] rows (bottom-right causal, as attention_prefill with is_causal).
+
+    q [B,Hq,Lq,D]; codes [B,Hkv,Lmax,D]; returns (out [B,Hq,Lq,D], lse [B,Hq,Lq]) fp64.
+    """
+    qd = widen(q)
+    K = dequantize_kv8(k_codes, fmt, k_scale)
+    V = dequantize_kv8(v_codes, fmt, v_scale)
+    sl = np.asarray(seqlens.cpu().numpy() if hasattr(seqlens, "cpu") else seqlens, dtype=np.int64)
+    B, Hq, Lq, D = qd.shape
+    outs = np.zeros((B, Hq, Lq, D), dtype=np.float64)
+    lses = np.zeros((B, Hq, Lq), dtype=np.float64)
+    for b in range(B):
+        n = int(sl[b])
+        o, l = attention_prefill(qd[b:b + 1], np.ascontiguousarray(K[b:b + 1, :, :n]),
+                                 np.ascontiguousarray(V[b:b + 1, :, :n]), scale, True, nthreads=nthreads)
+        outs[b], lses[b] = o[0], l[0]
+    return outs, lses

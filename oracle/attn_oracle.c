@@ -231,3 +231,84 @@ int oracle_attn_decode(const void* q, const void* k_cache, const void* v_cache, 
     }
     return failed ? -2 : 0;
 }
+
+/*
+ * 8-bit KV caches (the library's attn_decode_kv8).  The pages only name the
+ * q8_0 cache type (the llama.cpp server configuration on the "Attention
+ * Slack" page) and define no format; the two formats here are written from
+ * their published definitions:
+ *
+ *   FP8 E4M3 (OCP 8-bit floating point, E4M3): bit 7 sign, bits 6-3 exponent
+ *   e with bias 7, bits 2-0 mantissa m.
+ *     e = 0          : (-1)^s * m * 2^-9            (subnormal, and +-0)
+ *     e = 15, m = 7  : NaN                          (no infinities)
+ *     otherwise      : (-1)^s * (1 + m / 8) * 2^(e - 7)
+ *   Dequantised element [b,g,r,d] = k_scale[g] * value(code) (one fp32 scale
+ *   per KV head).
+ *
+ *   q8_0: int8 codes (two's complement) with one scale per 32 consecutive
+ *   values of a row, the scale an IEEE binary16 number: bit 15 sign, bits
+ *   14-10 exponent e with bias 15, bits 9-0 mantissa m.
+ *     e = 0          : (-1)^s * m * 2^-24
+ *     e = 31         : +-inf (m = 0) or NaN
+ *     otherwise      : (-1)^s * (1 + m / 1024) * 2^(e - 15)
+ *   Dequantised element [b,g,r,d] = scale[b,g,r,d / 32] * code.
+ */
+double oracle_e4m3_value(uint8_t code) {
+    const int s = code >> 7, e = (code >> 3) & 15, m = code & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0)
+        v = ldexp((double)m, -9);
+    else
+        v = ldexp(1.0 + m / 8.0, e - 7);
+    return s ? -v : v;
+}
+
+double oracle_f16_value(uint16_t bits) {
+    const int s = bits >> 15, e = (bits >> 10) & 31, m = bits & 1023;
+    double v;
+    if (e == 31) return m ? NAN : (s ? -INFINITY : INFINITY);
+    if (e == 0)
+        v = ldexp((double)m, -24);
+    else
+        v = ldexp(1.0 + m / 1024.0, e - 15);
+    return s ? -v : v;
+}
+
+enum { ORACLE_KV_E4M3 = 1, ORACLE_KV_Q8_0 = 2 };
+
+/*
+ * codes [B,Hkv,L,D] (uint8) -> out [B,Hkv,L,D] fp64.
+ *   fmt E4M3: scales = float [Hkv]
+ *   fmt Q8_0: scales = binary16 bit patterns [B,Hkv,L,D/32]  (D % 32 == 0)
+ */
+int oracle_dequant_kv8(const uint8_t* codes, int fmt, const void* scales, int B, int Hkv, int L, int D,
+                       double* out) {
+    if (!codes || !scales || !out || B < 0 || Hkv <= 0 || L < 0 || D <= 0) return -1;
+    if (fmt != ORACLE_KV_E4M3 && fmt != ORACLE_KV_Q8_0) return -1;
+    if (fmt == ORACLE_KV_Q8_0 && D % 32 != 0) return -1;
+    for (long bg = 0; bg < (long)B * Hkv; ++bg) {
+        const int g = (int)(bg % Hkv);
+        for (long r = 0; r < L; ++r) {
+            const size_t row = ((size_t)bg * (size_t)L + (size_t)r) * (size_t)D;
+            for (int d = 0; d < D; ++d) {
+                if (fmt == ORACLE_KV_E4M3) {
+                    out[row + d] = (double)((const float*)scales)[g] * oracle_e4m3_value(codes[row + d]);
+                } else {
+                    const size_t srow = ((size_t)bg * (size_t)L + (size_t)r) * (size_t)(D / 32);
+                    const double sc = oracle_f16_value(((const uint16_t*)scales)[srow + d / 32]);
+                    out[row + d] = sc * (double)(int8_t)codes[row + d];
+                }
+            }
+        }
+    }
+    return 0;
+}
+
+/* n elements of the given type (fp64, fp32 or bf16 bits) widened to fp64. */
+int oracle_widen(const void* x, int dtype, size_t n, double* out) {
+    if ((!x && n) || (!out && n) || dtype < ORACLE_F64 || dtype > ORACLE_BF16) return -1;
+    for (size_t i = 0; i < n; ++i) out[i] = load_elem(x, dtype, i);
+    return 0;
+}

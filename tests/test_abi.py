@@ -159,3 +159,28 @@ def test_decode_paged_rejects(lib):
     assert lib.attn_decode_paged_workspace_size(2, 8, 2, 1, 96, 8, 128) == 0
     assert lib.attn_decode_paged_workspace_size(2, 8, 2, 1, 128, 8, 128) == \
         lib.attn_decode_mq_workspace_size(2, 8, 2, 1, 1024, 128)
+
+
+def _decode_kv8(lib, **kw):
+    args = dict(q=A, k=A, v=A, ks=A, vs=A, fmt=1, sl=A, out=A, lse=NULL, B=2, Hq=8, Hkv=2, Lq=1, Lmax=64, D=128,
+                scale=0.1, ws=A, wsb=1 << 30)
+    args.update(kw)
+    return lib.attn_decode_kv8(args["q"], args["k"], args["v"], args["ks"], args["vs"], args["fmt"], args["sl"],
+                               args["out"], args["lse"], args["B"], args["Hq"], args["Hkv"], args["Lq"], args["Lmax"],
+                               args["D"], args["scale"], args["ws"], args["wsb"], None)
+
+
+@pytest.mark.parametrize("bad,code", [
+    (dict(fmt=0), -1), (dict(fmt=3), -1), (dict(ks=NULL), -1), (dict(vs=NULL), -1), (dict(Lq=0), -1),
+    (dict(sl=NULL), -1), (dict(fmt=2, Lmax=66), -1), (dict(D=256), -2), (dict(D=96), -2),
+    (dict(Hq=128, Hkv=1), -2), (dict(Lq=9, Hq=16), -2), (dict(ws=NULL), -3), (dict(wsb=64), -3),
+])
+def test_decode_kv8_rejects(lib, bad, code):
+    assert _decode_kv8(lib, **bad) == code
+
+
+def test_decode_kv8_empty_batch_and_workspace(lib):
+    assert _decode_kv8(lib, B=0) == 0
+    f = lib.attn_decode_kv8_workspace_size
+    assert f(2, 8, 2, 1, 1000, 256) == 0 and f(2, 64, 1, 2, 1000, 128) == 0 and f(0, 8, 2, 1, 64, 128) == 0
+    assert f(2, 8, 2, 1, 1000, 128) > 0 and f(2, 8, 2, 1, 1000, 128) % 256 == 0

@@ -293,3 +293,87 @@ def test_bf16_bits_widen_exactly(oracle_mod):
     c, lc = oracle_mod.attention_prefill(q.float().numpy(), k.float().numpy(), v.float().numpy(),
                                          0.3, True)
     assert np.array_equal(a, c) and np.array_equal(la, lc)
+
+
+# ---------------------------------------------------------------------------
+# 8-bit caches: the element decoders against library routines and closed
+# forms, the scale indexing against a structured input, and the attention
+# against the pinned bf16 oracle on inputs both can represent.
+# ---------------------------------------------------------------------------
+def test_e4m3_values_match_torch_for_all_codes(oracle_mod):
+    codes = np.arange(256, dtype=np.uint8)
+    ours = np.array([oracle_mod.e4m3_value(c) for c in codes])
+    lib = torch.from_numpy(codes).view(torch.float8_e4m3fn).double().numpy()
+    assert np.array_equal(np.isnan(ours), np.isnan(lib))
+    assert np.array_equal(ours[~np.isnan(ours)], lib[~np.isnan(lib)])
+    assert np.isnan(ours).sum() == 2          # S.1111.111 only: no infinities
+    # closed forms from the format definition
+    assert oracle_mod.e4m3_value(0x38) == 1.0
+    assert oracle_mod.e4m3_value(0x7E) == 448.0 and oracle_mod.e4m3_value(0xFE) == -448.0
+    assert oracle_mod.e4m3_value(0x01) == 2.0 ** -9 and oracle_mod.e4m3_value(0x08) == 2.0 ** -6
+    assert oracle_mod.e4m3_value(0x07) == 7 * 2.0 ** -9
+    assert math.copysign(1.0, oracle_mod.e4m3_value(0x80)) == -1.0 and oracle_mod.e4m3_value(0x80) == 0.0
+
+
+def test_f16_values_match_numpy_for_all_patterns(oracle_mod):
+    bits = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+    ours = np.array([oracle_mod.f16_value(b) for b in bits[::7]] + [oracle_mod.f16_value(b) for b in
+                                                                      (0x0001, 0x03FF, 0x0400, 0x7BFF, 0x7C00)])
+    lib = np.concatenate([bits[::7], np.array([0x0001, 0x03FF, 0x0400, 0x7BFF, 0x7C00], np.uint16)])
+    lib = lib.view(np.float16).astype(np.float64)
+    assert np.array_equal(np.isnan(ours), np.isnan(lib))
+    ok = ~np.isnan(ours)
+    assert np.array_equal(ours[ok], lib[ok])
+    assert oracle_mod.f16_value(0x0001) == 2.0 ** -24 and oracle_mod.f16_value(0x7BFF) == 65504.0
+
+
+def test_q8_0_scale_indexing(oracle_mod):
+    """Each scale is a distinct integer naming (b, g, r, block) (exact in fp16); code 1
+    everywhere shows which scale every element used, and code -3 checks the int8 sign."""
+    B, Hkv, L, D = 2, 3, 5, 64
+    name = np.zeros((B, Hkv, L, D // 32), dtype=np.int64)
+    for b in range(B):
+        for g in range(Hkv):
+            for r in range(L):
+                for c in range(D // 32):
+                    name[b, g, r, c] = 1 + ((b * Hkv + g) * L + r) * 2 + c
+    scales = name.astype(np.float16)
+    codes = np.ones((B, Hkv, L, D), dtype=np.uint8)
+    codes[..., 5] = np.uint8(256 - 3)
+    out = oracle_mod.dequantize_kv8(codes, oracle_mod.KV_Q8_0, scales)
+    for d in (0, 5, 31, 32, 63):
+        want = name[..., d // 32].astype(np.float64) * (-3 if d == 5 else 1)
+        assert np.array_equal(out[..., d], want), d
+
+
+def test_e4m3_per_head_scale(oracle_mod):
+    codes = np.full((2, 3, 4, 32), 0x38, dtype=np.uint8)     # value 1.0
+    scales = np.array([0.5, 2.0, -4.0], dtype=np.float32)
+    out = oracle_mod.dequantize_kv8(codes, oracle_mod.KV_E4M3, scales)
+    for g in range(3):
+        assert np.all(out[:, g] == scales[g])
+
+
+def test_kv8_attention_equals_bf16_oracle_on_shared_values(oracle_mod):
+    """Unit scales and codes whose values are exact in bf16: the 8-bit oracle must
+    equal the pinned bf16 decode oracle (last row of a causal prefill) on the same values."""
+    rng = np.random.default_rng(4)
+    B, Hq, Hkv, L, D = 2, 4, 2, 40, 64
+    q = torch.randn(B, Hq, 1, D, generator=torch.Generator().manual_seed(4)).to(torch.bfloat16)
+    seqlens = np.array([40, 17])
+    for fmt in (oracle_mod.KV_E4M3, oracle_mod.KV_Q8_0):
+        if fmt == oracle_mod.KV_E4M3:
+            pool = np.array([c for c in range(256) if abs(oracle_mod.e4m3_value(c)) <= 4.0], dtype=np.uint8)
+            kc = rng.choice(pool, size=(B, Hkv, L, D)).astype(np.uint8)
+            vc = rng.choice(pool, size=(B, Hkv, L, D)).astype(np.uint8)
+            ks = vs = np.ones(Hkv, np.float32)
+        else:
+            kc = rng.integers(-4, 5, size=(B, Hkv, L, D)).astype(np.int8).view(np.uint8)
+            vc = rng.integers(-4, 5, size=(B, Hkv, L, D)).astype(np.int8).view(np.uint8)
+            ks = vs = np.ones((B, Hkv, L, D // 32), np.float16)
+        o8, l8 = oracle_mod.attention_decode_kv8(q, kc, vc, fmt, ks, vs, seqlens, 0.125)
+        kf = torch.from_numpy(oracle_mod.dequantize_kv8(kc, fmt, ks)).to(torch.bfloat16)
+        vf = torch.from_numpy(oracle_mod.dequantize_kv8(vc, fmt, vs)).to(torch.bfloat16)
+        assert torch.equal(kf.double(), torch.from_numpy(oracle_mod.dequantize_kv8(kc, fmt, ks)))  # exact in bf16
+        ob, lb = oracle_mod.attention_decode(q[:, :, 0], kf, vf, seqlens.astype(np.int32), 0.125)
+        assert np.allclose(o8[:, :, 0], ob, rtol=0, atol=1e-12) and np.allclose(l8[:, :, 0], lb, rtol=0, atol=1e-12)
