@@ -229,6 +229,18 @@ int launch_decode_kv8_split(const CUtensorMap& tk, const CUtensorMap& tv, const 
     return check_launch("attn_decode_kv8_kernel");
 }
 
+template <int D, int NR, int FMT>
+int launch_decode_kv8t(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tks, const CUtensorMap& tvs,
+                       const DecodeParams& prm, cudaStream_t stream) {
+    static int smem_done[64];
+    using L = DecodeKv8tSmem<D, FMT>;
+    int st;
+    if ((st = ensure_smem(attn_decode_kv8t_kernel<D, NR, FMT>, L::kAlloc, smem_done)) != ATTN_OK) return st;
+    dim3 grid(prm.n_splits, prm.Hkv, prm.B);
+    attn_decode_kv8t_kernel<D, NR, FMT><<<grid, kDecThreads, L::kAlloc, stream>>>(tk, tv, tks, tvs, prm);
+    return check_launch("attn_decode_kv8t_kernel");
+}
+
 template <int D, int FMT>
 int launch_decode_kv8(const void* q, const void* kc, const void* vc, const void* k_scale, const void* v_scale,
                       const int32_t* seqlens, void* out, float* lse, int B, int Hq, int Hkv, int Lq, int Lmax,
@@ -270,8 +282,10 @@ int launch_decode_kv8(const void* q, const void* kc, const void* vc, const void*
     if (prm.n_splits > 65535 || Hkv > 65535 || B > 65535)
         return fail(ATTN_ERR_UNSUPPORTED, "decode grid (%d, %d, %d) exceeds launch limits", prm.n_splits, Hkv, B);
     const int rows = prm.G * Lq;
-    if (rows <= 16)
-        st = launch_decode_kv8_split<D, 16, FMT>(tk, tv, tks, tvs, prm, stream);
+    if (rows <= 8)
+        st = launch_decode_kv8t<D, 1, FMT>(tk, tv, tks, tvs, prm, stream);
+    else if (rows <= 16)
+        st = launch_decode_kv8t<D, 2, FMT>(tk, tv, tks, tvs, prm, stream);
     else if (rows <= 32)
         st = launch_decode_kv8_split<D, 32, FMT>(tk, tv, tks, tvs, prm, stream);
     else

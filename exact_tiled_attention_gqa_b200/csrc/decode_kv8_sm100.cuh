@@ -28,8 +28,13 @@
 // P is rounded to f16 (11 significant bits), a finer grid than the bf16 P of
 // the other kernels.
 //
-// Shared-memory reads without bank conflicts.  A cache tile is 64 rows x D
-// bytes, TMA-swizzled (128-byte swizzle for D = 128, 64-byte for D = 64).
+// Two kernels: attn_decode_kv8t_kernel (below) for up to 16 query rows per KV
+// head, with the cache rows as the MMA's M dimension, and
+// attn_decode_kv8_kernel for 17 to 64 rows, with the query rows as M.
+//
+// Shared-memory reads without bank conflicts (row-major kernel; the
+// transposed one is described with it).  A cache tile is 64 rows x D bytes,
+// TMA-swizzled (128-byte swizzle for D = 128, 64-byte for D = 64).
 //  - K (the B operand of S = Q K^T): the MMA sums over d, so any d order used
 //    by both Q and K is valid.  Lane (grp, tq) takes the 4 contiguous bytes
 //    d = 16 kk + 4 tq .. + 3 of key grp as its k slots {2tq, 2tq+1, 2tq+8,
@@ -78,13 +83,20 @@ __device__ __forceinline__ uint32_t kv8_swz(int row, int col) {
         return static_cast<uint32_t>(row * 64 + ((((col >> 4) ^ (row >> 1)) & 3) << 4) + (col & 15));
 }
 
-// two codes (bytes 0 and 1 of x) -> f16x2
+// A 32-bit word of codes as the converters below take it: E4M3 codes as they
+// are, int8 codes in offset form (sign bits flipped once per word, not per pair).
+template <int FMT>
+__device__ __forceinline__ uint32_t kv8_word(uint32_t raw) {
+    return FMT == kKvFmtE4M3 ? raw : raw ^ 0x80808080u;
+}
+
+// two codes (bytes 0 and 1 of a kv8_word) -> f16x2
 template <int FMT>
 __device__ __forceinline__ uint32_t kv8_pair(uint32_t x) {
     if constexpr (FMT == kKvFmtE4M3)
         return e4m3x2_to_f16x2(x);
     else
-        return int8x2_to_f16x2(x);
+        return offset_u8x2_to_f16x2(x);
 }
 
 // KPW = cache rows of each 64-row tile handled by one compute warp (16, 32 or 64).
@@ -258,7 +270,7 @@ __global__ void __maxnreg__(200)
 #pragma unroll
                 for (int nt = 0; nt < kNT; ++nt) {
                     const int key_local = key_off + nt * 8 + grp;
-                    const uint32_t w = ld_shared_u32(kbase + kv8_swz<D>(key_local, kk * 16 + 4 * tq));
+                    const uint32_t w = kv8_word<FMT>(ld_shared_u32(kbase + kv8_swz<D>(key_local, kk * 16 + 4 * tq)));
                     mma_f16_16816(FMT == kKvFmtQ8_0 ? bacc[nt] : sacc[nt], qa[kk], kv8_pair<FMT>(w),
                                   kv8_pair<FMT>(w >> 16));
                 }
@@ -357,10 +369,10 @@ __global__ void __maxnreg__(200)
                     a[3] = pack_f16x2(pb8 * s8, pb9 * s9);
                 }
                 const int col = c * 32 + 4 * grp;
-                const uint32_t w0 = v0 ? ld_shared_u32(vbase + kv8_swz<D>(klo, col)) : 0u;
-                const uint32_t w1 = v1 ? ld_shared_u32(vbase + kv8_swz<D>(klo + 1, col)) : 0u;
-                const uint32_t w8 = v8 ? ld_shared_u32(vbase + kv8_swz<D>(klo + 8, col)) : 0u;
-                const uint32_t w9 = v9 ? ld_shared_u32(vbase + kv8_swz<D>(klo + 9, col)) : 0u;
+                const uint32_t w0 = kv8_word<FMT>(v0 ? ld_shared_u32(vbase + kv8_swz<D>(klo, col)) : 0u);
+                const uint32_t w1 = kv8_word<FMT>(v1 ? ld_shared_u32(vbase + kv8_swz<D>(klo + 1, col)) : 0u);
+                const uint32_t w8 = kv8_word<FMT>(v8 ? ld_shared_u32(vbase + kv8_swz<D>(klo + 8, col)) : 0u);
+                const uint32_t w9 = kv8_word<FMT>(v9 ? ld_shared_u32(vbase + kv8_swz<D>(klo + 9, col)) : 0u);
                 // key pairs of byte i: {w0.i, w1.i} and {w8.i, w9.i}; two bytes per permute
                 const uint32_t lo01 = prmt(w0, w1, 0x5140u), hi01 = prmt(w0, w1, 0x7362u);
                 const uint32_t lo89 = prmt(w8, w9, 0x5140u), hi89 = prmt(w8, w9, 0x7362u);
@@ -417,6 +429,367 @@ __global__ void __maxnreg__(200)
             const float sc = (mw == -INFINITY) ? 0.0f : ex2_approx(mw - M);
             Lsum += sm_l[ww * 16 + rr] * sc;
             acc += sm_o[(ww * 16 + rr) * D + d] * sc;
+        }
+        const size_t prow = (group_row0 + row) * p.n_splits + split;
+        p.o_part[prow * D + d] = (Lsum > 0.0f) ? acc * vscale / Lsum : 0.0f;
+        if (d == 0) p.lse_part[prow] = (Lsum > 0.0f) ? M + __log2f(Lsum) : -INFINITY;
+    }
+}
+
+// ---------------------------------------------------------------------------
+// Up to 16 query rows per KV head (NR = 1 or 2 groups of 8): the transposed
+// form.  With R <= 16 rows, an m16 MMA over query rows is mostly padding, so
+// the cache rows take the M dimension instead:
+//   S^T = K Q^T     M = 16 cache rows, N = 8 query rows, K = 16 columns of d
+//   O^T = V^T P^T   M = 16 columns of d, N = 8 query rows, K = 16 cache rows
+// Half the MMAs and half the accumulator registers of the row-major form, so
+// more CTAs fit on an SM.  The S^T accumulator holds a cache row per lane
+// group and query rows across the quad; P^T reaches the B-operand layout of
+// the second MMA by one 8x8 transpose (movmatrix) per 8 cache rows.
+//  - K (A operand of S^T): lane (grp, tq) loads the 4 bytes d = 16 kk + 4 tq
+//    .. + 3 of cache rows grp and grp + 8 (Q's B fragments use the same d order).
+//  - V^T (A operand of O^T): lane loads 4 bytes d = 32 c + 4 grp .. + 3 of cache
+//    rows 2 tq, 2 tq + 1, 2 tq + 8, 2 tq + 9 and byte-permutes them into the key
+//    pairs of two M tiles: M tile (c, h) row grp holds d = 32 c + 4 grp + 2 h,
+//    row grp + 8 holds d + 1.
+template <int D, int FMT>
+struct DecodeKv8tSmem {
+    static constexpr int kTileBytes = kDecKT * D;
+    static constexpr int kScaleBytes = (FMT == kKvFmtQ8_0) ? kDecKT * (D / 32) * 2 : 0;
+    static constexpr int kVOff = kTileBytes;
+    static constexpr int kKsOff = 2 * kTileBytes;
+    static constexpr int kVsOff = kKsOff + kScaleBytes;
+    static constexpr int kStageBytes = ((2 * kTileBytes + 2 * kScaleBytes) + 1023) & ~1023;
+    static constexpr int kStageTx = 2 * kTileBytes + 2 * kScaleBytes;
+    // 3 (D = 128) or 5 (D = 64) stages: four CTAs fit in an SM's shared memory,
+    // with 192 KB of cache rows in flight per SM
+    static constexpr int kStages = (D == 128) ? 3 : 5;
+    static constexpr int kRingBytes = kStages * kStageBytes;
+    // merge area (reuses the ring): m[4][16], l[4][16], O[4][16][D]
+    static constexpr int kMergeBytes = 4 * 16 * 4 * 2 + 4 * 16 * D * 4;
+    static_assert(kMergeBytes <= kRingBytes, "merge area must fit in the ring");
+    static constexpr int kBarOff = kRingBytes;
+    static constexpr int kBytes = kBarOff + 2 * kStages * 8 + 16;
+    static constexpr int kAlloc = kBytes + 1024;
+};
+
+// CTAs per SM the register budget is sized for (one query-row group: 4; two: 2)
+template <int NR>
+constexpr int kv8t_min_blocks() { return NR == 1 ? 4 : 2; }
+
+template <int D, int NR, int FMT>
+__global__ void __launch_bounds__(kDecThreads, kv8t_min_blocks<NR>())
+    attn_decode_kv8t_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                            const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
+                            const DecodeParams p) {
+    using L = DecodeKv8tSmem<D, FMT>;
+    constexpr int kBlk = D / 32;
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw_base = smem_u32(smem_raw);
+    const uint32_t base = (raw_base + 1023u) & ~1023u;
+    uint8_t* smem = smem_raw + (base - raw_base);
+
+    const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
+    const int seqlen = decode_seqlen(p, b);
+    const int k_begin = split * p.chunk;
+    if (k_begin >= seqlen) return;   // uniform: this split has no rows
+    const int k_end = min(k_begin + p.chunk, seqlen);
+    const int n_tiles = (k_end - k_begin + kDecKT - 1) / kDecKT;
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const uint32_t ring = base;
+    const uint32_t bar0 = base + L::kBarOff;
+    auto bar_full = [&](int s) { return bar0 + 8u * s; };
+    auto bar_empty = [&](int s) { return bar0 + 8u * (L::kStages + s); };
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kBarOff + 2 * L::kStages * 8);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < L::kStages; ++s) {
+            mbar_init(bar_full(s), 1);
+            mbar_init(bar_empty(s), 4);
+        }
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp == 4) {
+        // ================= TMA producer =================
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_k);
+            tma_prefetch_desc(&tm_v);
+            if constexpr (FMT == kKvFmtQ8_0) {
+                tma_prefetch_desc(&tm_ks);
+                tma_prefetch_desc(&tm_vs);
+            }
+            const int outer = b * p.Hkv + g;
+            int issued = 0;
+            for (int t = 0; t < n_tiles; ++t) {
+                const int s = t % L::kStages;
+                const uint32_t round = static_cast<uint32_t>(t / L::kStages);
+                const int key0 = k_begin + t * kDecKT;
+                if (!mbar_wait(bar_empty(s), (round & 1u) ^ 1u, abort_flag, &g_attn_err, kDevErrTimeout)) break;
+                mbar_arrive_expect_tx(bar_full(s), L::kStageTx);
+                const uint32_t dst = ring + s * L::kStageBytes;
+                tma_load_3d(dst, &tm_k, bar_full(s), 0, key0, outer);
+                tma_load_3d(dst + L::kVOff, &tm_v, bar_full(s), 0, key0, outer);
+                if constexpr (FMT == kKvFmtQ8_0) {
+                    tma_load_2d(dst + L::kKsOff, &tm_ks, bar_full(s), key0 * kBlk, outer);
+                    tma_load_2d(dst + L::kVsOff, &tm_vs, bar_full(s), key0 * kBlk, outer);
+                }
+                issued = t + 1;
+            }
+            if (issued < n_tiles) {
+                for (int t = max(0, issued - L::kStages); t < issued; ++t) {
+                    const uint64_t t0 = global_timer_ns();
+                    while (!mbar_try_wait(bar_full(t % L::kStages), static_cast<uint32_t>(t / L::kStages) & 1u) &&
+                           global_timer_ns() - t0 < 100000000ull) {
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        return;
+    }
+
+    // ================= compute warps: warp w owns cache rows 16 w .. 16 w + 15 of each tile =================
+    const int grp = lane >> 2, tq = lane & 3;
+    const int key_off = warp * 16;
+    const int R = p.G * p.Lq;
+    const size_t group_row0 = (static_cast<size_t>(b) * p.Hq + static_cast<size_t>(g) * p.G) * p.Lq;
+    const int lim_lo = min(k_end, seqlen - p.Lq + 1);
+
+    // ---- Q^T as B fragments: n-tile j, column grp = query row 8 j + grp; rows
+    // scaled by 2^-e into f16 range (e per row, folded into that row's score scale) ----
+    uint32_t qb[D / 16][NR][2];
+    float sl2[NR][2];   // score scale of the rows this lane's accumulators hold: 8 j + 2 tq (+1)
+    int lim[NR][2];
+    {
+        const float ks = (FMT == kKvFmtE4M3) ? p.k_scale[g] : 1.0f;
+#pragma unroll
+        for (int j = 0; j < NR; ++j) {
+            const int r = 8 * j + grp;
+            const bool valid = r < R;
+            const uint2* qrow = reinterpret_cast<const uint2*>(p.q + (group_row0 + (valid ? r : 0)) * D);
+            uint2 w[D / 16];
+            float mx = 0.0f;
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                w[kk] = valid ? __ldg(qrow + 4 * kk + tq) : make_uint2(0u, 0u);
+                mx = fmaxf(mx, fmaxf(fmaxf(fabsf(__uint_as_float(w[kk].x << 16)),
+                                           fabsf(__uint_as_float(w[kk].x & 0xffff0000u))),
+                                     fmaxf(fabsf(__uint_as_float(w[kk].y << 16)),
+                                           fabsf(__uint_as_float(w[kk].y & 0xffff0000u)))));
+            }
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
+            int e = 0;
+            if (mx > 0.0f && mx < INFINITY) e = max(-100, min(100, static_cast<int>((__float_as_uint(mx) >> 23) & 0xff) - 141));
+            const float f = __uint_as_float(static_cast<uint32_t>(127 - e) << 23);
+#pragma unroll
+            for (int kk = 0; kk < D / 16; ++kk) {
+                qb[kk][j][0] = pack_f16x2(__uint_as_float(w[kk].x << 16) * f, __uint_as_float(w[kk].x & 0xffff0000u) * f);
+                qb[kk][j][1] = pack_f16x2(__uint_as_float(w[kk].y << 16) * f, __uint_as_float(w[kk].y & 0xffff0000u) * f);
+            }
+            // the exponents of rows 8 j + 2 tq and 8 j + 2 tq + 1 live in lanes 8 tq and 8 tq + 4
+            const int e0 = __shfl_sync(0xffffffffu, e, 8 * tq);
+            const int e1 = __shfl_sync(0xffffffffu, e, 8 * tq + 4);
+            sl2[j][0] = p.scale_log2 * ks * __uint_as_float(static_cast<uint32_t>(127 + e0) << 23);
+            sl2[j][1] = p.scale_log2 * ks * __uint_as_float(static_cast<uint32_t>(127 + e1) << 23);
+            const int r0 = 8 * j + 2 * tq;
+            lim[j][0] = min(k_end, seqlen - p.Lq + r0 % p.Lq + 1);
+            lim[j][1] = min(k_end, seqlen - p.Lq + (r0 + 1) % p.Lq + 1);
+        }
+    }
+
+    float oacc[D / 16][NR][4];
+#pragma unroll
+    for (int mt = 0; mt < D / 16; ++mt)
+#pragma unroll
+        for (int j = 0; j < NR; ++j) oacc[mt][j][0] = oacc[mt][j][1] = oacc[mt][j][2] = oacc[mt][j][3] = 0.0f;
+    float m_run[NR][2], l_run[NR][2];
+#pragma unroll
+    for (int j = 0; j < NR; ++j) {
+        m_run[j][0] = m_run[j][1] = -INFINITY;
+        l_run[j][0] = l_run[j][1] = 0.0f;
+    }
+    bool ok = true;
+
+    for (int t = 0; t < n_tiles; ++t) {
+        const int s = t % L::kStages;
+        ok = mbar_wait(bar_full(s), static_cast<uint32_t>(t / L::kStages) & 1u, abort_flag, &g_attn_err, kDevErrTimeout);
+        if (!ok) break;
+        const uint32_t kbase = ring + s * L::kStageBytes;
+        const uint32_t vbase = kbase + L::kVOff;
+        const __half* ks_tile = reinterpret_cast<const __half*>(smem + s * L::kStageBytes + L::kKsOff);
+        const __half* vs_tile = reinterpret_cast<const __half*>(smem + s * L::kStageBytes + L::kVsOff);
+        const int tile_key0 = k_begin + t * kDecKT + key_off;   // absolute row of this warp's cache row 0
+        const bool tail = (k_begin + (t + 1) * kDecKT > k_end);
+        const bool masked = (k_begin + (t + 1) * kDecKT > lim_lo);
+
+        // ---- S^T = K Q^T: rows key_off + grp (c0, c1) and + 8 (c2, c3), columns 8 j + 2 tq (+1) ----
+        float sacc[NR][4];
+#pragma unroll
+        for (int j = 0; j < NR; ++j) sacc[j][0] = sacc[j][1] = sacc[j][2] = sacc[j][3] = 0.0f;
+#pragma unroll
+        for (int c = 0; c < kBlk; ++c) {
+            float bacc[NR][4];
+#pragma unroll
+            for (int j = 0; j < NR; ++j) bacc[j][0] = bacc[j][1] = bacc[j][2] = bacc[j][3] = 0.0f;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int kk = 2 * c + h;
+                const uint32_t wl = kv8_word<FMT>(ld_shared_u32(kbase + kv8_swz<D>(key_off + grp, kk * 16 + 4 * tq)));
+                const uint32_t wh =
+                    kv8_word<FMT>(ld_shared_u32(kbase + kv8_swz<D>(key_off + grp + 8, kk * 16 + 4 * tq)));
+                const uint32_t a[4] = {kv8_pair<FMT>(wl), kv8_pair<FMT>(wh), kv8_pair<FMT>(wl >> 16),
+                                       kv8_pair<FMT>(wh >> 16)};
+#pragma unroll
+                for (int j = 0; j < NR; ++j)
+                    mma_f16_16816(FMT == kKvFmtQ8_0 ? bacc[j] : sacc[j], a, qb[kk][j][0], qb[kk][j][1]);
+            }
+            if constexpr (FMT == kKvFmtQ8_0) {
+                const float s_lo = __half2float(ks_tile[(key_off + grp) * kBlk + c]);
+                const float s_hi = __half2float(ks_tile[(key_off + grp + 8) * kBlk + c]);
+#pragma unroll
+                for (int j = 0; j < NR; ++j) {
+                    sacc[j][0] = fmaf(bacc[j][0], s_lo, sacc[j][0]);
+                    sacc[j][1] = fmaf(bacc[j][1], s_lo, sacc[j][1]);
+                    sacc[j][2] = fmaf(bacc[j][2], s_hi, sacc[j][2]);
+                    sacc[j][3] = fmaf(bacc[j][3], s_hi, sacc[j][3]);
+                }
+            }
+        }
+        // ---- masking, online softmax per query row (a column of S^T) ----
+        const int key_lo = tile_key0 + grp, key_hi = key_lo + 8;
+#pragma unroll
+        for (int j = 0; j < NR; ++j) {
+            if (masked) {
+                if (key_lo >= lim[j][0]) sacc[j][0] = -INFINITY;
+                if (key_lo >= lim[j][1]) sacc[j][1] = -INFINITY;
+                if (key_hi >= lim[j][0]) sacc[j][2] = -INFINITY;
+                if (key_hi >= lim[j][1]) sacc[j][3] = -INFINITY;
+            }
+            float mx0 = fmaxf(sacc[j][0], sacc[j][2]), mx1 = fmaxf(sacc[j][1], sacc[j][3]);
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) {
+                mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, o));
+                mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, o));
+            }
+            const float mn0 = fmaxf(m_run[j][0], mx0 * sl2[j][0]), mn1 = fmaxf(m_run[j][1], mx1 * sl2[j][1]);
+            const float f0 = (m_run[j][0] == -INFINITY) ? 0.0f : ex2_approx(m_run[j][0] - mn0);
+            const float f1 = (m_run[j][1] == -INFINITY) ? 0.0f : ex2_approx(m_run[j][1] - mn1);
+            const float ms0 = (mn0 == -INFINITY) ? 0.0f : mn0;
+            const float ms1 = (mn1 == -INFINITY) ? 0.0f : mn1;
+            m_run[j][0] = mn0;
+            m_run[j][1] = mn1;
+            sacc[j][0] = ex2_approx(fmaf(sacc[j][0], sl2[j][0], -ms0));
+            sacc[j][1] = ex2_approx(fmaf(sacc[j][1], sl2[j][1], -ms1));
+            sacc[j][2] = ex2_approx(fmaf(sacc[j][2], sl2[j][0], -ms0));
+            sacc[j][3] = ex2_approx(fmaf(sacc[j][3], sl2[j][1], -ms1));
+            l_run[j][0] = l_run[j][0] * f0 + (sacc[j][0] + sacc[j][2]);
+            l_run[j][1] = l_run[j][1] * f1 + (sacc[j][1] + sacc[j][3]);
+            if (__any_sync(0xffffffffu, f0 != 1.0f || f1 != 1.0f)) {
+#pragma unroll
+                for (int mt = 0; mt < D / 16; ++mt) {
+                    oacc[mt][j][0] *= f0;
+                    oacc[mt][j][1] *= f1;
+                    oacc[mt][j][2] *= f0;
+                    oacc[mt][j][3] *= f1;
+                }
+            }
+        }
+        // ---- O^T += V^T P^T ----
+        // cache rows past the valid length may hold anything (NaN codes or scales included)
+        const bool k0v = !tail || key_lo < k_end, k8v = !tail || key_hi < k_end;
+        const int vk = key_off + 2 * tq;           // this lane's V rows: vk, vk+1, vk+8, vk+9
+        const int vabs = tile_key0 + 2 * tq;
+        const bool v0 = !tail || vabs < k_end, v1 = !tail || vabs + 1 < k_end;
+        const bool v8 = !tail || vabs + 8 < k_end, v9 = !tail || vabs + 9 < k_end;
+        uint32_t pb[NR][2];   // P^T B fragments (E4M3: one set for all column blocks)
+        if constexpr (FMT == kKvFmtE4M3) {
+#pragma unroll
+            for (int j = 0; j < NR; ++j) {
+                pb[j][0] = movmatrix_trans(pack_f16x2(sacc[j][0], sacc[j][1]));
+                pb[j][1] = movmatrix_trans(pack_f16x2(sacc[j][2], sacc[j][3]));
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < kBlk; ++c) {
+            if constexpr (FMT == kKvFmtQ8_0) {
+                const float s_lo = k0v ? __half2float(vs_tile[(key_off + grp) * kBlk + c]) : 0.0f;
+                const float s_hi = k8v ? __half2float(vs_tile[(key_off + grp + 8) * kBlk + c]) : 0.0f;
+#pragma unroll
+                for (int j = 0; j < NR; ++j) {
+                    pb[j][0] = movmatrix_trans(pack_f16x2(sacc[j][0] * s_lo, sacc[j][1] * s_lo));
+                    pb[j][1] = movmatrix_trans(pack_f16x2(sacc[j][2] * s_hi, sacc[j][3] * s_hi));
+                }
+            }
+            const int col = c * 32 + 4 * grp;
+            const uint32_t w0 = kv8_word<FMT>(v0 ? ld_shared_u32(vbase + kv8_swz<D>(vk, col)) : 0u);
+            const uint32_t w1 = kv8_word<FMT>(v1 ? ld_shared_u32(vbase + kv8_swz<D>(vk + 1, col)) : 0u);
+            const uint32_t w8 = kv8_word<FMT>(v8 ? ld_shared_u32(vbase + kv8_swz<D>(vk + 8, col)) : 0u);
+            const uint32_t w9 = kv8_word<FMT>(v9 ? ld_shared_u32(vbase + kv8_swz<D>(vk + 9, col)) : 0u);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const uint32_t sel = h ? 0x7362u : 0x5140u;
+                const uint32_t p01 = prmt(w0, w1, sel), p89 = prmt(w8, w9, sel);
+                const uint32_t a[4] = {kv8_pair<FMT>(p01), kv8_pair<FMT>(p01 >> 16), kv8_pair<FMT>(p89),
+                                       kv8_pair<FMT>(p89 >> 16)};
+#pragma unroll
+                for (int j = 0; j < NR; ++j) mma_f16_16816(oacc[2 * c + h][j], a, pb[j][0], pb[j][1]);
+            }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_empty(s));
+    }
+
+    // ---- merge the four warps' key slices through shared memory ----
+#pragma unroll
+    for (int j = 0; j < NR; ++j)
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+#pragma unroll
+            for (int o = 4; o < 32; o <<= 1) l_run[j][i] += __shfl_xor_sync(0xffffffffu, l_run[j][i], o);
+    asm volatile("bar.sync 1, 128;" ::: "memory");   // every compute warp is done with the ring
+    float* sm_m = reinterpret_cast<float*>(smem);
+    float* sm_l = sm_m + 4 * 16;
+    float* sm_o = sm_l + 4 * 16;
+#pragma unroll
+    for (int j = 0; j < NR; ++j) {
+        const int r0 = 8 * j + 2 * tq;
+        if (grp == 0) {
+            sm_m[warp * 16 + r0] = m_run[j][0];
+            sm_m[warp * 16 + r0 + 1] = m_run[j][1];
+            sm_l[warp * 16 + r0] = l_run[j][0];
+            sm_l[warp * 16 + r0 + 1] = l_run[j][1];
+        }
+#pragma unroll
+        for (int mt = 0; mt < D / 16; ++mt) {
+            const int d = (mt >> 1) * 32 + 4 * grp + 2 * (mt & 1);   // row grp; row grp + 8 is d + 1
+            float* o0 = sm_o + (warp * 16 + r0) * D;
+            float* o1 = o0 + D;
+            o0[d] = oacc[mt][j][0];
+            o1[d] = oacc[mt][j][1];
+            o0[d + 1] = oacc[mt][j][2];
+            o1[d + 1] = oacc[mt][j][3];
+        }
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (!ok) return;
+    const float vscale = (FMT == kKvFmtE4M3) ? p.v_scale[g] : 1.0f;
+    for (int idx = threadIdx.x; idx < R * D; idx += 128) {
+        const int row = idx / D, d = idx % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) M = fmaxf(M, sm_m[w * 16 + row]);
+        float Lsum = 0.0f, acc = 0.0f;
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+            const float mw = sm_m[w * 16 + row];
+            const float sc = (mw == -INFINITY) ? 0.0f : ex2_approx(mw - M);
+            Lsum += sm_l[w * 16 + row] * sc;
+            acc += sm_o[(w * 16 + row) * D + d] * sc;
         }
         const size_t prow = (group_row0 + row) * p.n_splits + split;
         p.o_part[prow * D + d] = (Lsum > 0.0f) ? acc * vscale / Lsum : 0.0f;

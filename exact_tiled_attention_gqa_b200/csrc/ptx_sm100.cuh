@@ -376,6 +376,14 @@ __device__ __forceinline__ void mma_f16_16816(float* c, const uint32_t* a, uint3
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
+// transpose an 8x8 matrix of 16-bit elements held one row pair per lane
+// (lane t: row t / 4, columns 2 (t % 4), 2 (t % 4) + 1) into the same layout
+__device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
+    uint32_t r;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(r) : "r"(x));
+    return r;
+}
+
 // two fp32 -> packed f16x2 (lo in bits 0-15), round to nearest even
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
     uint32_t r;
@@ -398,15 +406,18 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     return r;
 }
 
-// two int8 codes (bytes 0 and 1 of x) -> f16x2, exactly: with u = code + 128
-// (the code's bits with the sign bit flipped), the f16 with bits 0x6400 | u
-// is 1024 + u, and 1024 + u - 1152 = code.
-__device__ __forceinline__ uint32_t int8x2_to_f16x2(uint32_t x) {
-    const uint32_t biased = prmt(x ^ 0x8080u, 0x64646464u, 0x4140u);   // {0x64, u1, 0x64, u0}
+// two int8 codes in offset form (bytes 0 and 1 of u, u = code + 128, i.e. the
+// code's bits with the sign bit flipped) -> f16x2, exactly: the f16 with bits
+// 0x6400 | u is 1024 + u, and 1024 + u - 1152 = code.
+__device__ __forceinline__ uint32_t offset_u8x2_to_f16x2(uint32_t u) {
+    const uint32_t h = prmt(u, 0x64646464u, 0x4140u);   // {0x64, u1, 0x64, u0}
     uint32_t r;
-    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(biased), "r"(0x64806480u));   // 1152 = 0x6480 in f16
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(h), "r"(0x64806480u));   // 1152 = 0x6480 in f16
     return r;
 }
+
+// two int8 codes (bytes 0 and 1 of x) -> f16x2, exactly
+__device__ __forceinline__ uint32_t int8x2_to_f16x2(uint32_t x) { return offset_u8x2_to_f16x2(x ^ 0x8080u); }
 
 __device__ __forceinline__ float f16_bits_to_float(uint16_t h) {
     float f;
