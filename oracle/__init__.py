@@ -11,8 +11,14 @@ softmax(scale * Q K^T + mask) V with grouped-query heads (query head h reads
 KV head h // G), the bottom-right causal mask of the causal-alignment section
 of the SDPA / FlashAttention selection guide, and the natural-log LSE.
 
+For an 8-bit KV cache (``attention_decode_kv8``) the codes are first turned
+into fp64 element values by ``dequantize_kv8`` (FP8 E4M3 with one scale per KV
+head, or q8_0 int8 codes with an fp16 scale per 32 values; the decoders are in
+``attn_oracle.c``), and the same eager attention runs on them.
+
 Every function here is pinned by ``tests/test_oracle_pins.py`` against values
-the pages print (the numpy mask demonstration) and against closed forms.
+the pages print (the numpy mask demonstration), against closed forms, and (the
+8-bit decoders) against torch's and numpy's own decoders.
 """
 from __future__ import annotations
 
