@@ -25,6 +25,7 @@ workloads on this host's cores (rank 0 only).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import math
 import os
@@ -62,6 +63,8 @@ def parse():
                     help="profiling aid: time one call type only (the JSON line is then partial)")
     ap.add_argument("--decode-batch", type=int, default=None,
                     help="profiling aid: use the first N sequences of the decode batch")
+    ap.add_argument("--decode-cache", choices=["bf16", "e4m3", "q8_0"], default="bf16",
+                    help="with --only decode: the cache element format (8-bit caches use attn_decode_kv8)")
     ap.add_argument("--decode-group", type=int, default=None,
                     help="profiling aid: with --only decode, use the group-size sweep shape with this G")
     ap.add_argument("--no-sweeps", action="store_true",
@@ -168,18 +171,31 @@ def run_ours(args, rank, world, local_rank):
     if args.only == "decode":
         q_h, k_h, v_h = W.prefill_inputs(1, PREFILL.Hq, PREFILL.Hkv, 128, 128, PREFILL.D, seed=seed)
         q, k, v = q_h.to(dev), k_h.to(dev), v_h.to(dev)
-    dq, dk, dv, dsl = W.decode_inputs_for(dshape, seed=seed, device=dev)
+    if args.decode_cache != "bf16" and args.only != "decode":
+        raise SystemExit("--decode-cache applies to --only decode")
+    kv8 = args.decode_cache != "bf16"
+    if kv8:
+        dshape = dataclasses.replace(dshape, name=dshape.name + f", {args.decode_cache} KV cache")
+        dq, dk, dv, dks, dvs, dsl = W.decode_inputs_kv8(dshape.B, dshape.Hq, dshape.Hkv, dshape.Lmax, dshape.D,
+                                                        dshape.seqlen_lo, dshape.seqlen_hi, args.decode_cache,
+                                                        seed=seed, device=dev)
+        dq = dq[:, :, 0].contiguous()
+    else:
+        dq, dk, dv, dsl = W.decode_inputs_for(dshape, seed=seed, device=dev)
     if args.only is not None:
         print(json.dumps({"profiling_workload": dshape.name if args.only == "decode" else PREFILL.name}), flush=True)
     seqlens_host = dsl.cpu()
     p_flops = RL.prefill_flops(PREFILL.B, PREFILL.Hq, PREFILL.Lq, PREFILL.Lk, PREFILL.D, PREFILL.is_causal)
-    d_bytes = RL.decode_bytes(seqlens_host.tolist(), dshape.B, dshape.Hq, dshape.Hkv, dshape.D)
+    d_bytes = (RL.decode_kv8_bytes(seqlens_host.tolist(), dshape.B, dshape.Hq, dshape.Hkv, dshape.D,
+                                   args.decode_cache == "q8_0") if kv8 else
+               RL.decode_bytes(seqlens_host.tolist(), dshape.B, dshape.Hq, dshape.Hkv, dshape.D))
     p_out = torch.empty_like(q)
     p_lse = torch.empty((PREFILL.B, PREFILL.Hq, PREFILL.Lq), dtype=torch.float32, device=dev)
     d_out = torch.empty_like(dq)
     d_lse = torch.empty((dshape.B, dshape.Hq), dtype=torch.float32, device=dev)
-    ws = torch.empty(attn.decode_workspace_size(dshape.B, dshape.Hq, dshape.Hkv, dshape.Lmax, dshape.D),
-                     dtype=torch.uint8, device=dev)
+    ws_bytes = (attn.decode_kv8_workspace_size(dshape.B, dshape.Hq, dshape.Hkv, 1, dshape.Lmax, dshape.D) if kv8
+                else attn.decode_workspace_size(dshape.B, dshape.Hq, dshape.Hkv, dshape.Lmax, dshape.D))
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     do_pre = args.only in (None, "prefill")
@@ -190,7 +206,9 @@ def run_ours(args, rank, world, local_rank):
             attn.prefill(q, k, v, is_causal=True, out=p_out, lse=p_lse, stream=stream)
 
     def call_decode():
-        if do_dec:
+        if do_dec and kv8:
+            attn.decode_kv8(dq, dk, dv, dks, dvs, dsl, out=d_out, lse=d_lse, workspace=ws, stream=stream)
+        elif do_dec:
             attn.decode(dq, dk, dv, dsl, out=d_out, lse=d_lse, workspace=ws, stream=stream)
 
     def step():
