@@ -58,6 +58,8 @@ def parse():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip the oracle timing leg")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU seconds per oracle sample")
+    ap.add_argument("--ref-seconds", type=float, default=120.0,
+                    help="--impl reference: target CPU seconds for the whole run (warm-up + timed samples)")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--only", choices=["prefill", "decode"], default=None,
                     help="profiling aid: time one call type only (the JSON line is then partial)")
@@ -540,7 +542,7 @@ def run_reference(args, rank, world):
     q_h, k_h, v_h = W.prefill_inputs_for(PREFILL, seed=args.seed, device="cpu")
     cores = oracle.num_threads(0)
     f0, t0, _ = oracle_prefill_rate(q_h, k_h, v_h, 8)
-    budget = 120.0 / max(1, args.steps + args.warmup)          # whole run within a few minutes
+    budget = args.ref_seconds / max(1, args.steps + args.warmup)   # whole run within a few minutes
     n = int(max(8, min(PREFILL.Lq, 8 * budget / max(t0, 1e-3))))
     for _ in range(args.warmup):
         oracle_prefill_rate(q_h, k_h, v_h, 8)
