@@ -27,7 +27,8 @@ import torch
 from . import _native
 from ._native import AttnError
 
-__all__ = ["prefill", "decode", "decode_mq", "decode_paged", "decode_noalloc", "decode_kv8", "decode_workspace_size",
+__all__ = ["prefill", "decode", "decode_mq", "decode_paged", "decode_noalloc", "decode_kv8", "decode_kv8_paged",
+           "decode_workspace_size",
            "decode_mq_workspace_size", "decode_kv8_workspace_size", "device_error", "AttnError", "library_path"]
 
 
@@ -199,6 +200,60 @@ def decode_kv8(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, k_
                                            _ptr(seqlens), _ptr(out), _ptr(lse), B, Hq, Hkv, Lq, Lmax, D,
                                            float(scale), _ptr(workspace), workspace.numel(), _stream_handle(stream))
     _native.check(st, "attn_decode_kv8")
+    if squeeze:
+        out = out.squeeze(2) if out.dim() == 4 else out
+        lse = None if lse is None else (lse.squeeze(2) if lse.dim() == 3 else lse)
+    return out, lse
+
+
+def decode_kv8_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, k_scale: torch.Tensor,
+                     v_scale: torch.Tensor, block_table: torch.Tensor, seqlens: torch.Tensor, *,
+                     scale: Optional[float] = None, out: Optional[torch.Tensor] = None,
+                     lse: Optional[torch.Tensor] = None, want_lse: bool = True,
+                     workspace: Optional[torch.Tensor] = None, stream=None):
+    """Paged decode against an 8-bit cache.  q [B,Hq,Lq,D] (or [B,Hq,D]) bf16; code pools
+    [n_pages,Hkv,page_size,D] of torch.float8_e4m3fn (k_scale / v_scale float32 [Hkv]) or torch.int8
+    (k_scale / v_scale float16 [n_pages,Hkv,page_size,D/32]); block_table int32 [B,max_pages]; seqlens int32 [B]."""
+    squeeze = q.dim() == 3
+    if squeeze:
+        q = q.unsqueeze(2)
+    _check_tensor("q", q, torch.bfloat16, 4)
+    if k_pages.dtype == torch.float8_e4m3fn:
+        fmt, sdt, sdim = _native.ATTN_KV_E4M3, torch.float32, 1
+    elif k_pages.dtype == torch.int8:
+        fmt, sdt, sdim = _native.ATTN_KV_Q8_0, torch.float16, 4
+    else:
+        raise TypeError(f"k_pages must be torch.float8_e4m3fn or torch.int8, got {k_pages.dtype}")
+    _check_tensor("k_pages", k_pages, k_pages.dtype, 4)
+    _check_tensor("v_pages", v_pages, k_pages.dtype, 4)
+    _check_tensor("k_scale", k_scale, sdt, sdim)
+    _check_tensor("v_scale", v_scale, sdt, sdim)
+    _check_tensor("block_table", block_table, torch.int32, 2)
+    _check_tensor("seqlens", seqlens, torch.int32, 1)
+    B, Hq, Lq, D = q.shape
+    n_pages, Hkv, page_size = k_pages.shape[0], k_pages.shape[1], k_pages.shape[2]
+    max_pages = block_table.shape[1]
+    if (k_pages.shape[3] != D or v_pages.shape != k_pages.shape or block_table.shape[0] != B
+            or seqlens.shape[0] != B):
+        raise ValueError("shape mismatch between q, the page pools, block_table and seqlens")
+    want_scale = (Hkv,) if fmt == _native.ATTN_KV_E4M3 else (n_pages, Hkv, page_size, D // 32)
+    if tuple(k_scale.shape) != want_scale or tuple(v_scale.shape) != want_scale:
+        raise ValueError(f"k_scale / v_scale must have shape {want_scale}")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    need = int(_native.lib().attn_decode_kv8_paged_workspace_size(B, Hq, Hkv, Lq, page_size, max_pages, D))
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    with torch.cuda.device(q.device):
+        st = _native.lib().attn_decode_kv8_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(k_scale), _ptr(v_scale),
+                                                 fmt, _ptr(block_table), _ptr(seqlens), _ptr(out), _ptr(lse), B, Hq,
+                                                 Hkv, Lq, n_pages, page_size, max_pages, D, float(scale),
+                                                 _ptr(workspace), workspace.numel(), _stream_handle(stream))
+    _native.check(st, "attn_decode_kv8_paged")
     if squeeze:
         out = out.squeeze(2) if out.dim() == 4 else out
         lse = None if lse is None else (lse.squeeze(2) if lse.dim() == 3 else lse)

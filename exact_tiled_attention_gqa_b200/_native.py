@@ -41,6 +41,9 @@ SIGNATURES = {
     "attn_decode_kv8_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32]),
     "attn_decode_kv8": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32,
                                _f32, _vp, _sz, _vp]),
+    "attn_decode_kv8_paged_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32, _i32]),
+    "attn_decode_kv8_paged": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
+                                     _i32, _i32, _i32, _f32, _vp, _sz, _vp]),
     "attn_selftest_kv8_convert": (_i32, [_vp, _vp, _i32, _i32, _vp]),
     "attn_selftest_exp2": (_i32, [_vp, _vp, _i32, _vp]),
     "attn_status_string": (ctypes.c_char_p, [_i32]),

@@ -217,6 +217,12 @@ int launch_decode_split(const CUtensorMap& tk, const CUtensorMap& tv, const Deco
     return check_launch("attn_decode_split_kernel");
 }
 
+// Paged cache description (block_table == nullptr: the contiguous layout).
+struct PagedKV {
+    const int32_t* block_table = nullptr;
+    int page_size = 0, max_pages = 0, n_pages = 0;
+};
+
 template <int D, int KPW, int FMT>
 int launch_decode_kv8_split(const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& tks,
                             const CUtensorMap& tvs, const DecodeParams& prm, cudaStream_t stream) {
@@ -244,18 +250,21 @@ int launch_decode_kv8t(const CUtensorMap& tk, const CUtensorMap& tv, const CUten
 template <int D, int FMT>
 int launch_decode_kv8(const void* q, const void* kc, const void* vc, const void* k_scale, const void* v_scale,
                       const int32_t* seqlens, void* out, float* lse, int B, int Hq, int Hkv, int Lq, int Lmax,
-                      float scale, void* workspace, cudaStream_t stream) {
+                      float scale, void* workspace, cudaStream_t stream, PagedKV paged = PagedKV()) {
     const DecodeLayout lay = decode_layout(B, Hq, Hkv, Lmax, D, Lq, true);
     CUtensorMap tk, tv, tks, tvs;
     int st;
-    const uint64_t outer = static_cast<uint64_t>(B) * Hkv;
-    if ((st = encode_u8_3d(&tk, kc, D, static_cast<uint64_t>(Lmax), outer, D, kDecKT, "k_cache")) != ATTN_OK) return st;
-    if ((st = encode_u8_3d(&tv, vc, D, static_cast<uint64_t>(Lmax), outer, D, kDecKT, "v_cache")) != ATTN_OK) return st;
+    // the [outer, rows, D] view TMA reads 64-row boxes from (pages: [n_pages * Hkv, page_size, D])
+    const uint64_t view_rows = paged.block_table ? static_cast<uint64_t>(paged.page_size) : static_cast<uint64_t>(Lmax);
+    const uint64_t outer = paged.block_table ? static_cast<uint64_t>(paged.n_pages) * Hkv
+                                             : static_cast<uint64_t>(B) * Hkv;
+    if ((st = encode_u8_3d(&tk, kc, D, view_rows, outer, D, kDecKT, "k_cache")) != ATTN_OK) return st;
+    if ((st = encode_u8_3d(&tv, vc, D, view_rows, outer, D, kDecKT, "v_cache")) != ATTN_OK) return st;
     if (FMT == kKvFmtQ8_0) {
         const uint64_t per_row = D / 32;
-        if ((st = encode_u16_2d(&tks, k_scale, per_row * Lmax, outer, kDecKT * (D / 32), "k_scale")) != ATTN_OK)
+        if ((st = encode_u16_2d(&tks, k_scale, per_row * view_rows, outer, kDecKT * (D / 32), "k_scale")) != ATTN_OK)
             return st;
-        if ((st = encode_u16_2d(&tvs, v_scale, per_row * Lmax, outer, kDecKT * (D / 32), "v_scale")) != ATTN_OK)
+        if ((st = encode_u16_2d(&tvs, v_scale, per_row * view_rows, outer, kDecKT * (D / 32), "v_scale")) != ATTN_OK)
             return st;
     } else {
         tks = tk;   // unused
@@ -272,8 +281,10 @@ int launch_decode_kv8(const void* q, const void* kc, const void* vc, const void*
     prm.Lmax = Lmax;
     prm.G = Hq / Hkv;
     prm.Lq = Lq;
-    prm.block_table = nullptr;
-    prm.page_size = prm.max_pages = prm.n_pages = 0;
+    prm.block_table = paged.block_table;
+    prm.page_size = paged.page_size;
+    prm.max_pages = paged.max_pages;
+    prm.n_pages = paged.n_pages;
     prm.chunk = lay.chunk;
     prm.n_splits = lay.n_splits;
     prm.scale_log2 = scale * kLog2e;
@@ -296,11 +307,6 @@ int launch_decode_kv8(const void* q, const void* kc, const void* vc, const void*
     return check_launch("attn_decode_combine_kernel");
 }
 
-// Paged cache description (block_table == nullptr: the contiguous layout).
-struct PagedKV {
-    const int32_t* block_table = nullptr;
-    int page_size = 0, max_pages = 0, n_pages = 0;
-};
 
 template <int D>
 int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* seqlens, void* out, float* lse, int B,
@@ -650,10 +656,22 @@ extern "C" size_t attn_decode_kv8_workspace_size(int B, int Hq, int Hkv, int Lq,
     return decode_layout(B, Hq, Hkv, Lmax, D, Lq, true).total;
 }
 
-extern "C" int attn_decode_kv8(const void* q, const void* k_cache, const void* v_cache, const void* k_scale,
-                               const void* v_scale, int kv_format, const int32_t* seqlens, void* out, float* lse,
-                               int B, int Hq, int Hkv, int Lq, int Lmax, int D, float scale, void* workspace,
-                               size_t workspace_bytes, void* stream) {
+extern "C" size_t attn_decode_kv8_paged_workspace_size(int B, int Hq, int Hkv, int Lq, int page_size, int max_pages,
+                                                       int D) {
+    if (page_size < 64 || page_size % 64 != 0 || max_pages < 1 ||
+        static_cast<long long>(page_size) * max_pages > 0x7fffffffLL)
+        return 0;
+    return attn_decode_kv8_workspace_size(B, Hq, Hkv, Lq, page_size * max_pages, D);
+}
+
+namespace {
+// Checks and launch shared by the contiguous and the paged 8-bit entry points.
+// Lmax: the cache rows one sequence can have (paged: page_size * max_pages);
+// scale_rows: rows of one (b or page, KV head) slab of the q8_0 scale plane.
+int decode_kv8_checked(const void* q, const void* k_cache, const void* v_cache, const void* k_scale,
+                       const void* v_scale, int kv_format, const int32_t* seqlens, void* out, float* lse, int B,
+                       int Hq, int Hkv, int Lq, int Lmax, int scale_rows, int D, float scale, void* workspace,
+                       size_t workspace_bytes, void* stream, PagedKV paged) {
     int st = check_common(q, k_cache, v_cache, out, lse, B, Hq, Hkv, Lq, Lmax, D, scale, "Lq", "Lmax");
     if (st != ATTN_OK) return st;
     if (kv_format != ATTN_KV_E4M3 && kv_format != ATTN_KV_Q8_0)
@@ -669,7 +687,8 @@ extern "C" int attn_decode_kv8(const void* q, const void* k_cache, const void* v
     if (kv_format == ATTN_KV_Q8_0) {
         if (!aligned16(k_scale) || !aligned16(v_scale))
             return fail(ATTN_ERR_INVALID_ARG, "Q8_0 scale planes must be 16-byte aligned");
-        if (Lmax % 4 != 0) return fail(ATTN_ERR_INVALID_ARG, "Q8_0 caches need Lmax %% 4 == 0 (got %d)", Lmax);
+        if (scale_rows % 4 != 0)
+            return fail(ATTN_ERR_INVALID_ARG, "Q8_0 caches need Lmax %% 4 == 0 (got %d)", scale_rows);
     }
     if (D != 64 && D != 128) return fail(ATTN_ERR_UNSUPPORTED, "8-bit cache head dim D=%d (built: 64, 128)", D);
     if (static_cast<long long>(Hq / Hkv) * Lq > 64)
@@ -686,15 +705,47 @@ extern "C" int attn_decode_kv8(const void* q, const void* k_cache, const void* v
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (kv_format == ATTN_KV_E4M3)
         st = (D == 128) ? launch_decode_kv8<128, kKvFmtE4M3>(q, k_cache, v_cache, k_scale, v_scale, seqlens, out, lse,
-                                                              B, Hq, Hkv, Lq, Lmax, scale, workspace, s)
+                                                              B, Hq, Hkv, Lq, Lmax, scale, workspace, s, paged)
                         : launch_decode_kv8<64, kKvFmtE4M3>(q, k_cache, v_cache, k_scale, v_scale, seqlens, out, lse,
-                                                             B, Hq, Hkv, Lq, Lmax, scale, workspace, s);
+                                                             B, Hq, Hkv, Lq, Lmax, scale, workspace, s, paged);
     else
         st = (D == 128) ? launch_decode_kv8<128, kKvFmtQ8_0>(q, k_cache, v_cache, k_scale, v_scale, seqlens, out, lse,
-                                                              B, Hq, Hkv, Lq, Lmax, scale, workspace, s)
+                                                              B, Hq, Hkv, Lq, Lmax, scale, workspace, s, paged)
                         : launch_decode_kv8<64, kKvFmtQ8_0>(q, k_cache, v_cache, k_scale, v_scale, seqlens, out, lse,
-                                                             B, Hq, Hkv, Lq, Lmax, scale, workspace, s);
+                                                             B, Hq, Hkv, Lq, Lmax, scale, workspace, s, paged);
     return st == ATTN_OK ? ok() : st;
+}
+}  // namespace
+
+extern "C" int attn_decode_kv8(const void* q, const void* k_cache, const void* v_cache, const void* k_scale,
+                               const void* v_scale, int kv_format, const int32_t* seqlens, void* out, float* lse,
+                               int B, int Hq, int Hkv, int Lq, int Lmax, int D, float scale, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+    return decode_kv8_checked(q, k_cache, v_cache, k_scale, v_scale, kv_format, seqlens, out, lse, B, Hq, Hkv, Lq,
+                              Lmax, Lmax, D, scale, workspace, workspace_bytes, stream, PagedKV());
+}
+
+extern "C" int attn_decode_kv8_paged(const void* q, const void* k_pages, const void* v_pages, const void* k_scale,
+                                     const void* v_scale, int kv_format, const int32_t* block_table,
+                                     const int32_t* seqlens, void* out, float* lse, int B, int Hq, int Hkv, int Lq,
+                                     int n_pages, int page_size, int max_pages, int D, float scale, void* workspace,
+                                     size_t workspace_bytes, void* stream) {
+    if (page_size < 64 || page_size % 64 != 0)
+        return fail(ATTN_ERR_INVALID_ARG, "page_size=%d must be a positive multiple of 64", page_size);
+    if (n_pages < 1 || max_pages < 1) return fail(ATTN_ERR_INVALID_ARG, "n_pages and max_pages must be >= 1");
+    if (static_cast<long long>(page_size) * max_pages > 0x7fffffffLL ||
+        static_cast<long long>(n_pages) * Hkv > 0x7fffffffLL)
+        return fail(ATTN_ERR_UNSUPPORTED, "page pool too large");
+    if (B > 0 && !block_table) return fail(ATTN_ERR_INVALID_ARG, "null block_table");
+    if (reinterpret_cast<uintptr_t>(block_table) & 3u)
+        return fail(ATTN_ERR_INVALID_ARG, "block_table must be 4-byte aligned");
+    PagedKV pg;
+    pg.block_table = block_table;
+    pg.page_size = page_size;
+    pg.max_pages = max_pages;
+    pg.n_pages = n_pages;
+    return decode_kv8_checked(q, k_pages, v_pages, k_scale, v_scale, kv_format, seqlens, out, lse, B, Hq, Hkv, Lq,
+                              page_size * max_pages, page_size, D, scale, workspace, workspace_bytes, stream, pg);
 }
 
 namespace attn {

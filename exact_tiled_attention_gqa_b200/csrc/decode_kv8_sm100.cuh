@@ -57,6 +57,7 @@ constexpr int kKvFmtQ8_0 = 2;
 
 template <int D, int FMT>
 struct DecodeKv8Smem {
+    static constexpr int kBlk = D / 32;
     static constexpr int kTileBytes = kDecKT * D;                       // 64 rows of codes
     static constexpr int kScaleBytes = (FMT == kKvFmtQ8_0) ? kDecKT * (D / 32) * 2 : 0;
     static constexpr int kVOff = kTileBytes;
@@ -97,6 +98,63 @@ __device__ __forceinline__ uint32_t kv8_pair(uint32_t x) {
         return e4m3x2_to_f16x2(x);
     else
         return offset_u8x2_to_f16x2(x);
+}
+
+// TMA producer of both kernels (one thread): the 64-row tiles of cache rows
+// k_begin .. of (b, g) into the ring, codes and (q8_0) scales.  Contiguous
+// cache: tile of rows r .. r+63 is box (0, r, b * Hkv + g).  Paged cache: row r
+// lives in page block_table[b][r / page_size] at row r % page_size (page_size
+// a multiple of 64, so a tile never straddles pages): box (0, r % page_size,
+// page * Hkv + g).  A page outside the pool is flagged and replaced by page 0.
+template <typename L, int FMT>
+__device__ __forceinline__ void kv8_produce(const CUtensorMap* tm_k, const CUtensorMap* tm_v, const CUtensorMap* tm_ks,
+                                            const CUtensorMap* tm_vs, const DecodeParams& p, int b, int g,
+                                            int k_begin, int n_tiles, uint32_t ring, uint32_t bar0,
+                                            volatile int* abort_flag) {
+    constexpr int kBlk = L::kBlk;
+    auto bar_full = [&](int s) { return bar0 + 8u * s; };
+    auto bar_empty = [&](int s) { return bar0 + 8u * (L::kStages + s); };
+    tma_prefetch_desc(tm_k);
+    tma_prefetch_desc(tm_v);
+    if constexpr (FMT == kKvFmtQ8_0) {
+        tma_prefetch_desc(tm_ks);
+        tma_prefetch_desc(tm_vs);
+    }
+    int issued = 0;
+    for (int t = 0; t < n_tiles; ++t) {
+        const int s = t % L::kStages;
+        const uint32_t round = static_cast<uint32_t>(t / L::kStages);
+        const int key0 = k_begin + t * kDecKT;
+        int row = key0, outer = b * p.Hkv + g;
+        if (p.block_table != nullptr) {
+            int page = __ldg(p.block_table + static_cast<size_t>(b) * p.max_pages + key0 / p.page_size);
+            if (page < 0 || page >= p.n_pages) {   // the tile would read another tenant's rows
+                atomicOr(&g_attn_err, kDevErrPage);
+                page = 0;
+            }
+            row = key0 % p.page_size;
+            outer = page * p.Hkv + g;
+        }
+        if (!mbar_wait(bar_empty(s), (round & 1u) ^ 1u, abort_flag, &g_attn_err, kDevErrTimeout)) break;
+        mbar_arrive_expect_tx(bar_full(s), L::kStageTx);
+        const uint32_t dst = ring + s * L::kStageBytes;
+        tma_load_3d(dst, tm_k, bar_full(s), 0, row, outer);
+        tma_load_3d(dst + L::kVOff, tm_v, bar_full(s), 0, row, outer);
+        if constexpr (FMT == kKvFmtQ8_0) {
+            tma_load_2d(dst + L::kKsOff, tm_ks, bar_full(s), row * kBlk, outer);
+            tma_load_2d(dst + L::kVsOff, tm_vs, bar_full(s), row * kBlk, outer);
+        }
+        issued = t + 1;
+    }
+    if (issued < n_tiles) {
+        // unwinding after a timeout: let issued copies land first
+        for (int t = max(0, issued - L::kStages); t < issued; ++t) {
+            const uint64_t t0 = global_timer_ns();
+            while (!mbar_try_wait(bar_full(t % L::kStages), static_cast<uint32_t>(t / L::kStages) & 1u) &&
+                   global_timer_ns() - t0 < 100000000ull) {
+            }
+        }
+    }
 }
 
 // KPW = cache rows of each 64-row tile handled by one compute warp (16, 32 or 64).
@@ -140,40 +198,7 @@ __global__ void __maxnreg__(200)
 
     if (warp == 4) {
         // ================= TMA producer =================
-        if (lane == 0) {
-            tma_prefetch_desc(&tm_k);
-            tma_prefetch_desc(&tm_v);
-            if constexpr (FMT == kKvFmtQ8_0) {
-                tma_prefetch_desc(&tm_ks);
-                tma_prefetch_desc(&tm_vs);
-            }
-            const int outer = b * p.Hkv + g;
-            int issued = 0;
-            for (int t = 0; t < n_tiles; ++t) {
-                const int s = t % L::kStages;
-                const uint32_t round = static_cast<uint32_t>(t / L::kStages);
-                const int key0 = k_begin + t * kDecKT;
-                if (!mbar_wait(bar_empty(s), (round & 1u) ^ 1u, abort_flag, &g_attn_err, kDevErrTimeout)) break;
-                mbar_arrive_expect_tx(bar_full(s), L::kStageTx);
-                const uint32_t dst = ring + s * L::kStageBytes;
-                tma_load_3d(dst, &tm_k, bar_full(s), 0, key0, outer);
-                tma_load_3d(dst + L::kVOff, &tm_v, bar_full(s), 0, key0, outer);
-                if constexpr (FMT == kKvFmtQ8_0) {
-                    tma_load_2d(dst + L::kKsOff, &tm_ks, bar_full(s), key0 * kBlk, outer);
-                    tma_load_2d(dst + L::kVsOff, &tm_vs, bar_full(s), key0 * kBlk, outer);
-                }
-                issued = t + 1;
-            }
-            if (issued < n_tiles) {
-                // unwinding after a timeout: let issued copies land first
-                for (int t = max(0, issued - L::kStages); t < issued; ++t) {
-                    const uint64_t t0 = global_timer_ns();
-                    while (!mbar_try_wait(bar_full(t % L::kStages), static_cast<uint32_t>(t / L::kStages) & 1u) &&
-                           global_timer_ns() - t0 < 100000000ull) {
-                    }
-                }
-            }
-        }
+        if (lane == 0) kv8_produce<L, FMT>(&tm_k, &tm_v, &tm_ks, &tm_vs, p, b, g, k_begin, n_tiles, ring, bar0, abort_flag);
         __syncwarp();
         return;   // the producer takes no part in the merge below
     }
@@ -454,6 +479,7 @@ __global__ void __maxnreg__(200)
 //    row grp + 8 holds d + 1.
 template <int D, int FMT>
 struct DecodeKv8tSmem {
+    static constexpr int kBlk = D / 32;
     static constexpr int kTileBytes = kDecKT * D;
     static constexpr int kScaleBytes = (FMT == kKvFmtQ8_0) ? kDecKT * (D / 32) * 2 : 0;
     static constexpr int kVOff = kTileBytes;
@@ -515,39 +541,7 @@ __global__ void __launch_bounds__(kDecThreads, kv8t_min_blocks<NR>())
 
     if (warp == 4) {
         // ================= TMA producer =================
-        if (lane == 0) {
-            tma_prefetch_desc(&tm_k);
-            tma_prefetch_desc(&tm_v);
-            if constexpr (FMT == kKvFmtQ8_0) {
-                tma_prefetch_desc(&tm_ks);
-                tma_prefetch_desc(&tm_vs);
-            }
-            const int outer = b * p.Hkv + g;
-            int issued = 0;
-            for (int t = 0; t < n_tiles; ++t) {
-                const int s = t % L::kStages;
-                const uint32_t round = static_cast<uint32_t>(t / L::kStages);
-                const int key0 = k_begin + t * kDecKT;
-                if (!mbar_wait(bar_empty(s), (round & 1u) ^ 1u, abort_flag, &g_attn_err, kDevErrTimeout)) break;
-                mbar_arrive_expect_tx(bar_full(s), L::kStageTx);
-                const uint32_t dst = ring + s * L::kStageBytes;
-                tma_load_3d(dst, &tm_k, bar_full(s), 0, key0, outer);
-                tma_load_3d(dst + L::kVOff, &tm_v, bar_full(s), 0, key0, outer);
-                if constexpr (FMT == kKvFmtQ8_0) {
-                    tma_load_2d(dst + L::kKsOff, &tm_ks, bar_full(s), key0 * kBlk, outer);
-                    tma_load_2d(dst + L::kVsOff, &tm_vs, bar_full(s), key0 * kBlk, outer);
-                }
-                issued = t + 1;
-            }
-            if (issued < n_tiles) {
-                for (int t = max(0, issued - L::kStages); t < issued; ++t) {
-                    const uint64_t t0 = global_timer_ns();
-                    while (!mbar_try_wait(bar_full(t % L::kStages), static_cast<uint32_t>(t / L::kStages) & 1u) &&
-                           global_timer_ns() - t0 < 100000000ull) {
-                    }
-                }
-            }
-        }
+        if (lane == 0) kv8_produce<L, FMT>(&tm_k, &tm_v, &tm_ks, &tm_vs, p, b, g, k_begin, n_tiles, ring, bar0, abort_flag);
         __syncwarp();
         return;
     }

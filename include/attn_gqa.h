@@ -297,6 +297,23 @@ int attn_decode_kv8(const void* q, const void* k_cache, const void* v_cache, con
                     size_t workspace_bytes, void* stream);
 
 /*
+ * attn_decode_kv8_paged_workspace_size / attn_decode_kv8_paged -- attn_decode_kv8
+ * over a paged 8-bit cache: the page layout of attn_decode_paged (pools
+ * [n_pages, Hkv, page_size, D], block_table [B, max_pages], logical row r of
+ * sequence b in page block_table[b][r / page_size] at row r % page_size) with
+ * 8-bit codes.  ATTN_KV_Q8_0 scale pools are [n_pages, Hkv, page_size, D / 32]
+ * fp16, paged like the codes; ATTN_KV_E4M3 scales stay [Hkv] fp32.
+ *   page_size: a positive multiple of 64.  Other arguments, limits and
+ *   errors as attn_decode_kv8 and attn_decode_paged; block-table entries
+ *   outside [0, n_pages) set ATTN_DEVERR_PAGE and are never dereferenced.
+ */
+size_t attn_decode_kv8_paged_workspace_size(int B, int Hq, int Hkv, int Lq, int page_size, int max_pages, int D);
+int attn_decode_kv8_paged(const void* q, const void* k_pages, const void* v_pages, const void* k_scale,
+                          const void* v_scale, int kv_format, const int32_t* block_table, const int32_t* seqlens,
+                          void* out, float* lse, int B, int Hq, int Hkv, int Lq, int n_pages, int page_size,
+                          int max_pages, int D, float scale, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * attn_selftest_kv8_convert -- diagnostic: out[i] = the f16x2 (two f16 bit
  * patterns, code byte 0 in bits 0-15) that attn_decode_kv8 feeds its MMAs for
  * the two 8-bit codes in codes[i] (byte 0 in bits 0-7), for kv_format

@@ -184,3 +184,16 @@ def test_decode_kv8_empty_batch_and_workspace(lib):
     f = lib.attn_decode_kv8_workspace_size
     assert f(2, 8, 2, 1, 1000, 256) == 0 and f(2, 64, 1, 2, 1000, 128) == 0 and f(0, 8, 2, 1, 64, 128) == 0
     assert f(2, 8, 2, 1, 1000, 128) > 0 and f(2, 8, 2, 1, 1000, 128) % 256 == 0
+
+
+def test_decode_kv8_paged_rejects(lib):
+    f = lambda **kw: lib.attn_decode_kv8_paged(
+        *[kw.get(n, d) for n, d in (("q", A), ("k", A), ("v", A), ("ks", A), ("vs", A), ("fmt", 1), ("bt", A),
+                                    ("sl", A), ("out", A), ("lse", NULL), ("B", 2), ("Hq", 8), ("Hkv", 2), ("Lq", 1),
+                                    ("n_pages", 10), ("page_size", 64), ("max_pages", 4), ("D", 128),
+                                    ("scale", 0.1), ("ws", A), ("wsb", 1 << 30))], None)
+    assert f(page_size=32) == -1 and f(page_size=100) == -1 and f(n_pages=0) == -1 and f(bt=NULL) == -1
+    assert f(fmt=5) == -1 and f(D=256) == -2 and f(ws=NULL) == -3 and f(B=0) == 0
+    w = lib.attn_decode_kv8_paged_workspace_size
+    assert w(2, 8, 2, 1, 64, 4, 128) == lib.attn_decode_kv8_workspace_size(2, 8, 2, 1, 256, 128)
+    assert w(2, 8, 2, 1, 100, 4, 128) == 0

@@ -140,3 +140,73 @@ def test_kv8_full_size_sampled(oracle_mod, fmt):
                                                        v[b:b + 1, g:g + 1, :n].cpu(), _oracle_fmt(oracle_mod, fmt),
                                                        ksl, vsl, np.array([n]), shape.scale)
         assert_close(out[b:b + 1, h:h + 1], lse[b:b + 1, h:h + 1], ref_o, ref_l, f"{shape.name} b{b} h{h}")
+
+
+def _paged_kv8(fmt, seqlens, Hq, Hkv, Lq, D, page_size, seed, spare_pages=2):
+    """Contiguous 8-bit inputs, then the same rows scattered into shuffled pages
+    (unused pages and rows hold NaN codes / NaN scales)."""
+    B = len(seqlens)
+    Lmax = max(64, -(-max(seqlens) // page_size) * page_size)
+    q, k, v, ks, vs, _ = W.decode_inputs_kv8(B, Hq, Hkv, Lmax, D, 1, Lmax, fmt, seed=seed, Lq=Lq)
+    pages_per = [max(1, -(-n // page_size)) for n in seqlens]
+    max_pages = max(pages_per) + 1
+    n_pages = sum(pages_per) + spare_pages
+    order = torch.randperm(n_pages, generator=torch.Generator().manual_seed(seed))
+    kp = torch.empty((n_pages, Hkv, page_size, D), dtype=k.dtype)
+    vp = torch.empty_like(kp)
+    kp.view(torch.uint8).fill_(0x7F if fmt == W.KV_E4M3 else 0x80)
+    vp.view(torch.uint8).fill_(0x7F if fmt == W.KV_E4M3 else 0x80)
+    if fmt == W.KV_Q8_0:
+        ksp = torch.full((n_pages, Hkv, page_size, D // 32), float("nan"), dtype=torch.float16)
+        vsp = torch.full_like(ksp, float("nan"))
+    else:
+        ksp, vsp = ks, vs
+    table = torch.full((B, max_pages), -1, dtype=torch.int32)
+    nxt = 0
+    for b, n in enumerate(seqlens):
+        for i in range(pages_per[b]):
+            pg = int(order[nxt]); nxt += 1
+            table[b, i] = pg
+            rows = min(page_size, n - i * page_size)
+            if rows <= 0:
+                continue
+            sl = slice(i * page_size, i * page_size + rows)
+            kp[pg, :, :rows] = k[b, :, sl]
+            vp[pg, :, :rows] = v[b, :, sl]
+            if fmt == W.KV_Q8_0:
+                ksp[pg, :, :rows] = ks[b, :, sl]
+                vsp[pg, :, :rows] = vs[b, :, sl]
+    return q, k, v, ks, vs, kp, vp, ksp, vsp, table
+
+
+@pytest.mark.parametrize("fmt", [W.KV_E4M3, W.KV_Q8_0])
+@pytest.mark.parametrize("page_size", [64, 128, 256])
+@pytest.mark.parametrize("G,Lq,D", [(4, 1, 128), (8, 2, 64), (1, 1, 128), (32, 1, 128)])
+def test_kv8_paged_against_oracle(oracle_mod, fmt, page_size, G, Lq, D):
+    from exact_tiled_attention_gqa_b200 import decode_kv8_paged
+    Hkv = 2
+    seqlens = [1000, 1, 0, 257, 64, 2100]
+    q, k, v, ks, vs, kp, vp, ksp, vsp, table = _paged_kv8(fmt, seqlens, G * Hkv, Hkv, Lq, D, page_size,
+                                                           seed=page_size + G + Lq + D)
+    sl = torch.tensor(seqlens, dtype=torch.int32)
+    scale = 1 / math.sqrt(D)
+    out, lse = decode_kv8_paged(q.cuda(), kp.cuda(), vp.cuda(), ksp.cuda(), vsp.cuda(), table.cuda(), sl.cuda(),
+                                scale=scale)
+    torch.cuda.synchronize()
+    assert device_error(reset=True) == 0
+    ref_o, ref_l = oracle_mod.attention_decode_kv8(q, k, v, _oracle_fmt(oracle_mod, fmt), ks, vs, sl, scale)
+    assert_close(out, lse, ref_o, ref_l, f"paged {fmt} ps{page_size} G{G} Lq{Lq} D{D}")
+    # the same rows read contiguously give the same answer
+    mo, ml = decode_kv8(q.cuda(), k.cuda(), v.cuda(), ks.cuda(), vs.cuda(), sl.cuda(), scale=scale)
+    torch.cuda.synchronize()
+    assert (mo.float() - out.float()).abs().max().item() <= 2e-2
+
+
+def test_kv8_paged_bad_page_is_flagged():
+    from exact_tiled_attention_gqa_b200 import decode_kv8_paged
+    q, k, v, ks, vs, kp, vp, ksp, vsp, table = _paged_kv8(W.KV_E4M3, [300], 4, 1, 1, 128, 128, seed=1)
+    table[0, 1] = 10_000
+    decode_kv8_paged(q.cuda(), kp.cuda(), vp.cuda(), ksp.cuda(), vsp.cuda(), table.cuda(),
+                     torch.tensor([300], dtype=torch.int32).cuda())
+    torch.cuda.synchronize()
+    assert device_error(reset=True) & 0x4
