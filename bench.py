@@ -364,24 +364,28 @@ _L2_FLUSH = None
 
 
 def _time_calls(fn, stream, n_warm=2, n=10, flush=False):
-    """Mean device time of fn() over n calls (CUDA events on `stream`).  With
+    """Mean device time of fn() over n calls (CUDA events on `stream` around each
+    call).  All n calls are enqueued before one synchronisation, so the host's
+    launch work overlaps the device's and no event pair holds an idle gap.  With
     flush, a 256 MB write (twice the L2) precedes every call, outside its events."""
     global _L2_FLUSH
     for _ in range(n_warm):
         fn()
     if flush and _L2_FLUSH is None:
         _L2_FLUSH = torch.empty(256 << 20, dtype=torch.uint8, device=torch.cuda.current_device())
-    total = 0.0
+    evs = []
+    torch.cuda.synchronize()
     for _ in range(n):
         if flush:
-            _L2_FLUSH.fill_(1)
+            with torch.cuda.stream(stream):
+                _L2_FLUSH.fill_(1)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         fn()
         e1.record(stream)
-        e1.synchronize()
-        total += e0.elapsed_time(e1)
-    return total / n
+        evs.append((e0, e1))
+    torch.cuda.synchronize()
+    return sum(e0.elapsed_time(e1) for e0, e1 in evs) / n
 
 
 def run_sweeps(attn, dev, stream, seed, max_over_ranks):
