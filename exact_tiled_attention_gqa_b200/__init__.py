@@ -27,9 +27,9 @@ import torch
 from . import _native
 from ._native import AttnError
 
-__all__ = ["prefill", "decode", "decode_mq", "decode_paged", "decode_noalloc", "decode_kv8", "decode_kv8_paged",
-           "decode_workspace_size",
-           "decode_mq_workspace_size", "decode_kv8_workspace_size", "device_error", "AttnError", "library_path"]
+__all__ = ["prefill", "prefill_host", "decode", "decode_mq", "decode_paged", "decode_noalloc", "decode_kv8",
+           "decode_kv8_paged", "prefill_host_scratch_size", "decode_workspace_size", "decode_mq_workspace_size",
+           "decode_kv8_workspace_size", "device_error", "AttnError", "library_path"]
 
 
 def library_path() -> str:
@@ -83,6 +83,45 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: Optiona
         st = _native.lib().attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Lq, Lk, D,
                                         float(scale), int(bool(is_causal)), _stream_handle(stream))
     _native.check(st, "attn_prefill")
+    return out, lse
+
+
+def prefill_host_scratch_size(B: int, Hq: int, Hkv: int, Lq: int, Lk: int, D: int) -> int:
+    return int(_native.lib().attn_prefill_host_scratch_size(B, Hq, Hkv, Lq, Lk, D))
+
+
+def prefill_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: Optional[float] = None,
+                 is_causal: bool = True, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                 want_lse: bool = True, scratch: Optional[torch.Tensor] = None, device=None, stream=None):
+    """attn_prefill on CPU tensors (pinned for overlap): copies in, kernels and copies out are
+    pipelined by the library.  Results are in `out` / `lse` once `stream` (default: the current
+    stream of `device`) has passed the call, e.g. after stream.synchronize()."""
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not isinstance(t, torch.Tensor) or t.is_cuda or t.dtype != torch.bfloat16 or t.dim() != 4 \
+                or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous 4-d bf16 CPU tensor")
+    B, Hq, Lq, D = q.shape
+    Hkv, Lk = k.shape[1], k.shape[2]
+    if k.shape[0] != B or k.shape[3] != D or v.shape != k.shape:
+        raise ValueError("shape mismatch between q, k, v")
+    device = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=True)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, pin_memory=True)
+    for name, t in (("out", out), ("lse", lse)):
+        if t is not None and (t.is_cuda or not t.is_contiguous()):
+            raise ValueError(f"{name} must be a contiguous CPU tensor")
+    need = prefill_host_scratch_size(B, Hq, Hkv, Lq, Lk, D)
+    if scratch is None:
+        scratch = torch.empty(max(need, 1), dtype=torch.uint8, device=device)
+    with torch.cuda.device(device):
+        st = _native.lib().attn_prefill_host(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Lq, Lk,
+                                             D, float(scale), int(bool(is_causal)), _ptr(scratch), scratch.numel(),
+                                             _stream_handle(stream))
+    _native.check(st, "attn_prefill_host")
     return out, lse
 
 

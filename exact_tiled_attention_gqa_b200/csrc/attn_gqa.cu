@@ -414,6 +414,165 @@ extern "C" int attn_prefill(const void* q, const void* k, const void* v, void* o
     return st == ATTN_OK ? ok() : st;
 }
 
+namespace attn {
+namespace {
+// ---- attn_prefill_host: host buffers in, host buffers out, copies overlapped ----
+//
+// Work is cut into units of (sequence b, hc consecutive KV heads); the slabs of
+// q, k, v, out and lse that a unit touches are contiguous in [B, H, L, D], so a
+// unit is three host-to-device copies, one prefill launch (B = 1, Hq = hc G,
+// Hkv = hc) and two device-to-host copies.  Units alternate between two device
+// slots; copies in run on one library stream, copies out on another, the
+// kernels on the caller's stream, ordered by events per slot, so unit u's
+// copy in, unit u-1's kernel and unit u-2's copy out can run at once.
+struct HostPipe {
+    bool ready = false;
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t start = nullptr, in_done[2] = {}, comp_done[2] = {}, out_done[2] = {};
+};
+HostPipe g_pipes[64];
+std::mutex g_pipe_mu;
+
+int host_pipe(HostPipe** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= 64) return fail(ATTN_ERR_CUDA, "device ordinal %d out of range", dev);
+    HostPipe& p = g_pipes[dev];
+    if (!p.ready) {
+        const unsigned ef = cudaEventDisableTiming;
+        e = cudaStreamCreateWithFlags(&p.h2d, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&p.d2h, cudaStreamNonBlocking);
+        if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p.start, ef);
+        for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
+            e = cudaEventCreateWithFlags(&p.in_done[i], ef);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p.comp_done[i], ef);
+            if (e == cudaSuccess) e = cudaEventCreateWithFlags(&p.out_done[i], ef);
+        }
+        if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "creating the copy streams: %s", cudaGetErrorString(e));
+        p.ready = true;
+    }
+    *out = &p;
+    return ATTN_OK;
+}
+
+struct HostUnits {
+    int hc = 1, n_units = 0;
+    size_t q_bytes = 0, kv_bytes = 0, lse_bytes = 0;   // one unit's slabs
+    size_t q_off = 0, k_off = 0, v_off = 0, o_off = 0, l_off = 0, slot_bytes = 0;
+};
+
+HostUnits host_units(int B, int Hq, int Hkv, int Lq, int Lk, int D) {
+    HostUnits u;
+    const int G = Hq / Hkv;
+    const int NQ = (D == 256) ? 1 : 2;
+    const long long n_mblk = (Lq + static_cast<long long>(NQ) * (kBM / G) - 1) / (static_cast<long long>(NQ) * (kBM / G));
+    // the smallest run of KV heads (a divisor of Hkv) whose kernel still fills a wave of CTAs:
+    // small units keep the pipeline's fill and drain short
+    u.hc = Hkv;
+    for (int hc = 1; hc <= Hkv; ++hc)
+        if (Hkv % hc == 0 && hc * n_mblk >= 148) {
+            u.hc = hc;
+            break;
+        }
+    u.n_units = B * (Hkv / u.hc);
+    u.q_bytes = static_cast<size_t>(u.hc) * G * Lq * D * 2;
+    u.kv_bytes = static_cast<size_t>(u.hc) * Lk * D * 2;
+    u.lse_bytes = static_cast<size_t>(u.hc) * G * Lq * 4;
+    u.q_off = 0;
+    u.k_off = align256(u.q_off + u.q_bytes);
+    u.v_off = align256(u.k_off + u.kv_bytes);
+    u.o_off = align256(u.v_off + u.kv_bytes);
+    u.l_off = align256(u.o_off + u.q_bytes);
+    u.slot_bytes = align256(u.l_off + u.lse_bytes);
+    return u;
+}
+}  // namespace
+}  // namespace attn
+
+extern "C" size_t attn_prefill_host_scratch_size(int B, int Hq, int Hkv, int Lq, int Lk, int D) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Lq < 1 || Lk < 0 || (D != 64 && D != 128 && D != 256) ||
+        Hq / Hkv > kBM)
+        return 0;
+    return 2 * host_units(B, Hq, Hkv, Lq, Lk, D).slot_bytes;
+}
+
+extern "C" int attn_prefill_host(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
+                                 int Hkv, int Lq, int Lk, int D, float scale, int is_causal, void* scratch,
+                                 size_t scratch_bytes, void* stream) {
+    int st = check_common(q, k, v, out, lse, B, Hq, Hkv, Lq, Lk, D, scale, "Lq", "Lk");
+    if (st != ATTN_OK) return st;
+    if (Hq / Hkv > kBM) return fail(ATTN_ERR_UNSUPPORTED, "group size G=%d > %d", Hq / Hkv, kBM);
+    if (static_cast<long long>(B) * Hq > 0x7fffffffLL || static_cast<long long>(B) * Hkv > 0x7fffffffLL)
+        return fail(ATTN_ERR_UNSUPPORTED, "B*H too large");
+    if (B == 0 || Lq == 0) return ok();
+    const HostUnits u = host_units(B, Hq, Hkv, Lq, Lk, D);
+    if (!scratch || scratch_bytes < 2 * u.slot_bytes)
+        return fail(ATTN_ERR_WORKSPACE, "prefill host scratch needs %zu bytes, got %zu", 2 * u.slot_bytes,
+                    scratch ? scratch_bytes : static_cast<size_t>(0));
+    if (reinterpret_cast<uintptr_t>(scratch) & 255u)
+        return fail(ATTN_ERR_INVALID_ARG, "scratch must be 256-byte aligned");
+    std::lock_guard<std::mutex> lock(g_pipe_mu);
+    HostPipe* hp = nullptr;
+    if ((st = host_pipe(&hp)) != ATTN_OK) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const int G = Hq / Hkv, chunks = Hkv / u.hc;
+    auto cuda_ok = [](cudaError_t e, const char* what) {
+        return e == cudaSuccess ? ATTN_OK : fail(ATTN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    };
+    // the copies must not overtake work the caller queued before (it may still use the scratch)
+    if ((st = cuda_ok(cudaEventRecord(hp->start, cs), "cudaEventRecord")) != ATTN_OK) return st;
+    if ((st = cuda_ok(cudaStreamWaitEvent(hp->h2d, hp->start, 0), "cudaStreamWaitEvent")) != ATTN_OK) return st;
+    for (int n = 0; n < u.n_units; ++n) {
+        const int slot = n & 1, b = n / chunks, c = n % chunks;
+        uint8_t* base = static_cast<uint8_t*>(scratch) + slot * u.slot_bytes;
+        const size_t qrow = (static_cast<size_t>(b) * Hq + static_cast<size_t>(c) * u.hc * G) * Lq;   // first q row
+        const size_t krow = (static_cast<size_t>(b) * Hkv + static_cast<size_t>(c) * u.hc) * Lk;     // first k row
+        const uint8_t* qh = static_cast<const uint8_t*>(q) + qrow * D * 2;
+        const uint8_t* kh = static_cast<const uint8_t*>(k) + krow * D * 2;
+        const uint8_t* vh = static_cast<const uint8_t*>(v) + krow * D * 2;
+        uint8_t* oh = static_cast<uint8_t*>(out) + qrow * D * 2;
+        float* lh = lse ? lse + qrow : nullptr;
+        // in: after the kernel that last read this slot's inputs
+        st = cuda_ok(cudaStreamWaitEvent(hp->h2d, hp->comp_done[slot], 0), "cudaStreamWaitEvent");
+        if (st == ATTN_OK) st = cuda_ok(cudaMemcpyAsync(base + u.q_off, qh, u.q_bytes, cudaMemcpyHostToDevice, hp->h2d), "copy q in");
+        if (st == ATTN_OK && u.kv_bytes) {
+            st = cuda_ok(cudaMemcpyAsync(base + u.k_off, kh, u.kv_bytes, cudaMemcpyHostToDevice, hp->h2d), "copy k in");
+            if (st == ATTN_OK)
+                st = cuda_ok(cudaMemcpyAsync(base + u.v_off, vh, u.kv_bytes, cudaMemcpyHostToDevice, hp->h2d), "copy v in");
+        }
+        if (st == ATTN_OK) st = cuda_ok(cudaEventRecord(hp->in_done[slot], hp->h2d), "cudaEventRecord");
+        // kernel: after its inputs are in and the slot's previous outputs are out
+        if (st == ATTN_OK) st = cuda_ok(cudaStreamWaitEvent(cs, hp->in_done[slot], 0), "cudaStreamWaitEvent");
+        if (st == ATTN_OK) st = cuda_ok(cudaStreamWaitEvent(cs, hp->out_done[slot], 0), "cudaStreamWaitEvent");
+        if (st != ATTN_OK) return st;
+        void* od = base + u.o_off;
+        float* ld = lh ? reinterpret_cast<float*>(base + u.l_off) : nullptr;
+        if (Lk == 0) {
+            fill_no_key_rows_kernel<<<1184, 256, 0, cs>>>(static_cast<__nv_bfloat16*>(od), ld,
+                                                          static_cast<size_t>(u.hc) * G * Lq, D);
+            st = check_launch("fill_no_key_rows_kernel");
+        } else {
+            const void *qd = base + u.q_off, *kd = base + u.k_off, *vd = base + u.v_off;
+            st = (D == 256)   ? launch_prefill<256>(qd, kd, vd, od, ld, 1, u.hc * G, u.hc, Lq, Lk, scale, is_causal, cs)
+                 : (D == 128) ? launch_prefill<128>(qd, kd, vd, od, ld, 1, u.hc * G, u.hc, Lq, Lk, scale, is_causal, cs)
+                              : launch_prefill<64>(qd, kd, vd, od, ld, 1, u.hc * G, u.hc, Lq, Lk, scale, is_causal, cs);
+        }
+        if (st != ATTN_OK) return st;
+        if ((st = cuda_ok(cudaEventRecord(hp->comp_done[slot], cs), "cudaEventRecord")) != ATTN_OK) return st;
+        // out: after the kernel
+        st = cuda_ok(cudaStreamWaitEvent(hp->d2h, hp->comp_done[slot], 0), "cudaStreamWaitEvent");
+        if (st == ATTN_OK) st = cuda_ok(cudaMemcpyAsync(oh, od, u.q_bytes, cudaMemcpyDeviceToHost, hp->d2h), "copy out");
+        if (st == ATTN_OK && lh) st = cuda_ok(cudaMemcpyAsync(lh, ld, u.lse_bytes, cudaMemcpyDeviceToHost, hp->d2h), "copy lse out");
+        if (st == ATTN_OK) st = cuda_ok(cudaEventRecord(hp->out_done[slot], hp->d2h), "cudaEventRecord");
+        if (st != ATTN_OK) return st;
+    }
+    // the caller's stream passes this call only once every result is in host memory
+    for (int slot = 0; slot < 2; ++slot)
+        if ((st = cuda_ok(cudaStreamWaitEvent(cs, hp->out_done[slot], 0), "cudaStreamWaitEvent")) != ATTN_OK) return st;
+    return ok();
+}
+
 extern "C" size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, int D) {
     if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Lmax < 1 || (D != 64 && D != 128 && D != 256) || Hq / Hkv > 128)
         return 0;

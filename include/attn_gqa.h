@@ -90,6 +90,40 @@ int attn_prefill(const void* q, const void* k, const void* v, void* out, float* 
                  void* stream);
 
 /*
+ * attn_prefill_host_scratch_size / attn_prefill_host -- attn_prefill with
+ * q, k, v, out and lse in HOST memory: the call copies the inputs to the device,
+ * computes, and copies the results back, overlapping the three.
+ *
+ * Same operation, arguments, layouts and limits as attn_prefill, except:
+ *   q, k, v, out, lse  host pointers (page-locked memory lets the copies run
+ *                      asynchronously and overlap; pageable memory works but
+ *                      each copy then waits for the host); lse may be NULL
+ *   scratch            device memory of attn_prefill_host_scratch_size(...)
+ *                      bytes, 256-byte aligned, owned by the caller (two
+ *                      slots of one work unit each; see below)
+ *
+ * The work is cut into units of one sequence and a run of KV heads (the
+ * smallest divisor of Hkv whose kernel still fills a wave of CTAs); for each
+ * unit the q, k, v slabs are copied in on a library-owned stream, the prefill
+ * kernel runs on `stream`, and the out and lse slabs are copied back on a second
+ * library-owned stream, with events ordering the two device slots, so one
+ * unit's copy in, the previous unit's kernel and the one before's copy out run
+ * at once.  The library creates its two copy streams and a few events once per
+ * device and keeps them for the life of the process.
+ *
+ * Completion: when `stream` has passed the work this call enqueued, every
+ * result is in host memory.  The host buffers must stay valid until then.
+ * Calls from several host threads on one device are serialised while they
+ * enqueue.  Errors: as attn_prefill, plus ATTN_ERR_WORKSPACE for a missing or
+ * small scratch and ATTN_ERR_INVALID_ARG for a misaligned one; a CUDA failure
+ * part-way returns ATTN_ERR_CUDA with the units before it enqueued.
+ */
+size_t attn_prefill_host_scratch_size(int B, int Hq, int Hkv, int Lq, int Lk, int D);
+int attn_prefill_host(const void* q, const void* k, const void* v, void* out, float* lse,
+                      int B, int Hq, int Hkv, int Lq, int Lk, int D, float scale, int is_causal,
+                      void* scratch, size_t scratch_bytes, void* stream);
+
+/*
  * attn_decode_workspace_size -- bytes of scratch attn_decode needs for these
  * sizes (split-KV partial outputs and their log-sum-exps).  Depends only on
  * the arguments.  Returns 0 for sizes attn_decode would reject.

@@ -197,3 +197,14 @@ def test_decode_kv8_paged_rejects(lib):
     w = lib.attn_decode_kv8_paged_workspace_size
     assert w(2, 8, 2, 1, 64, 4, 128) == lib.attn_decode_kv8_workspace_size(2, 8, 2, 1, 256, 128)
     assert w(2, 8, 2, 1, 100, 4, 128) == 0
+
+
+def test_prefill_host_rejects(lib):
+    f = lambda **kw: lib.attn_prefill_host(
+        *[kw.get(n, d) for n, d in (("q", A), ("k", A), ("v", A), ("out", A), ("lse", NULL), ("B", 2), ("Hq", 8),
+                                    ("Hkv", 2), ("Lq", 64), ("Lk", 64), ("D", 128), ("scale", 0.1), ("causal", 1),
+                                    ("ws", A), ("wsb", 1 << 30))], None)
+    assert f(ws=NULL) == -3 and f(wsb=1024) == -3 and f(ws=ctypes.c_void_p(0x10010)) == -1
+    assert f(D=96) == -2 and f(Hq=7) == -1 and f(B=0) == 0
+    s = lib.attn_prefill_host_scratch_size
+    assert s(2, 8, 2, 64, 64, 128) > 0 and s(2, 8, 2, 64, 64, 96) == 0 and s(0, 8, 2, 64, 64, 128) == 0
