@@ -73,6 +73,7 @@
 
 #include "ptx_sm100.cuh"
 #include "device_error.cuh"
+#include "ring_order.cuh"
 
 namespace attn {
 
@@ -119,34 +120,6 @@ struct PrefillSmem {
     static_assert(kAlloc <= 232448, "dynamic shared memory per CTA");
 };
 
-// Ring order of the K/V entries.  NQ = 2: K_0 V_0 K_1 V_1 ...  NQ = 1:
-// K_0 K_1 V_0 K_2 V_1 K_3 V_2 ... V_{n-1}, each tile as kItemsPerTile entries.
-// Position (in tiles) of K_j and V_j, and the inverse map.
-template <int NQ>
-__device__ __forceinline__ int ring_pos_k(int j) { return NQ == 2 ? 2 * j : (j == 0 ? 0 : 2 * j - 1); }
-template <int NQ>
-__device__ __forceinline__ int ring_pos_v(int j, int n_kt) {
-    return NQ == 2 ? 2 * j + 1 : (j + 1 < n_kt ? 2 * j + 2 : 2 * n_kt - 1);
-}
-template <int NQ>
-__device__ __forceinline__ void ring_tile(int pos, int n_kt, bool& is_v, int& j) {
-    if (NQ == 2) {
-        is_v = pos & 1;
-        j = pos >> 1;
-    } else if (pos == 0) {
-        is_v = false;
-        j = 0;
-    } else if (pos == 2 * n_kt - 1) {
-        is_v = true;
-        j = n_kt - 1;
-    } else if (pos & 1) {
-        is_v = false;
-        j = (pos + 1) >> 1;
-    } else {
-        is_v = true;
-        j = (pos - 2) >> 1;
-    }
-}
 
 struct PrefillParams {
     void* out;          // [B,Hq,Lq,D] bf16
