@@ -1,5 +1,7 @@
 // decode_tc_sm100.cuh -- split-KV decode on the tcgen05 tensor cores, for KV
-// heads with many query rows (G x Lq > 16).
+// heads with many query rows (G x Lq > 16), and for every group size at
+// D = 256 (a 256-wide O does not fit the mma.sync kernel's registers; there
+// Q, the two slots and 384 TMEM columns make it one CTA per SM).
 //
 // Same computation, split and partial format as attn_decode_split_kernel
 // (decode_sm100.cuh): a CTA owns `chunk` cache rows of one (b, KV head) and
