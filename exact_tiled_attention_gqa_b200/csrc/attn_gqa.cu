@@ -158,6 +158,8 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
     prm.G = G;
     prm.P = P;
     prm.n_mblk = (Lq + NQ * P - 1) / (NQ * P);
+    // longest-first across groups when all of K and V fit in half the L2 (126 MB)
+    prm.mblk_major = (static_cast<double>(B) * Hkv * Lk * D * 2 * 2 <= 63e6) ? 1 : 0;
     prm.is_causal = is_causal ? 1 : 0;
     prm.scale_log2 = scale * kLog2e;
     const long long grid = static_cast<long long>(B) * Hkv * prm.n_mblk;

@@ -127,6 +127,7 @@ struct PrefillParams {
     int B, Hq, Hkv, Lq, Lk;
     int G, P;           // group size, positions per Q tile (P = 128 / G)
     int n_mblk;         // ceil(Lq / (NQ P))
+    int mblk_major;     // CTA order: 0 group-major, 1 position-block-major (see the kernel)
     int is_causal;
     float scale_log2;   // scale * log2(e)
 };
@@ -149,11 +150,16 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
-    // ---- work unit: one (b, KV head) group after another, so CTAs running at
-    // the same time share that group's K/V in L2; within a group the heaviest
-    // (latest) position blocks come first ----
-    const int mblk = p.n_mblk - 1 - static_cast<int>(blockIdx.x % static_cast<unsigned>(p.n_mblk));
-    const int bh = static_cast<int>(blockIdx.x / static_cast<unsigned>(p.n_mblk));
+    // ---- work unit.  Group-major: one (b, KV head) group after another, so CTAs
+    // running at the same time share that group's K/V in L2; within a group the
+    // heaviest (latest) position blocks come first.  Position-block-major (when
+    // all of K/V fits in L2 anyway): the heaviest blocks of every group first,
+    // the longest-first order that keeps a causal grid's tail short. ----
+    const unsigned n_bh = static_cast<unsigned>(p.B * p.Hkv);
+    const int mblk = p.mblk_major ? p.n_mblk - 1 - static_cast<int>(blockIdx.x / n_bh)
+                                  : p.n_mblk - 1 - static_cast<int>(blockIdx.x % static_cast<unsigned>(p.n_mblk));
+    const int bh = p.mblk_major ? static_cast<int>(blockIdx.x % n_bh)
+                                : static_cast<int>(blockIdx.x / static_cast<unsigned>(p.n_mblk));
     const int b = bh / p.Hkv;
     const int g = bh % p.Hkv;
     const int P = p.P;
