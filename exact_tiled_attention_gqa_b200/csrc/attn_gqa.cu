@@ -169,22 +169,20 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
     return check_launch("attn_prefill_sm100_kernel");
 }
 
-// Cache rows per decode split: the largest power of two in [min_chunk, 4096]
-// that still gives about four waves of CTAs on a 148-SM part.
-// The tcgen05 split kernel (more than 16 query rows per KV head) keeps its
-// pipeline short per CTA, so it wants long splits: measured on B200 at
-// 131072 cached rows, G = 64 ran 1.8x faster with 2048-row splits than with
-// 256-row ones.
-#ifndef ATTN_TC_MIN_CHUNK
-#define ATTN_TC_MIN_CHUNK 2048
-#endif
+// Cache rows per decode split, a power of two in [256, 4096].
+//  - mma.sync split kernel: the largest that still gives about four waves of
+//    CTAs on a 148-SM part (1184 CTAs).
+//  - tcgen05 kernel: the largest (down to 512) that still gives one CTA per SM.
+//    Its CTAs carry more setup and each split adds a partial for the combine
+//    to merge, so long splits win: measured on B200 at 131072 cached rows,
+//    G = 64 took 0.148 / 0.122 / 0.106 ms with 1024 / 2048 / 4096-row splits.
 // D = 256 always takes the tcgen05 kernel: a 256-wide O per row does not fit
 // the mma.sync kernel's registers.
 bool decode_uses_tc(int D, int rows_per_group) { return D == 256 || rows_per_group > 16; }
 
 int decode_chunk(int B, int Hkv, int Lmax, bool tc_path) {
-    const long long target = 148LL * 2 * 4;
-    const int min_chunk = tc_path ? ATTN_TC_MIN_CHUNK : 256;
+    const long long target = tc_path ? 148LL : 148LL * 2 * 4;
+    const int min_chunk = tc_path ? 512 : 256;
     int chunk = 4096;
     while (chunk > min_chunk && static_cast<long long>(B) * Hkv * ((Lmax + chunk - 1) / chunk) < target) chunk >>= 1;
     return chunk;

@@ -387,6 +387,9 @@ __global__ void __maxnreg__(200)
 }
 
 // One warp per query row: out = sum_s 2^(lse_s - lse) O_s,  lse = log2 sum_s 2^lse_s.
+// The 32 lanes read the splits' LSEs together (one split each); each lane then
+// sums its D / 32 columns over the splits, the loads unrolled so that several
+// are in flight (a row with 64-256 splits is otherwise one dependent load per split).
 template <int D>
 __global__ void __launch_bounds__(128)
     attn_decode_combine_kernel(const DecodeParams p, __nv_bfloat16* out, float* lse) {
@@ -400,17 +403,34 @@ __global__ void __launch_bounds__(128)
     const float* op = p.o_part + static_cast<size_t>(row) * p.n_splits * D;
     constexpr int kPer = D / 32;
     float M = -INFINITY;
-    for (int s = 0; s < n_valid; ++s) M = fmaxf(M, lp[s]);
+    for (int s = lane; s < n_valid; s += 32) M = fmaxf(M, lp[s]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float acc[kPer];
 #pragma unroll
     for (int i = 0; i < kPer; ++i) acc[i] = 0.0f;
     float Lsum = 0.0f;
-    for (int s = 0; s < n_valid; ++s) {
-        const float w = (lp[s] == -INFINITY) ? 0.0f : ex2_approx(lp[s] - M);
-        Lsum += w;
+    for (int s0 = 0; s0 < n_valid; s0 += 32) {
+        const int s = s0 + lane;
+        const float ls = (s < n_valid) ? lp[s] : -INFINITY;
+        const float wl = (ls == -INFINITY) ? 0.0f : ex2_approx(ls - M);   // this lane's split weight
+        Lsum += wl;
+        const int cnt = min(32, n_valid - s0);
+        const float* ob = op + static_cast<size_t>(s0) * D + lane * kPer;
+#pragma unroll 8
+        for (int i = 0; i < cnt; ++i) {
+            const float w = __shfl_sync(0xffffffffu, wl, i);
+            const float* src = ob + static_cast<size_t>(i) * D;
 #pragma unroll
-        for (int i = 0; i < kPer; ++i) acc[i] += w * op[static_cast<size_t>(s) * D + lane * kPer + i];
+            for (int c = 0; c < kPer; c += 2) {
+                const float2 v = *reinterpret_cast<const float2*>(src + c);
+                acc[c] = fmaf(w, v.x, acc[c]);
+                acc[c + 1] = fmaf(w, v.y, acc[c + 1]);
+            }
+        }
     }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, o);
     const float inv = (Lsum > 0.0f) ? 1.0f / Lsum : 0.0f;
     __nv_bfloat16* o = out + static_cast<size_t>(row) * D + lane * kPer;
 #pragma unroll
