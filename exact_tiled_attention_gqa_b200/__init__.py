@@ -27,7 +27,7 @@ import torch
 from . import _native
 from ._native import AttnError
 
-__all__ = ["prefill", "prefill_host", "decode", "decode_mq", "decode_paged", "decode_noalloc", "decode_kv8",
+__all__ = ["prefill", "prefill_host", "decode", "decode_partial", "decode_merge", "decode_mq", "decode_paged", "decode_noalloc", "decode_kv8",
            "decode_kv8_paged", "prefill_host_scratch_size", "decode_workspace_size", "decode_mq_workspace_size",
            "decode_kv8_workspace_size", "device_error", "AttnError", "library_path"]
 
@@ -155,6 +155,54 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, seqlen
                                        B, Hq, Hkv, Lmax, D, float(scale), _ptr(workspace), workspace.numel(),
                                        _stream_handle(stream))
     _native.check(st, "attn_decode")
+    return out, lse
+
+
+def decode_partial(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, seqlens: torch.Tensor, *,
+                   scale: Optional[float] = None, workspace: Optional[torch.Tensor] = None, stream=None):
+    """decode over the cache rows this device holds, results unrounded for decode_merge:
+    (o_part fp32 [B,Hq,D], lse_part fp32 [B,Hq], natural log, -inf where a sequence has no rows here)."""
+    _check_tensor("q", q, torch.bfloat16, 3)
+    _check_tensor("k_cache", k_cache, torch.bfloat16, 4)
+    _check_tensor("v_cache", v_cache, torch.bfloat16, 4)
+    _check_tensor("seqlens", seqlens, torch.int32, 1)
+    B, Hq, D = q.shape
+    Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
+    if k_cache.shape[0] != B or k_cache.shape[3] != D or v_cache.shape != k_cache.shape or seqlens.shape[0] != B:
+        raise ValueError("shape mismatch between q, the caches and seqlens")
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    o_part = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
+    lse_part = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+    need = decode_workspace_size(B, Hq, Hkv, Lmax, D)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    with torch.cuda.device(q.device):
+        st = _native.lib().attn_decode_partial(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(o_part),
+                                               _ptr(lse_part), B, Hq, Hkv, Lmax, D, float(scale), _ptr(workspace),
+                                               workspace.numel(), _stream_handle(stream))
+    _native.check(st, "attn_decode_partial")
+    return o_part, lse_part
+
+
+def decode_merge(o_parts: torch.Tensor, lse_parts: torch.Tensor, *, out: Optional[torch.Tensor] = None,
+                 lse: Optional[torch.Tensor] = None, want_lse: bool = True, stream=None):
+    """Merge partial decode results over disjoint cache rows: o_parts fp32 [n, ..., D], lse_parts fp32 [n, ...]
+    (natural log) -> (out bf16 [..., D], lse fp32 [...])."""
+    _check_tensor("o_parts", o_parts, torch.float32, o_parts.dim())
+    _check_tensor("lse_parts", lse_parts, torch.float32, lse_parts.dim())
+    n, D = o_parts.shape[0], o_parts.shape[-1]
+    if tuple(lse_parts.shape) != tuple(o_parts.shape[:-1]) or o_parts.dim() < 3:
+        raise ValueError("o_parts must be [n, ..., D] and lse_parts [n, ...]")
+    rows = lse_parts[0].numel()
+    if out is None:
+        out = torch.empty(o_parts.shape[1:], dtype=torch.bfloat16, device=o_parts.device)
+    if lse is None and want_lse:
+        lse = torch.empty(lse_parts.shape[1:], dtype=torch.float32, device=o_parts.device)
+    with torch.cuda.device(o_parts.device):
+        st = _native.lib().attn_decode_merge(_ptr(o_parts), _ptr(lse_parts), n, rows, D, _ptr(out), _ptr(lse),
+                                             _stream_handle(stream))
+    _native.check(st, "attn_decode_merge")
     return out, lse
 
 

@@ -303,7 +303,7 @@ int launch_decode_kv8(const void* q, const void* kc, const void* vc, const void*
         st = launch_decode_kv8_split<D, 64, FMT>(tk, tv, tks, tvs, prm, stream);
     if (st != ATTN_OK) return st;
     const int n_rows = B * Hq * Lq;
-    attn_decode_combine_kernel<D><<<(n_rows + 3) / 4, 128, 0, stream>>>(prm, static_cast<__nv_bfloat16*>(out), lse);
+    attn_decode_combine_kernel<D><<<(n_rows + 3) / 4, 128, 0, stream>>>(prm, out, lse);
     return check_launch("attn_decode_combine_kernel");
 }
 
@@ -311,7 +311,7 @@ int launch_decode_kv8(const void* q, const void* kc, const void* vc, const void*
 template <int D>
 int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* seqlens, void* out, float* lse, int B,
                   int Hq, int Hkv, int Lmax, float scale, void* workspace, cudaStream_t stream, int Lq = 1,
-                  PagedKV paged = PagedKV()) {
+                  PagedKV paged = PagedKV(), bool f32_out = false) {
     const DecodeLayout lay = decode_layout(B, Hq, Hkv, Lmax, D, Lq);
     CUtensorMap tk, tv;
     int st;
@@ -364,7 +364,10 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
         st = launch_decode_split<D, 64>(tk, tv, prm, stream);
     if (st != ATTN_OK) return st;
     const int rows = B * Hq * Lq;
-    attn_decode_combine_kernel<D><<<(rows + 3) / 4, 128, 0, stream>>>(prm, static_cast<__nv_bfloat16*>(out), lse);
+    if (f32_out)
+        attn_decode_combine_kernel<D, true><<<(rows + 3) / 4, 128, 0, stream>>>(prm, out, lse);
+    else
+        attn_decode_combine_kernel<D><<<(rows + 3) / 4, 128, 0, stream>>>(prm, out, lse);
     return check_launch("attn_decode_combine_kernel");
 }
 
@@ -580,9 +583,10 @@ extern "C" size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, i
     return decode_layout(B, Hq, Hkv, Lmax, D).total;
 }
 
-extern "C" int attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens, void* out,
-                           float* lse, int B, int Hq, int Hkv, int Lmax, int D, float scale, void* workspace,
-                           size_t workspace_bytes, void* stream) {
+namespace {
+int decode_checked(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens, void* out,
+                   float* lse, int B, int Hq, int Hkv, int Lmax, int D, float scale, void* workspace,
+                   size_t workspace_bytes, void* stream, bool f32_out) {
     int st = check_common(q, k_cache, v_cache, out, lse, B, Hq, Hkv, Lmax, Lmax, D, scale, "Lmax", "Lmax");
     if (st != ATTN_OK) return st;
     if (!seqlens && B > 0) return fail(ATTN_ERR_INVALID_ARG, "null seqlens");
@@ -598,9 +602,51 @@ extern "C" int attn_decode(const void* q, const void* k_cache, const void* v_cac
     if (reinterpret_cast<uintptr_t>(workspace) & 255u)
         return fail(ATTN_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    st = (D == 256)   ? launch_decode<256>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s)
-         : (D == 128) ? launch_decode<128>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s)
-                      : launch_decode<64>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s);
+    const PagedKV none;
+    st = (D == 256)   ? launch_decode<256>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s,
+                                           1, none, f32_out)
+         : (D == 128) ? launch_decode<128>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s,
+                                           1, none, f32_out)
+                      : launch_decode<64>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s,
+                                          1, none, f32_out);
+    return st == ATTN_OK ? ok() : st;
+}
+}  // namespace
+
+extern "C" int attn_decode(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens, void* out,
+                           float* lse, int B, int Hq, int Hkv, int Lmax, int D, float scale, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+    return decode_checked(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, D, scale, workspace,
+                          workspace_bytes, stream, false);
+}
+
+extern "C" int attn_decode_partial(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,
+                                   float* o_part, float* lse_part, int B, int Hq, int Hkv, int Lmax, int D, float scale,
+                                   void* workspace, size_t workspace_bytes, void* stream) {
+    if (B > 0 && !lse_part) return fail(ATTN_ERR_INVALID_ARG, "null lse_part");
+    return decode_checked(q, k_cache, v_cache, seqlens, o_part, lse_part, B, Hq, Hkv, Lmax, D, scale, workspace,
+                          workspace_bytes, stream, true);
+}
+
+extern "C" int attn_decode_merge(const float* o_parts, const float* lse_parts, int n_parts, int rows, int D,
+                                 void* out, float* lse, void* stream) {
+    if (n_parts < 1 || rows < 0) return fail(ATTN_ERR_INVALID_ARG, "n_parts must be >= 1 and rows >= 0");
+    if (D != 64 && D != 128 && D != 256) return fail(ATTN_ERR_UNSUPPORTED, "head dim D=%d (built: 64, 128, 256)", D);
+    if (rows == 0) return ok();
+    if (!o_parts || !lse_parts || !out) return fail(ATTN_ERR_INVALID_ARG, "null o_parts, lse_parts or out");
+    if (!aligned16(o_parts) || !aligned16(out) || (reinterpret_cast<uintptr_t>(lse_parts) & 3u) ||
+        (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+        return fail(ATTN_ERR_INVALID_ARG, "o_parts and out must be 16-byte aligned, lse arrays 4-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const unsigned grid = static_cast<unsigned>((rows + 3) / 4);
+    auto* o = static_cast<__nv_bfloat16*>(out);
+    if (D == 256)
+        attn_decode_merge_kernel<256><<<grid, 128, 0, s>>>(o_parts, lse_parts, n_parts, rows, o, lse);
+    else if (D == 128)
+        attn_decode_merge_kernel<128><<<grid, 128, 0, s>>>(o_parts, lse_parts, n_parts, rows, o, lse);
+    else
+        attn_decode_merge_kernel<64><<<grid, 128, 0, s>>>(o_parts, lse_parts, n_parts, rows, o, lse);
+    const int st = check_launch("attn_decode_merge_kernel");
     return st == ATTN_OK ? ok() : st;
 }
 

@@ -390,9 +390,10 @@ __global__ void __maxnreg__(200)
 // The 32 lanes read the splits' LSEs together (one split each); each lane then
 // sums its D / 32 columns over the splits, the loads unrolled so that several
 // are in flight (a row with 64-256 splits is otherwise one dependent load per split).
-template <int D>
+// F32: out is fp32 [rows, D] instead of bf16 (a partial result that is merged later).
+template <int D, bool F32 = false>
 __global__ void __launch_bounds__(128)
-    attn_decode_combine_kernel(const DecodeParams p, __nv_bfloat16* out, float* lse) {
+    attn_decode_combine_kernel(const DecodeParams p, void* out_ptr, float* lse) {
     const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= p.B * p.Hq * p.Lq) return;
@@ -432,13 +433,67 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, o);
     const float inv = (Lsum > 0.0f) ? 1.0f / Lsum : 0.0f;
-    __nv_bfloat16* o = out + static_cast<size_t>(row) * D + lane * kPer;
+    if constexpr (F32) {
+        float* o = static_cast<float*>(out_ptr) + static_cast<size_t>(row) * D + lane * kPer;
 #pragma unroll
-    for (int i = 0; i < kPer; i += 2) {
-        const uint32_t v2 = pack_bf16x2(acc[i] * inv, acc[i + 1] * inv);
-        *reinterpret_cast<uint32_t*>(o + i) = v2;
+        for (int i = 0; i < kPer; i += 2) *reinterpret_cast<float2*>(o + i) = make_float2(acc[i] * inv, acc[i + 1] * inv);
+    } else {
+        __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out_ptr) + static_cast<size_t>(row) * D + lane * kPer;
+#pragma unroll
+        for (int i = 0; i < kPer; i += 2) {
+            const uint32_t v2 = pack_bf16x2(acc[i] * inv, acc[i + 1] * inv);
+            *reinterpret_cast<uint32_t*>(o + i) = v2;
+        }
     }
     if (lse != nullptr && lane == 0) lse[row] = (Lsum > 0.0f) ? (M + __log2f(Lsum)) * kLn2 : -INFINITY;
+}
+
+// Merge of decode results over disjoint sets of cache rows (KV parallelism: each
+// set held by one GPU, the NVIDIA attention page, "Parameter four: parallelism"):
+// out[r] = sum_p exp(lse_p[r] - lse[r]) O_p[r],  lse[r] = ln sum_p exp(lse_p[r]).
+// o_parts [n_parts][rows][D] fp32 (each normalised over its own rows), lse_parts
+// [n_parts][rows] natural log (-inf: no rows).  One warp per row, as the combine.
+template <int D>
+__global__ void __launch_bounds__(128)
+    attn_decode_merge_kernel(const float* o_parts, const float* lse_parts, int n_parts, int rows,
+                             __nv_bfloat16* out, float* lse) {
+    const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    constexpr int kPer = D / 32;
+    float M = -INFINITY;
+    for (int q = lane; q < n_parts; q += 32) M = fmaxf(M, lse_parts[static_cast<size_t>(q) * rows + row]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float acc[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) acc[i] = 0.0f;
+    float Lsum = 0.0f;
+    for (int q0 = 0; q0 < n_parts; q0 += 32) {
+        const int q = q0 + lane;
+        const float ls = (q < n_parts) ? lse_parts[static_cast<size_t>(q) * rows + row] : -INFINITY;
+        const float wl = (ls == -INFINITY) ? 0.0f : ex2_approx((ls - M) * kLog2e);
+        Lsum += wl;
+        const int cnt = min(32, n_parts - q0);
+#pragma unroll 4
+        for (int i = 0; i < cnt; ++i) {
+            const float w = __shfl_sync(0xffffffffu, wl, i);
+            const float* src = o_parts + (static_cast<size_t>(q0 + i) * rows + row) * D + lane * kPer;
+#pragma unroll
+            for (int c = 0; c < kPer; c += 2) {
+                const float2 v = *reinterpret_cast<const float2*>(src + c);
+                acc[c] = fmaf(w, v.x, acc[c]);
+                acc[c + 1] = fmaf(w, v.y, acc[c + 1]);
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, o);
+    const float inv = (Lsum > 0.0f) ? 1.0f / Lsum : 0.0f;
+    __nv_bfloat16* o = out + static_cast<size_t>(row) * D + lane * kPer;
+#pragma unroll
+    for (int i = 0; i < kPer; i += 2) *reinterpret_cast<uint32_t*>(o + i) = pack_bf16x2(acc[i] * inv, acc[i + 1] * inv);
+    if (lse != nullptr && lane == 0) lse[row] = (Lsum > 0.0f) ? M + __logf(Lsum) : -INFINITY;
 }
 
 }  // namespace attn

@@ -166,6 +166,37 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, const i
                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * attn_decode_partial / attn_decode_merge -- decode split across devices by
+ * cache rows (the KV parallelism of the NVIDIA attention page, "Parameter
+ * four: parallelism"): each device holds a disjoint set of every sequence's
+ * cached rows, computes attention over its own rows with attn_decode_partial,
+ * the partial results are exchanged (an all-gather), and attn_decode_merge
+ * combines them into exactly the attention over all rows.
+ *
+ * attn_decode_partial: attn_decode (same arguments, layouts, limits, workspace
+ * from attn_decode_workspace_size and errors) with its results left unrounded
+ * for the merge:
+ *   o_part    [B, Hq, D] fp32, written: O over this caller's rows
+ *   lse_part  [B, Hq]    fp32, written: natural-log LSE over those rows (-inf
+ *             when a sequence has none here); must not be NULL
+ *
+ * attn_decode_merge:
+ *   o_parts   [n_parts, rows, D] fp32, read (rows = B * Hq for decode)
+ *   lse_parts [n_parts, rows] fp32, read
+ *   out       [rows, D] bf16, written: sum_p exp(lse_p - lse) o_p
+ *   lse       [rows] fp32 or NULL, written: ln sum_p exp(lse_p)
+ *   n_parts >= 1; D 64, 128 or 256; o_parts and out 16-byte aligned.
+ * A row with no rows in any part gets O = 0 and LSE = -inf.  Errors:
+ * ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED (D), ATTN_ERR_CUDA.  rows == 0
+ * returns ATTN_OK.
+ */
+int attn_decode_partial(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,
+                        float* o_part, float* lse_part, int B, int Hq, int Hkv, int Lmax, int D, float scale,
+                        void* workspace, size_t workspace_bytes, void* stream);
+int attn_decode_merge(const float* o_parts, const float* lse_parts, int n_parts, int rows, int D,
+                      void* out, float* lse, void* stream);
+
+/*
  * attn_decode_mq_workspace_size -- bytes of scratch attn_decode_mq needs for
  * these sizes.  Depends only on the arguments; 0 for sizes it would reject.
  */

@@ -208,3 +208,14 @@ def test_prefill_host_rejects(lib):
     assert f(D=96) == -2 and f(Hq=7) == -1 and f(B=0) == 0
     s = lib.attn_prefill_host_scratch_size
     assert s(2, 8, 2, 64, 64, 128) > 0 and s(2, 8, 2, 64, 64, 96) == 0 and s(0, 8, 2, 64, 64, 128) == 0
+
+
+def test_decode_partial_and_merge_reject(lib):
+    m = lambda **kw: lib.attn_decode_merge(*[kw.get(n, d) for n, d in (("o", A), ("l", A), ("n", 2), ("rows", 8),
+                                                                        ("D", 128), ("out", A), ("lse", NULL))], None)
+    assert m(n=0) == -1 and m(rows=-1) == -1 and m(D=96) == -2 and m(rows=0) == 0 and m(o=NULL) == -1
+    assert m(o=ctypes.c_void_p(0x10008)) == -1
+    p = lambda **kw: lib.attn_decode_partial(*[kw.get(n, d) for n, d in (
+        ("q", A), ("k", A), ("v", A), ("sl", A), ("o", A), ("l", A), ("B", 2), ("Hq", 8), ("Hkv", 2), ("Lmax", 64),
+        ("D", 128), ("scale", 0.1), ("ws", A), ("wsb", 1 << 30))], None)
+    assert p(l=NULL) == -1 and p(D=96) == -2 and p(ws=NULL) == -3 and p(B=0) == 0

@@ -114,3 +114,27 @@ def test_qwen_decode_full_size_sampled(oracle_mod):
 @pytest.mark.parametrize("G", W.GROUP_SWEEP)
 def test_group_sweep_full_size_sampled(oracle_mod, G):
     _sampled_check(oracle_mod, W.group_sweep_decode(G), seed=G, n_pairs=6, fill_nan=False)
+
+
+@pytest.mark.parametrize("n_parts,D", [(2, 128), (3, 64), (4, 256), (1, 128)])
+def test_partial_and_merge_equal_full_decode(oracle_mod, n_parts, D):
+    """KV parallelism on one GPU: the cache split by rows into n_parts shards, each
+    decoded with decode_partial, merged with decode_merge, equals the whole decode."""
+    from exact_tiled_attention_gqa_b200 import decode_merge, decode_partial
+    from exact_tiled_attention_gqa_b200.multigpu import kv_shard_rows, shard_seqlens
+    seqlens = [5000, 4097, 1, 0, 2500, 700]
+    Lmax = 5000
+    q, k, v, sl = _inputs(len(seqlens), 16, 2, Lmax, D, seqlens, seed=n_parts * 10 + D)
+    qd, kd, vd, sld = q.cuda(), k.cuda(), v.cuda(), sl.cuda()
+    os_, ls_ = [], []
+    for r in range(n_parts):
+        rows = kv_shard_rows(Lmax, r, n_parts)
+        o, l = decode_partial(qd, kd[:, :, rows.start:rows.stop].contiguous(), vd[:, :, rows.start:rows.stop].contiguous(),
+                              shard_seqlens(sld, rows), scale=1 / math.sqrt(D))
+        os_.append(o)
+        ls_.append(l)
+    out, lse = decode_merge(torch.stack(os_), torch.stack(ls_))
+    torch.cuda.synchronize()
+    assert device_error(reset=True) == 0
+    ref_o, ref_l = oracle_mod.attention_decode(q, k, v, sl, 1 / math.sqrt(D))
+    assert_close(out, lse, ref_o, ref_l, f"kv-parallel x{n_parts} D{D}")
