@@ -393,7 +393,7 @@ def run_sweeps(attn, dev, stream, seed, max_over_ranks):
     (Hq=64, D=128, batch 8, 131072 keys, G = 1 .. 64)."""
     peaks = RL.measured_peaks()
     out = {"prefill": [], "decode_group_sweep": []}
-    for shape in (W.QWEN_PREFILL_4K, W.CHUNKED_16K, W.CHUNKED_32K, W.HD256_PREFILL):
+    for shape in (W.QWEN_PREFILL_4K, W.CHUNKED_16K, W.CHUNKED_32K, W.HD256_PREFILL, W.HD64_PREFILL):
         q, k, v = (t.to(dev) for t in W.prefill_inputs_for(shape, seed=seed))
         o = torch.empty_like(q)
         l = torch.empty((shape.B, shape.Hq, shape.Lq), dtype=torch.float32, device=dev)

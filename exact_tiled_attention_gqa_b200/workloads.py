@@ -85,6 +85,9 @@ QWEN_DECODE_E4M3 = DecodeShape("Qwen3-8B decode B64 seqlen U[1024,32768], E4M3 K
                                1024, 32768)
 QWEN_DECODE_Q8_0 = DecodeShape("Qwen3-8B decode B64 seqlen U[1024,32768], q8_0 KV cache", 64, 32, 8, 32768, 128,
                                1024, 32768)
+# Head dim 64: the NVIDIA page ("Parameter two: head dimension") has it paying for a
+# 128-wide tile, while the softmax cost does not shrink with D.
+HD64_PREFILL = PrefillShape("head-dim-64 causal prefill B4 Hq32 Hkv8 L8192 D64", 4, 32, 8, 8192, 8192, 64)
 # Head dim 256, the other width the NVIDIA attention page recommends ("Parameter
 # two: head dimension"), at group size 8.
 HD256_PREFILL = PrefillShape("head-dim-256 causal prefill B2 Hq16 Hkv2 L8192 D256", 2, 16, 2, 8192, 8192, 256)

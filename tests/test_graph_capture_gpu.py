@@ -1,0 +1,58 @@
+"""The device-buffer calls can be captured into a CUDA graph and replayed (the
+inner loop of a serving step): after one ordinary call on the device (which sets
+each kernel's shared-memory limit), prefill, decode and 8-bit decode are captured
+with fixed shapes and buffers, replayed with new inputs copied into those
+buffers, and must equal ordinary calls bit for bit."""
+import pytest
+import torch
+
+import exact_tiled_attention_gqa_b200 as attn
+from exact_tiled_attention_gqa_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    attn.device_error(reset=True)
+    yield
+    assert attn.device_error(reset=True) == 0
+
+
+def test_capture_and_replay_step():
+    dev = torch.device("cuda")
+    q, k, v = (t.to(dev) for t in W.prefill_inputs(2, 8, 2, 600, 600, 128, seed=1))
+    dq, dk, dv, dsl = W.decode_inputs(4, 32, 8, 3000, 128, 100, 3000, seed=2, device=dev)
+    q8, k8, v8, ks8, vs8, sl8 = (t.to(dev) for t in W.decode_inputs_kv8(4, 32, 8, 3000, 128, 100, 3000, W.KV_E4M3,
+                                                                         seed=3))
+    p_out, p_lse = torch.empty_like(q), torch.empty(2, 8, 600, device=dev)
+    d_out, d_lse = torch.empty_like(dq), torch.empty(4, 32, device=dev)
+    k_out, k_lse = torch.empty_like(q8), torch.empty(4, 32, 1, device=dev)
+    ws = torch.empty(attn.decode_workspace_size(4, 32, 8, 3000, 128), dtype=torch.uint8, device=dev)
+    ws8 = torch.empty(attn.decode_kv8_workspace_size(4, 32, 8, 1, 3000, 128), dtype=torch.uint8, device=dev)
+
+    def step(stream=None):
+        attn.prefill(q, k, v, out=p_out, lse=p_lse, stream=stream)
+        attn.decode(dq, dk, dv, dsl, out=d_out, lse=d_lse, workspace=ws, stream=stream)
+        attn.decode_kv8(q8, k8, v8, ks8, vs8, sl8, out=k_out, lse=k_lse, workspace=ws8, stream=stream)
+
+    step()                      # first calls: per-kernel setup outside the capture
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        step(stream=s)
+    # new inputs in the captured buffers, then replay
+    q.copy_(torch.randn_like(q, dtype=torch.float32).to(torch.bfloat16))
+    dq.copy_(torch.randn_like(dq, dtype=torch.float32).to(torch.bfloat16))
+    q8.copy_(torch.randn_like(q8, dtype=torch.float32).to(torch.bfloat16))
+    g.replay()
+    torch.cuda.synchronize()
+    got = [t.clone() for t in (p_out, p_lse, d_out, d_lse, k_out, k_lse)]
+    step()
+    torch.cuda.synchronize()
+    want = (p_out, p_lse, d_out, d_lse, k_out, k_lse)
+    assert all(torch.equal(a, b) for a, b in zip(got, want))
+    del g
