@@ -454,7 +454,7 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
         const float sl2 = p.scale_log2;
 
         float m_run = -INFINITY;   // running max used for the exponentials (log2 domain)
-        float l_run = 0.0f;        // running sum of P as rounded to bf16 (normalises O)
+        float l_run = 0.0f;        // running sum normalising O (see the exponentials below)
         float l_exact = 0.0f;      // running sum of the unrounded exponentials (for the LSE)
         bool ok = true;
         for (int j = 0; j < n_kt; ++j) {
@@ -536,7 +536,7 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
             const float m_sub = (m_run == -INFINITY) ? 0.0f : m_run;
             const uint64_t sl2x2 = f2_pack(sl2, sl2);
             const uint64_t negm2 = f2_pack(-m_sub, -m_sub);
-            uint64_t acc_r[2] = {0ull, 0ull}, acc_e[2] = {0ull, 0ull};
+            uint64_t acc_e[2] = {0ull, 0ull};
             auto exp_half = [&](auto masked_tag, int h) {
                 constexpr bool kMasked = decltype(masked_tag)::value;
                 uint32_t pk[32];
@@ -555,11 +555,7 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
                     float e0, e1;
                     f2_unpack(e, e0, e1);
                     pk[i] = pack_bf16x2(e0, e1);
-                    // O is normalised by the sum of P as the MMA sees it (bf16), so
-                    // the rounding of a dominant weight cancels in O / l; the LSE
-                    // takes the unrounded sum
                     acc_e[i & 1] = f2_add(acc_e[i & 1], e);
-                    acc_r[i & 1] = f2_add(acc_r[i & 1], bf16x2_to_f2(pk[i]));
                 }
                 tmem_st_32x32b_x32(tS + h * 32, pk);
                 tmem_wait_st();
@@ -573,10 +569,19 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
                 exp_half(std::false_type{}, 0);
                 exp_half(std::false_type{}, 1);
             }
-            float a0, a1, b0, b1;
-            f2_unpack(f2_add(acc_r[0], acc_r[1]), a0, a1);
+            // P reaches the MMA rounded to bf16.  O is normalised by the sum with the
+            // tile's largest P taken as rounded (its exponential is recomputed
+            // exactly as in the loop above): a key that dominates a row then has
+            // its rounding cancel in O / l, which is where rounding P costs most.
+            // The LSE takes the unrounded sum.
+            float d_round = 0.0f;
+            if (tmax != -INFINITY) {
+                const float pm = ex2_approx(fmaf(tmax, sl2, -m_sub));
+                d_round = __uint_as_float(pack_bf16x2(pm, 0.0f) << 16) - pm;
+            }
+            float b0, b1;
             f2_unpack(f2_add(acc_e[0], acc_e[1]), b0, b1);
-            l_run += a0 + a1;
+            l_run += (b0 + b1) + d_round;
             l_exact += b0 + b1;
         }
 
