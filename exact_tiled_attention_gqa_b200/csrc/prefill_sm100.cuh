@@ -197,8 +197,8 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
         }
         for (int q = 0; q < 2; ++q) {   // per Q tile (NQ = 2) or per S buffer (NQ = 1)
             mbar_init(bar_s_full(q), 1);
-            mbar_init(bar_p_half(q), 128);
-            mbar_init(bar_p_full(q), 128);
+            mbar_init(bar_p_half(q), 4);   // one arrival per softmax warp
+            mbar_init(bar_p_full(q), 4);
             mbar_init(bar_o_done(q), 1);
         }
         mbar_init(bar_drain, 1);
@@ -560,7 +560,8 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
                 tmem_st_32x32b_x32(tS + h * 32, pk);
                 tmem_wait_st();
                 tc_fence_before_sync();
-                mbar_arrive(h == 0 ? bar_p_half(buf) : bar_p_full(buf));
+                __syncwarp();   // every lane's P is in TMEM: one arrival for the warp
+                if (lane == 0) mbar_arrive(h == 0 ? bar_p_half(buf) : bar_p_full(buf));
             };
             if (masked) {
                 exp_half(std::true_type{}, 0);
