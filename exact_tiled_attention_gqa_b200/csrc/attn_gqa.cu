@@ -146,6 +146,8 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
     if ((st = encode_bf16_3d(&tq, q, D, Lq, static_cast<uint64_t>(B) * Hq, 64, P, G, "q")) != ATTN_OK) return st;
     if ((st = encode_bf16_3d(&tk, k, D, Lk, static_cast<uint64_t>(B) * Hkv, 64, kBN, 1, "k")) != ATTN_OK) return st;
     if ((st = encode_bf16_3d(&tv, v, D, Lk, static_cast<uint64_t>(B) * Hkv, 64, kBN, 1, "v")) != ATTN_OK) return st;
+    CUtensorMap to;   // O is written in the same boxes Q is read in
+    if ((st = encode_bf16_3d(&to, out, D, Lq, static_cast<uint64_t>(B) * Hq, 64, P, G, "out")) != ATTN_OK) return st;
     if ((st = ensure_smem(attn_prefill_sm100_kernel<D, NQ>, L::kAlloc, smem_done)) != ATTN_OK) return st;
     PrefillParams prm;
     prm.out = out;
@@ -165,7 +167,7 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
     const long long grid = static_cast<long long>(B) * Hkv * prm.n_mblk;
     if (grid > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "prefill grid too large (%lld CTAs)", grid);
     attn_prefill_sm100_kernel<D, NQ>
-        <<<static_cast<unsigned>(grid), prefill_threads<NQ>(), L::kAlloc, stream>>>(tq, tk, tv, prm);
+        <<<static_cast<unsigned>(grid), prefill_threads<NQ>(), L::kAlloc, stream>>>(tq, tk, tv, to, prm);
     return check_launch("attn_prefill_sm100_kernel");
 }
 

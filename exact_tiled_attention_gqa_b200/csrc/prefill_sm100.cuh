@@ -136,7 +136,8 @@ template <int D, int NQ>
 __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
     attn_prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                               const __grid_constant__ CUtensorMap tm_k,
-                              const __grid_constant__ CUtensorMap tm_v, const PrefillParams p) {
+                              const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
+                              const PrefillParams p) {
     using L = PrefillSmem<D>;
     static_assert(L::kNQ == NQ, "Q tiles per CTA follow from D");
     constexpr int kThreads = prefill_threads<NQ>();
@@ -586,15 +587,17 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
             l_exact += b0 + b1;
         }
 
-        // ---- epilogue: O / l -> bf16, LSE ----
+        // ---- epilogue: O / l -> bf16 into this Q tile's shared memory (no MMA reads
+        // it any more: the last QK^T precedes the last P.V, which o_done follows),
+        // in the TMA box layout with the 128-byte swizzle, then one TMA store per 64
+        // columns (positions past Lq are clipped by TMA); LSE per row ----
         bool have_o = ok && n_kt > 0;
         if (have_o) {
             have_o = mbar_wait(bar_o_done(q), 0, abort_flag, &g_attn_err, kDevErrTimeout);
             tc_fence_after_sync();
         }
         const float inv_l = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
-        __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.out) +
-                              ((static_cast<size_t>(b) * p.Hq + h) * p.Lq + (row_valid ? pos : 0)) * D;
+        uint8_t* stile = smem + L::kQOff + q * L::kQTileBytes;
 #pragma unroll 1
         for (int c = 0; c < D; c += 32) {
             uint32_t orr[32];
@@ -606,15 +609,25 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
 #pragma unroll
                 for (int i = 0; i < 32; ++i) orr[i] = 0u;
             }
-            if (row_valid) {
-                uint32_t ob[16];
+            uint32_t ob[16];
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    ob[i] = pack_bf16x2(__uint_as_float(orr[2 * i]) * inv_l, __uint_as_float(orr[2 * i + 1]) * inv_l);
-                uint4* dst = reinterpret_cast<uint4*>(orow + c);
+            for (int i = 0; i < 16; ++i)
+                ob[i] = pack_bf16x2(__uint_as_float(orr[2 * i]) * inv_l, __uint_as_float(orr[2 * i + 1]) * inv_l);
+            uint8_t* rowp = stile + (c >> 6) * L::kBlockBytes + r * 128;
+            const int chunk0 = (c & 63) >> 3;   // 16-byte chunk of the 128-byte row: 0 or 4
 #pragma unroll
-                for (int i = 0; i < 4; ++i) dst[i] = make_uint4(ob[4 * i], ob[4 * i + 1], ob[4 * i + 2], ob[4 * i + 3]);
-            }
+            for (int i = 0; i < 4; ++i)
+                *reinterpret_cast<uint4*>(rowp + (((chunk0 + i) ^ (r & 7)) << 4)) =
+                    make_uint4(ob[4 * i], ob[4 * i + 1], ob[4 * i + 2], ob[4 * i + 3]);
+        }
+        fence_proxy_async_smem();
+        asm volatile("bar.sync %0, 128;" ::"r"(1 + q) : "memory");   // the warpgroup's rows are all staged
+        if (r == 0) {
+            const int q_head0 = b * p.Hq + g * p.G;
+            for (int kb = 0; kb < L::kKB; ++kb)
+                tma_store_3d(&tm_o, smem_u32(stile) + kb * L::kBlockBytes, kb * 64, p_begin + q * P, q_head0);
+            tma_store_commit();
+            tma_store_wait_read();   // the shared memory may be released after this
         }
         if (row_valid && p.lse != nullptr) {
             const float lse = (l_exact > 0.0f) ? (m_run + __log2f(l_exact)) * kLn2 : -INFINITY;
