@@ -7,6 +7,8 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdarg>
 #include <cstdint>
@@ -117,6 +119,33 @@ int ensure_smem(Kernel kernel, int bytes, int* done_mask_per_device) {
     return ATTN_OK;
 }
 
+// SMs of the current device, and this launch's scheduling counters for a
+// persistent prefill (slots are taken in turn, see g_prefill_sched).
+int device_sms_and_sched(int* n_sm, int** sched) {
+    static int sms[64];
+    static int* sched_base[64];
+    static std::atomic<unsigned> ticket{0};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+    if (dev < 0 || dev >= 64) return fail(ATTN_ERR_CUDA, "device ordinal %d out of range", dev);
+    int n = __atomic_load_n(&sms[dev], __ATOMIC_ACQUIRE);
+    int* b = __atomic_load_n(&sched_base[dev], __ATOMIC_ACQUIRE);
+    if (n == 0 || b == nullptr) {
+        e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "cudaDeviceGetAttribute: %s", cudaGetErrorString(e));
+        void* addr = nullptr;
+        e = cudaGetSymbolAddress(&addr, g_prefill_sched);
+        if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "cudaGetSymbolAddress: %s", cudaGetErrorString(e));
+        b = static_cast<int*>(addr);
+        __atomic_store_n(&sched_base[dev], b, __ATOMIC_RELEASE);
+        __atomic_store_n(&sms[dev], n, __ATOMIC_RELEASE);
+    }
+    *n_sm = n;
+    *sched = b + 2 * (ticket.fetch_add(1, std::memory_order_relaxed) % kPrefillSchedSlots);
+    return ATTN_OK;
+}
+
 int check_launch(const char* what) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString(e));
@@ -160,12 +189,28 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
     prm.G = G;
     prm.P = P;
     prm.n_mblk = (Lq + NQ * P - 1) / (NQ * P);
-    // longest-first across groups when all of K and V fit in half the L2 (126 MB)
-    prm.mblk_major = (static_cast<double>(B) * Hkv * Lk * D * 2 * 2 <= 63e6) ? 1 : 0;
+    // Unit order: one band of every group when all of K and V fit in half the
+    // L2 (126 MB); otherwise bands of as many groups as fit in 16 MB.  (Bands of
+    // 60 MB raised DRAM reads of the Qwen3-8B B4 L8192 prefill from 403 to about
+    // 710 MB on B200: a tile read from both dies is held in both halves of L2.)
+    {
+        const double group_kv_bytes = static_cast<double>(Lk) * D * 2 * 2;
+        const double n_bh = static_cast<double>(B) * Hkv;
+        const double fit = (group_kv_bytes * n_bh <= 63e6) ? n_bh : std::floor(16e6 / std::max(group_kv_bytes, 1.0));
+        prm.band = static_cast<int>(std::min(std::max(fit, 1.0), n_bh));
+    }
     prm.is_causal = is_causal ? 1 : 0;
     prm.scale_log2 = scale * kLog2e;
-    const long long grid = static_cast<long long>(B) * Hkv * prm.n_mblk;
-    if (grid > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "prefill grid too large (%lld CTAs)", grid);
+    const long long units = static_cast<long long>(B) * Hkv * prm.n_mblk;
+    if (units > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "prefill has too many work units (%lld)", units);
+    prm.n_units = static_cast<int>(units);
+    prm.sched = nullptr;
+    long long grid = units;
+    if (L::kPersistent) {   // one CTA per SM, each taking units until they run out
+        int n_sm = 0;
+        if ((st = device_sms_and_sched(&n_sm, &prm.sched)) != ATTN_OK) return st;
+        grid = std::min<long long>(units, n_sm);
+    }
     attn_prefill_sm100_kernel<D, NQ>
         <<<static_cast<unsigned>(grid), prefill_threads<NQ>(), L::kAlloc, stream>>>(tq, tk, tv, to, prm);
     return check_launch("attn_prefill_sm100_kernel");

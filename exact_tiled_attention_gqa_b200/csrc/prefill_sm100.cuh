@@ -10,25 +10,33 @@
 // and the NVIDIA attention page ("Parameter one: group size": G query heads
 // share one KV head).
 //
-// Work unit (one CTA): one batch b, one KV head g, and NQ*P consecutive query
+// Work unit: one batch b, one KV head g, and NQ*P consecutive query
 // positions, as NQ "Q tiles" of M = 128 rows (NQ = 2 for D <= 128; NQ = 1 for
 // D = 256, whose O accumulator alone takes 256 TMEM columns).  A Q tile packs the G query
 // heads of the group with P = 128 / G positions each (row r = head r / P,
 // position p0 + r % P), so every K/V tile staged in shared memory feeds all
 // G heads of the group and both Q tiles.
 //
+// Persistent CTAs (NQ = 2): one CTA per SM takes unit after unit from an
+// atomic counter, in the unit order of prefill_unit (heaviest first within a
+// group), so the SMs stay balanced whatever the causal mix.  The producer
+// loads the next unit's Q as soon as the last Q K^T of the current unit has
+// read the Q tiles, and its first K/V tiles as ring entries free up, so a
+// unit's start (Q and K_0 in flight, the first Q K^T) overlaps the previous
+// unit's last P.V and epilogue.  An NQ = 1 CTA takes a single unit.
+//
 // Roles for NQ = 2 (384 threads = 3 warpgroups; for NQ = 1 the second softmax
 // warpgroup is absent, warps 4 and 5 are producer and MMA issuer, 256 threads,
 // and no registers are exchanged):
 //   warps 0-3  softmax warpgroup for Q tile 0 (thread = TMEM lane = row)
 //   warps 4-7  softmax warpgroup for Q tile 1
-//   warp  8    TMA producer: Q tiles once, then K_j, V_j into a ring of stages
+//   warp  8    TMA producer: per unit the Q tiles, then K_j, V_j into a ring of stages
 //   warp  9    TMEM allocator and single-thread tcgen05.mma issuer
 //   warps 10-11 idle
 // The block launches at 168 registers per thread (3 warps per SM sub-partition
 // x 168 x 32 = 16128 of its 16384).  The third warpgroup then gives registers
-// back (setmaxnreg.dec to 88) and the softmax warpgroups take them
-// (setmaxnreg.inc to 208): 2 x 208 + 88 = 3 x 168, so the exchange balances
+// back (setmaxnreg.dec to 104) and the softmax warpgroups take them
+// (setmaxnreg.inc to 200): 2 x 200 + 104 = 3 x 168, so the exchange balances
 // exactly and neither side waits.
 //
 // TMEM (512 columns): two S buffers at [0,128) and [128,256), then O.  For
@@ -81,8 +89,8 @@ template <int NQ>
 __host__ __device__ constexpr int prefill_threads() { return 32 * (4 * NQ + 4); }
 __host__ __device__ constexpr int prefill_nq(int D) { return D == 256 ? 1 : 2; }
 constexpr int kPrefillLaunchRegs = 168;    // must equal the compiled register count (checked by the build)
-constexpr int kSoftmaxRegs = 208;
-constexpr int kControlRegs = 88;
+constexpr int kSoftmaxRegs = 200;
+constexpr int kControlRegs = 104;
 static_assert(2 * kSoftmaxRegs + kControlRegs == 3 * kPrefillLaunchRegs, "register exchange must balance");
 constexpr int kBM = 128;               // rows per Q tile (MMA M)
 constexpr int kBN = 128;               // keys per K/V tile
@@ -104,6 +112,9 @@ struct PrefillSmem {
     static constexpr int kKVTileBytes = kBN * D * 2;     // one K or V tile
     static constexpr int kBlockBytes = 128 * 128;        // one 128-row x 128-byte block
     static constexpr int kNQ = prefill_nq(D);
+    // NQ = 2 CTAs are persistent and take work units from a counter; an NQ = 1
+    // CTA takes one unit (its shared memory has no room for the O staging block)
+    static constexpr bool kPersistent = (kNQ == 2);
     // ring entries: whole K or V tiles, or half tiles (32 KB each) for D = 256
     static constexpr int kItemsPerTile = (D == 256) ? 2 : 1;
     static constexpr int kItemBytes = kKVTileBytes / kItemsPerTile;
@@ -111,15 +122,26 @@ struct PrefillSmem {
     static constexpr int kStages = (D == 256) ? 5 : (D == 128) ? 4 : 8;
     static constexpr int kQOff = 0;
     static constexpr int kKVOff = kNQ * kQTileBytes;
-    static constexpr int kBarOff = kKVOff + kStages * kItemBytes;
-    // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_half[2], p_full[2], o_done[2], drain
-    static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 2 + 1;
-    static constexpr int kMiscOff = kBarOff + kNumBars * 8;   // tmem base (u32), abort flag (int)
+    // O staging for the epilogue, one 64-column block per softmax warpgroup
+    // (persistent CTAs: the Q tiles may already hold the next unit's queries)
+    static constexpr int kStgOff = kKVOff + kStages * kItemBytes;
+    static constexpr int kBarOff = kStgOff + (kPersistent ? kNQ * kBlockBytes : 0);
+    // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_half[2], p_full[2], o_done[2], drain,
+    //           q_empty, unit_full[2], unit_empty[2]
+    static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 2 + 1 + 1 + 2 + 2;
+    static constexpr int kMiscOff = kBarOff + kNumBars * 8;   // tmem base, abort flag, two unit slots (int each)
     static constexpr int kBytes = kMiscOff + 16;
     static constexpr int kAlloc = kBytes + 1024;              // slack to align the base to 1 KiB
     static_assert(kAlloc <= 232448, "dynamic shared memory per CTA");
+    static_assert(kStgOff % 1024 == 0, "swizzled TMA blocks start on 1 KiB");
 };
 
+// Scheduling counters of persistent launches: slot i is {next unit, CTAs
+// done}.  Each launch takes a slot in turn from the host; the last of its CTAs
+// to finish puts both counters back to zero, so a slot is ready for its next
+// launch without a memset.
+constexpr int kPrefillSchedSlots = 256;
+__device__ int g_prefill_sched[2 * kPrefillSchedSlots];
 
 struct PrefillParams {
     void* out;          // [B,Hq,Lq,D] bf16
@@ -127,10 +149,46 @@ struct PrefillParams {
     int B, Hq, Hkv, Lq, Lk;
     int G, P;           // group size, positions per Q tile (P = 128 / G)
     int n_mblk;         // ceil(Lq / (NQ P))
-    int mblk_major;     // CTA order: 0 group-major, 1 position-block-major (see the kernel)
+    int n_units;        // B * Hkv * n_mblk
+    int band;           // (b, KV head) groups per band of the unit order (see prefill_unit)
     int is_causal;
     float scale_log2;   // scale * log2(e)
+    int* sched;         // persistent launches: this launch's two counters (zero at launch)
 };
+
+// One work unit: batch b, KV head g, the NQ * P query positions from p_begin,
+// and how many 128-key tiles the latest of them sees.
+struct PrefillUnit {
+    int b, g, p_begin, n_kt;
+};
+
+// Unit `idx` of a launch.  Units run band by band: a band is `band`
+// consecutive (b, KV head) groups (the last band may hold fewer), as many as
+// keep their K/V in about half the L2, so the units that run at the same time
+// find their K/V there.  Within a band the heaviest (latest) position blocks
+// of all its groups come first: the longest-first order that keeps the tail of
+// a causal launch short, since the last units handed out are the lightest.
+template <int NQ>
+__device__ __forceinline__ PrefillUnit prefill_unit(const PrefillParams& p, int idx) {
+    const int n_bh = p.B * p.Hkv;
+    const int per_band = p.band * p.n_mblk;
+    const int k = idx / per_band;
+    const int g0 = k * p.band;
+    const int bs = min(p.band, n_bh - g0);   // groups in this band
+    const int local = idx - k * per_band;
+    const int mblk = p.n_mblk - 1 - local / bs;
+    const int bh = g0 + local % bs;
+    PrefillUnit u;
+    u.b = bh / p.Hkv;
+    u.g = bh % p.Hkv;
+    u.p_begin = mblk * NQ * p.P;
+    const long off = static_cast<long>(p.Lk) - static_cast<long>(p.Lq);
+    const int p_last = min(u.p_begin + NQ * p.P, p.Lq) - 1;
+    const long last_key = p.is_causal ? min(static_cast<long>(p_last) + off, static_cast<long>(p.Lk) - 1)
+                                      : static_cast<long>(p.Lk) - 1;
+    u.n_kt = last_key < 0 ? 0 : static_cast<int>(last_key / kBN) + 1;
+    return u;
+}
 
 template <int D, int NQ>
 __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
@@ -140,9 +198,11 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
                               const PrefillParams p) {
     using L = PrefillSmem<D>;
     static_assert(L::kNQ == NQ, "Q tiles per CTA follow from D");
+    constexpr bool kPersistent = L::kPersistent;
     constexpr int kThreads = prefill_threads<NQ>();
     constexpr int kProducerWarp = 4 * NQ;
     constexpr int kMmaWarp = 4 * NQ + 1;
+    constexpr int kUnitReaders = 1 + 4 * NQ;   // the MMA thread and every softmax warp
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);
     const uint32_t base = (raw_base + 1023u) & ~1023u;
@@ -150,30 +210,8 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-
-    // ---- work unit.  Group-major: one (b, KV head) group after another, so CTAs
-    // running at the same time share that group's K/V in L2; within a group the
-    // heaviest (latest) position blocks come first.  Position-block-major (when
-    // all of K/V fits in L2 anyway): the heaviest blocks of every group first,
-    // the longest-first order that keeps a causal grid's tail short. ----
-    const unsigned n_bh = static_cast<unsigned>(p.B * p.Hkv);
-    const int mblk = p.mblk_major ? p.n_mblk - 1 - static_cast<int>(blockIdx.x / n_bh)
-                                  : p.n_mblk - 1 - static_cast<int>(blockIdx.x % static_cast<unsigned>(p.n_mblk));
-    const int bh = p.mblk_major ? static_cast<int>(blockIdx.x % n_bh)
-                                : static_cast<int>(blockIdx.x / static_cast<unsigned>(p.n_mblk));
-    const int b = bh / p.Hkv;
-    const int g = bh % p.Hkv;
     const int P = p.P;
     const int rows_used = p.G * P;
-    const int p_begin = mblk * NQ * P;
-    const long off = static_cast<long>(p.Lk) - static_cast<long>(p.Lq);
-    int n_kt;
-    {
-        const int p_last = min(p_begin + NQ * P, p.Lq) - 1;
-        const long last_key = p.is_causal ? min(static_cast<long>(p_last) + off, static_cast<long>(p.Lk) - 1)
-                                          : static_cast<long>(p.Lk) - 1;
-        n_kt = last_key < 0 ? 0 : static_cast<int>(last_key / kBN) + 1;
-    }
 
     // ---- shared memory map ----
     const uint32_t sQ = base + L::kQOff;
@@ -187,11 +225,16 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
     auto bar_p_full = [&](int q) { return bar0 + 8u * (5 + 2 * L::kStages + q); };
     auto bar_o_done = [&](int q) { return bar0 + 8u * (7 + 2 * L::kStages + q); };
     const uint32_t bar_drain = bar0 + 8u * (9 + 2 * L::kStages);
+    const uint32_t bar_q_empty = bar0 + 8u * (10 + 2 * L::kStages);
+    auto bar_unit_full = [&](int s) { return bar0 + 8u * (11 + 2 * L::kStages + s); };
+    auto bar_unit_empty = [&](int s) { return bar0 + 8u * (13 + 2 * L::kStages + s); };
     uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+    volatile int* unit_slot = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 8);
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q_full, 1);
+        mbar_init(bar_q_empty, 1);
         for (int s = 0; s < L::kStages; ++s) {
             mbar_init(bar_kv_full(s), 1);
             mbar_init(bar_kv_empty(s), 1);
@@ -201,6 +244,8 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
             mbar_init(bar_p_half(q), 4);   // one arrival per softmax warp
             mbar_init(bar_p_full(q), 4);
             mbar_init(bar_o_done(q), 1);
+            mbar_init(bar_unit_full(q), 1);
+            mbar_init(bar_unit_empty(q), kUnitReaders);
         }
         mbar_init(bar_drain, 1);
         *abort_flag = 0;
@@ -208,6 +253,7 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
     }
     // Q rows the TMA box does not cover (G does not divide 128) must hold
     // finite values: zero them through the generic proxy, then hand them over.
+    // No TMA load writes them, so this holds for every unit.
     if (rows_used < kBM) {
         const int pad_bytes_per_block = (kBM - rows_used) * 128;
         for (int q = 0; q < NQ; ++q)
@@ -227,63 +273,120 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
     tc_fence_after_sync();
     const uint32_t tmem = *tmem_base_ptr;
 
+    // Work units reach the CTA through two shared-memory slots: the producer
+    // writes unit k (or -1: no more) into slot k % 2 and arrives on unit_full;
+    // the MMA thread and the softmax warps read it and arrive on unit_empty.
+    // The first unit is blockIdx.x; a persistent CTA then takes gridDim.x + c,
+    // c from the launch's counter, until the units run out.  Barrier phases
+    // and ring positions run on across units.
+
     if (warp >= kProducerWarp) {
       if constexpr (NQ == 2) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kControlRegs));
       if (warp == kProducerWarp) {
         // ================= TMA producer =================
-        if (lane == 0 && n_kt > 0) {
+        if (lane == 0) {
             tma_prefetch_desc(&tm_q);
             tma_prefetch_desc(&tm_k);
             tma_prefetch_desc(&tm_v);
-            const int q_head0 = b * p.Hq + g * p.G;
-            mbar_arrive_expect_tx(bar_q_full, static_cast<uint32_t>(NQ * L::kKB * rows_used * 128));
-            for (int q = 0; q < NQ; ++q)
-                for (int kb = 0; kb < L::kKB; ++kb)
-                    tma_load_3d(sQ + q * L::kQTileBytes + kb * L::kBlockBytes, &tm_q, bar_q_full, kb * 64,
-                                p_begin + q * P, q_head0);
-            const int kv_row = b * p.Hkv + g;
-            int issued = 0;
+            tma_prefetch_desc(&tm_o);
+            const uint32_t q_bytes = static_cast<uint32_t>(NQ * L::kKB * rows_used * 128);
+            int idx = blockIdx.x;
+            int t = 0;    // ring entries issued, over all units
+            int nu = 0;   // units with at least one key tile (Q loads)
             bool ok = true;
-            for (int t = 0; t < 2 * n_kt * L::kItemsPerTile && ok; ++t) {
-                const int s = t % L::kStages;
-                const uint32_t round = static_cast<uint32_t>(t / L::kStages);
-                ok = mbar_wait(bar_kv_empty(s), (round & 1u) ^ 1u, abort_flag, &g_attn_err, kDevErrTimeout);
+            for (int k = 0;; ++k) {
+                const int s = k & 1;
+                ok = mbar_wait(bar_unit_empty(s), static_cast<uint32_t>((k >> 1) & 1) ^ 1u, abort_flag, &g_attn_err,
+                               kDevErrTimeout);
                 if (!ok) break;
-                mbar_arrive_expect_tx(bar_kv_full(s), L::kItemBytes);
-                bool is_v;
-                int j;
-                ring_tile<NQ>(t / L::kItemsPerTile, n_kt, is_v, j);
-                const int kb0 = (t % L::kItemsPerTile) * L::kItemKB;
-                const CUtensorMap* map = is_v ? &tm_v : &tm_k;
-                for (int kb = 0; kb < L::kItemKB; ++kb)
-                    tma_load_3d(sKV + s * L::kItemBytes + kb * L::kBlockBytes, map, bar_kv_full(s), (kb0 + kb) * 64,
-                                j * kBN, kv_row);
-                issued = t + 1;
+                const bool have = idx < p.n_units;
+                unit_slot[s] = have ? idx : -1;
+                mbar_arrive(bar_unit_full(s));
+                if (!have) break;
+                const PrefillUnit u = prefill_unit<NQ>(p, idx);
+                // The next unit is taken once this one's loads are all issued (about
+                // two key tiles before its MMAs end), not earlier: a CTA that claimed
+                // its next unit at the start of a long one would hold it back from SMs
+                // that run dry at the end of the launch.
+                auto next_unit = [&]() {
+                    return kPersistent ? static_cast<int>(gridDim.x) + atomicAdd(p.sched, 1) : p.n_units;
+                };
+                if (u.n_kt == 0) {
+                    idx = next_unit();
+                    continue;
+                }
+                if (nu > 0) {   // the previous unit's last Q K^T has read the Q tiles
+                    ok = mbar_wait(bar_q_empty, static_cast<uint32_t>(nu - 1) & 1u, abort_flag, &g_attn_err,
+                                   kDevErrTimeout);
+                    if (!ok) break;
+                }
+                const int q_head0 = u.b * p.Hq + u.g * p.G;
+                mbar_arrive_expect_tx(bar_q_full, q_bytes);
+                for (int q = 0; q < NQ; ++q)
+                    for (int kb = 0; kb < L::kKB; ++kb)
+                        tma_load_3d(sQ + q * L::kQTileBytes + kb * L::kBlockBytes, &tm_q, bar_q_full, kb * 64,
+                                    u.p_begin + q * P, q_head0);
+                ++nu;
+                const int kv_row = u.b * p.Hkv + u.g;
+                const int n_items = 2 * u.n_kt * L::kItemsPerTile;
+                for (int i = 0; i < n_items; ++i) {
+                    const int st = t % L::kStages;
+                    const uint32_t round = static_cast<uint32_t>(t / L::kStages);
+                    ok = mbar_wait(bar_kv_empty(st), (round & 1u) ^ 1u, abort_flag, &g_attn_err, kDevErrTimeout);
+                    if (!ok) break;
+                    mbar_arrive_expect_tx(bar_kv_full(st), L::kItemBytes);
+                    bool is_v;
+                    int j;
+                    ring_tile<NQ>(i / L::kItemsPerTile, u.n_kt, is_v, j);
+                    const int kb0 = (i % L::kItemsPerTile) * L::kItemKB;
+                    const CUtensorMap* map = is_v ? &tm_v : &tm_k;
+                    for (int kb = 0; kb < L::kItemKB; ++kb)
+                        tma_load_3d(sKV + st * L::kItemBytes + kb * L::kBlockBytes, map, bar_kv_full(st),
+                                    (kb0 + kb) * 64, j * kBN, kv_row);
+                    ++t;
+                }
+                if (!ok) break;
+                idx = next_unit();
             }
             if (!ok) {
                 // Unwinding: let the copies already issued land before the CTA exits.
-                for (int t = max(0, issued - L::kStages); t < issued; ++t) {
-                    const int s = t % L::kStages;
+                for (int t2 = max(0, t - L::kStages); t2 < t; ++t2) {
+                    const int st = t2 % L::kStages;
                     const uint64_t t0 = global_timer_ns();
-                    while (!mbar_try_wait(bar_kv_full(s), static_cast<uint32_t>(t / L::kStages) & 1u) &&
+                    while (!mbar_try_wait(bar_kv_full(st), static_cast<uint32_t>(t2 / L::kStages) & 1u) &&
                            global_timer_ns() - t0 < 100000000ull) {
                     }
                 }
-                const uint64_t t0 = global_timer_ns();
-                while (!mbar_try_wait(bar_q_full, 0) && global_timer_ns() - t0 < 100000000ull) {
+                if (nu > 0) {
+                    const uint64_t t0 = global_timer_ns();
+                    while (!mbar_try_wait(bar_q_full, static_cast<uint32_t>(nu - 1) & 1u) &&
+                           global_timer_ns() - t0 < 100000000ull) {
+                    }
+                }
+            }
+            if constexpr (kPersistent) {
+                // This CTA takes no more units.  The last CTA to get here leaves
+                // both counters at zero for the slot's next launch.
+                __threadfence();
+                if (atomicAdd(p.sched + 1, 1) == static_cast<int>(gridDim.x) - 1) {
+                    atomicExch(p.sched, 0);
+                    atomicExch(p.sched + 1, 0);
                 }
             }
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // ================= MMA issuer =================
-        if (lane == 0 && n_kt > 0) {
+        if (lane == 0) {
             constexpr uint32_t kIdescQK = umma_idesc_bf16_f32(kBM, kBN, false);
             constexpr uint32_t kIdescPV = umma_idesc_bf16_f32(kBM, D, true);
             const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
             const uint32_t tO[2] = {tmem + 256u, tmem + 256u + D};
-            auto slot_of = [&](int t) { return t % L::kStages; };
-            auto par_of = [&](int t) { return static_cast<uint32_t>(t / L::kStages) & 1u; };
+            int tb = 0;      // ring entries of earlier units
+            int tiles = 0;   // key tiles of earlier units (phases of the per-tile barriers)
+            int nu = 0;      // earlier units with key tiles
+            auto slot_of = [&](int t) { return (tb + t) % L::kStages; };
+            auto par_of = [&](int t) { return static_cast<uint32_t>((tb + t) / L::kStages) & 1u; };
             // Shared-memory descriptors are built once; a k-step only moves the
             // start-address field (bits 0-13, address >> 4), so each MMA issue
             // costs one 64-bit add.
@@ -313,120 +416,133 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
             };
             // both halves of O_q += P_q(j) V_j, each as soon as the softmax has released it
             auto pv_tile = [&](int q, int t, int j) {
-                if (!mbar_wait(bar_p_half(q), static_cast<uint32_t>(j) & 1u, abort_flag, &g_attn_err, kDevErrTimeout))
-                    return false;
+                const uint32_t ph = static_cast<uint32_t>(tiles + j) & 1u;
+                if (!mbar_wait(bar_p_half(q), ph, abort_flag, &g_attn_err, kDevErrTimeout)) return false;
                 tc_fence_after_sync();
                 issue_pv(q, t, j > 0, 0);
-                if (!mbar_wait(bar_p_full(q), static_cast<uint32_t>(j) & 1u, abort_flag, &g_attn_err, kDevErrTimeout))
-                    return false;
+                if (!mbar_wait(bar_p_full(q), ph, abort_flag, &g_attn_err, kDevErrTimeout)) return false;
                 tc_fence_after_sync();
                 issue_pv(q, t, true, 1);
                 return true;
             };
-            bool ok = mbar_wait(bar_q_full, 0, abort_flag, &g_attn_err, kDevErrTimeout);
-          if constexpr (NQ == 2) {
-            if (ok) ok = mbar_wait(bar_kv_full(slot_of(0)), par_of(0), abort_flag, &g_attn_err, kDevErrTimeout);
-            if (ok) {
-                tc_fence_after_sync();
-                issue_qk(0, 0);
-                umma_commit(bar_s_full(0));
-                if constexpr (NQ == 2) {
+            bool ok = true;
+            for (int k = 0; ok; ++k) {
+                const int s = k & 1;
+                ok = mbar_wait(bar_unit_full(s), static_cast<uint32_t>(k >> 1) & 1u, abort_flag, &g_attn_err,
+                               kDevErrTimeout);
+                if (!ok) break;
+                const int idx = unit_slot[s];
+                mbar_arrive(bar_unit_empty(s));
+                if (idx < 0) break;
+                const int n_kt = prefill_unit<NQ>(p, idx).n_kt;
+                if (n_kt == 0) continue;
+                ok = mbar_wait(bar_q_full, static_cast<uint32_t>(nu) & 1u, abort_flag, &g_attn_err, kDevErrTimeout);
+              if constexpr (NQ == 2) {
+                if (ok) ok = mbar_wait(bar_kv_full(slot_of(0)), par_of(0), abort_flag, &g_attn_err, kDevErrTimeout);
+                if (ok) {
+                    tc_fence_after_sync();
+                    issue_qk(0, 0);
+                    umma_commit(bar_s_full(0));
                     issue_qk(1, 0);
                     umma_commit(bar_s_full(1));
+                    if (n_kt == 1) umma_commit(bar_q_empty);
+                    umma_commit(bar_kv_empty(slot_of(0)));
                 }
-                umma_commit(bar_kv_empty(slot_of(0)));
-            }
-            for (int j = 0; j < n_kt && ok; ++j) {
-                const int tv = 2 * j + 1, tk = 2 * j + 2;
-                const bool last = (j + 1 == n_kt);
-                // operands first (normally long landed), so only the P waits sit on the chain
-                ok = mbar_wait(bar_kv_full(slot_of(tv)), par_of(tv), abort_flag, &g_attn_err, kDevErrTimeout);
-                if (ok && !last)
-                    ok = mbar_wait(bar_kv_full(slot_of(tk)), par_of(tk), abort_flag, &g_attn_err, kDevErrTimeout);
-                ok = ok && pv_tile(0, tv, j);
-                if (!ok) break;
-                if (last) umma_commit(bar_o_done(0));
-                if (!last) {
-                    issue_qk(0, tk);
-                    umma_commit(bar_s_full(0));
-                }
-                if constexpr (NQ == 2) {
+                for (int j = 0; j < n_kt && ok; ++j) {
+                    const int tv = 2 * j + 1, tk = 2 * j + 2;
+                    const bool last = (j + 1 == n_kt);
+                    // operands first (normally long landed), so only the P waits sit on the chain
+                    ok = mbar_wait(bar_kv_full(slot_of(tv)), par_of(tv), abort_flag, &g_attn_err, kDevErrTimeout);
+                    if (ok && !last)
+                        ok = mbar_wait(bar_kv_full(slot_of(tk)), par_of(tk), abort_flag, &g_attn_err, kDevErrTimeout);
+                    ok = ok && pv_tile(0, tv, j);
+                    if (!ok) break;
+                    if (last) umma_commit(bar_o_done(0));
+                    if (!last) {
+                        issue_qk(0, tk);
+                        umma_commit(bar_s_full(0));
+                    }
                     ok = pv_tile(1, tv, j);
                     if (!ok) break;
                     if (last) umma_commit(bar_o_done(1));
-                }
-                umma_commit(bar_kv_empty(slot_of(tv)));
-                if (!last) {
-                    if constexpr (NQ == 2) {
+                    umma_commit(bar_kv_empty(slot_of(tv)));
+                    if (!last) {
                         issue_qk(1, tk);
                         umma_commit(bar_s_full(1));
+                        if (j + 2 == n_kt) umma_commit(bar_q_empty);   // the unit's last reads of Q
+                        umma_commit(bar_kv_empty(slot_of(tk)));
                     }
-                    umma_commit(bar_kv_empty(slot_of(tk)));
                 }
-            }
-          } else {
-            // ---- one Q tile, S double-buffered (D = 256) ----
-            constexpr uint32_t kIdescPVh = umma_idesc_bf16_f32(kBM, 128, true);
-            const uint32_t tOq = tmem + 256u;
-            auto wait_item = [&](int it) {
-                return mbar_wait(bar_kv_full(slot_of(it)), par_of(it), abort_flag, &g_attn_err, kDevErrTimeout);
-            };
-            // S(j) into buffer j % 2, K_j in two half entries (columns 0-127, 128-255)
-            auto qk = [&](int j) {
-                const int it0 = L::kItemsPerTile * ring_pos_k<NQ>(j);
-                const uint32_t tSb = tS[j & 1];
-                for (int hh = 0; hh < 2; ++hh) {
-                    if (!wait_item(it0 + hh)) return false;
+              } else if (ok) {
+                // ---- one Q tile, S double-buffered (D = 256; one unit per CTA, so
+                // ring positions and phases start at zero) ----
+                constexpr uint32_t kIdescPVh = umma_idesc_bf16_f32(kBM, 128, true);
+                const uint32_t tOq = tmem + 256u;
+                auto wait_item = [&](int it) {
+                    return mbar_wait(bar_kv_full(slot_of(it)), par_of(it), abort_flag, &g_attn_err, kDevErrTimeout);
+                };
+                // S(j) into buffer j % 2, K_j in two half entries (columns 0-127, 128-255)
+                auto qk = [&](int j) {
+                    const int it0 = L::kItemsPerTile * ring_pos_k<NQ>(j);
+                    const uint32_t tSb = tS[j & 1];
+                    for (int hh = 0; hh < 2; ++hh) {
+                        if (!wait_item(it0 + hh)) return false;
+                        tc_fence_after_sync();
+                        const uint64_t b0 = dK0 + static_cast<uint64_t>(slot_of(it0 + hh)) * kSlotStep;
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const int kq = hh * 8 + kk;
+                            const uint64_t koff =
+                                static_cast<uint64_t>(((kk >> 2) * L::kBlockBytes + (kk & 3) * 32) >> 4);
+                            const uint64_t qoff =
+                                static_cast<uint64_t>(((kq >> 2) * L::kBlockBytes + (kq & 3) * 32) >> 4);
+                            umma_ss(tSb, dQ[0] + qoff, b0 + koff, kIdescQK, kq > 0 ? 1u : 0u);
+                        }
+                        umma_commit(bar_kv_empty(slot_of(it0 + hh)));
+                    }
+                    umma_commit(bar_s_full(j & 1));
+                    return true;
+                };
+                // O[:, 128 hv .. +128) += P(j)[:, keys of `half`] V_j^(hv)
+                auto pv_part = [&](int j, int itv, int half) {
+                    const uint32_t tSb = tS[j & 1];
+#pragma unroll
+                    for (int hv = 0; hv < 2; ++hv) {
+                        const uint64_t b0 = dV0 + static_cast<uint64_t>(slot_of(itv + hv)) * kSlotStep;
+#pragma unroll
+                        for (int k4 = 0; k4 < kBN / 32; ++k4) {
+                            const int kk = half * (kBN / 32) + k4;
+                            umma_ts(tOq + 128u * hv, tSb + kk * 8, b0 + static_cast<uint64_t>((kk * 2048) >> 4),
+                                    kIdescPVh, (j > 0 || kk > 0) ? 1u : 0u);
+                        }
+                    }
+                };
+                ok = qk(0);
+                if (ok && n_kt > 1) ok = qk(1);
+                for (int j = 0; j < n_kt && ok; ++j) {
+                    const int buf = j & 1;
+                    const uint32_t ph = static_cast<uint32_t>(j >> 1) & 1u;
+                    const int itv = L::kItemsPerTile * ring_pos_v<NQ>(j, n_kt);
+                    ok = wait_item(itv) && wait_item(itv + 1);
+                    ok = ok && mbar_wait(bar_p_half(buf), ph, abort_flag, &g_attn_err, kDevErrTimeout);
+                    if (!ok) break;
                     tc_fence_after_sync();
-                    const uint64_t b0 = dK0 + static_cast<uint64_t>(slot_of(it0 + hh)) * kSlotStep;
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const int kq = hh * 8 + kk;
-                        const uint64_t koff = static_cast<uint64_t>(((kk >> 2) * L::kBlockBytes + (kk & 3) * 32) >> 4);
-                        const uint64_t qoff = static_cast<uint64_t>(((kq >> 2) * L::kBlockBytes + (kq & 3) * 32) >> 4);
-                        umma_ss(tSb, dQ[0] + qoff, b0 + koff, kIdescQK, kq > 0 ? 1u : 0u);
-                    }
-                    umma_commit(bar_kv_empty(slot_of(it0 + hh)));
+                    pv_part(j, itv, 0);
+                    ok = mbar_wait(bar_p_full(buf), ph, abort_flag, &g_attn_err, kDevErrTimeout);
+                    if (!ok) break;
+                    tc_fence_after_sync();
+                    pv_part(j, itv, 1);
+                    umma_commit(bar_o_done(1));              // o_ready: O holds tiles 0..j
+                    if (j + 1 == n_kt) umma_commit(bar_o_done(0));
+                    umma_commit(bar_kv_empty(slot_of(itv)));
+                    umma_commit(bar_kv_empty(slot_of(itv + 1)));
+                    if (j + 2 < n_kt) ok = qk(j + 2);
                 }
-                umma_commit(bar_s_full(j & 1));
-                return true;
-            };
-            // O[:, 128 hv .. +128) += P(j)[:, keys of `half`] V_j^(hv)
-            auto pv_part = [&](int j, int itv, int half) {
-                const uint32_t tSb = tS[j & 1];
-#pragma unroll
-                for (int hv = 0; hv < 2; ++hv) {
-                    const uint64_t b0 = dV0 + static_cast<uint64_t>(slot_of(itv + hv)) * kSlotStep;
-#pragma unroll
-                    for (int k4 = 0; k4 < kBN / 32; ++k4) {
-                        const int kk = half * (kBN / 32) + k4;
-                        umma_ts(tOq + 128u * hv, tSb + kk * 8, b0 + static_cast<uint64_t>((kk * 2048) >> 4),
-                                kIdescPVh, (j > 0 || kk > 0) ? 1u : 0u);
-                    }
-                }
-            };
-            if (ok) ok = qk(0);
-            if (ok && n_kt > 1) ok = qk(1);
-            for (int j = 0; j < n_kt && ok; ++j) {
-                const int buf = j & 1;
-                const uint32_t ph = static_cast<uint32_t>(j >> 1) & 1u;
-                const int itv = L::kItemsPerTile * ring_pos_v<NQ>(j, n_kt);
-                ok = wait_item(itv) && wait_item(itv + 1);
-                ok = ok && mbar_wait(bar_p_half(buf), ph, abort_flag, &g_attn_err, kDevErrTimeout);
-                if (!ok) break;
-                tc_fence_after_sync();
-                pv_part(j, itv, 0);
-                ok = mbar_wait(bar_p_full(buf), ph, abort_flag, &g_attn_err, kDevErrTimeout);
-                if (!ok) break;
-                tc_fence_after_sync();
-                pv_part(j, itv, 1);
-                umma_commit(bar_o_done(1));              // o_ready: O holds tiles 0..j
-                if (j + 1 == n_kt) umma_commit(bar_o_done(0));
-                umma_commit(bar_kv_empty(slot_of(itv)));
-                umma_commit(bar_kv_empty(slot_of(itv + 1)));
-                if (j + 2 < n_kt) ok = qk(j + 2);
+              }
+                tb += 2 * n_kt * L::kItemsPerTile;
+                tiles += n_kt;
+                ++nu;
             }
-          }
             // Drain: no MMA may still be running when TMEM is released.
             umma_commit(bar_drain);
             const uint64_t t0 = global_timer_ns();
@@ -440,199 +556,254 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
         // ================= softmax warpgroups =================
         const int q = warp >> 2;                 // Q tile of this warpgroup
         const int r = threadIdx.x & 127;         // row = TMEM lane
+        const int wg_bar = 1 + q;                // this warpgroup's named barrier
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t tS_q = tmem + (q ? 128u : 0u) + lane_off;
         const uint32_t tO = tmem + 256u + (q ? static_cast<uint32_t>(D) : 0u) + lane_off;
         const int head_local = r / P;
-        const int pos = p_begin + q * P + (r % P);
-        const bool row_valid = (r < rows_used) && (pos < p.Lq);
-        const int h = g * p.G + head_local;
-        // last visible key of this row, and the smallest such bound over the tile's rows
+        const long off = static_cast<long>(p.Lk) - static_cast<long>(p.Lq);
         const long lk1 = static_cast<long>(p.Lk) - 1;
-        const long bound = p.is_causal ? min(static_cast<long>(pos) + off, lk1) : lk1;
-        const int tile_p0 = p_begin + q * P;
-        const long tile_min_bound = p.is_causal ? min(static_cast<long>(tile_p0) + off, lk1) : lk1;
         const float sl2 = p.scale_log2;
-
-        float m_run = -INFINITY;   // running max used for the exponentials (log2 domain)
-        float l_run = 0.0f;        // running sum normalising O (see the exponentials below)
-        float l_exact = 0.0f;      // running sum of the unrounded exponentials (for the LSE)
+        int tiles = 0;   // key tiles of earlier units (barrier phases)
+        int nu = 0;      // earlier units with key tiles (o_done phase)
         bool ok = true;
-        for (int j = 0; j < n_kt; ++j) {
-            // S buffer of this tile, and the phase of its barriers
-            const int buf = (NQ == 2) ? q : (j & 1);
-            const uint32_t ph = static_cast<uint32_t>(NQ == 2 ? j : (j >> 1)) & 1u;
-            const uint32_t tS = (NQ == 2) ? tS_q : tS_q + (static_cast<uint32_t>(j & 1) << 7);
-            ok = mbar_wait(bar_s_full(buf), ph, abort_flag, &g_attn_err, kDevErrTimeout);
-            if (!ok) break;
-            tc_fence_after_sync();
-            uint32_t sr[128];
-            tmem_ld_32x32b_x32(tS + 0, sr + 0);
-            tmem_ld_32x32b_x32(tS + 32, sr + 32);
-            tmem_ld_32x32b_x32(tS + 64, sr + 64);
-            tmem_ld_32x32b_x32(tS + 96, sr + 96);
-            tmem_wait_ld();
-            reg_fence<128>(sr);
-            float s[kBN];
-#pragma unroll
-            for (int c = 0; c < kBN; ++c) s[c] = __uint_as_float(sr[c]);
-            const long key0 = static_cast<long>(j) * kBN;
-            const bool masked = key0 + kBN - 1 > tile_min_bound;
-            if (masked) {
-                // diagonal or ragged tile: mask keys beyond this row's bound
-#pragma unroll
-                for (int c = 0; c < kBN; ++c)
-                    if (key0 + c > bound) s[c] = -INFINITY;
+        for (int k = 0;; ++k) {
+            const int s = k & 1;
+            int idx = -1;
+            if (ok) {
+                ok = mbar_wait(bar_unit_full(s), static_cast<uint32_t>(k >> 1) & 1u, abort_flag, &g_attn_err,
+                               kDevErrTimeout);
+                if (ok) idx = unit_slot[s];
             }
-            float mx[8];
+            // The warpgroup decides together (its threads meet at named barriers
+            // in the epilogue); the barrier also orders every lane's read of the
+            // slot before the warp's release of it.
+            if (named_bar_or(wg_bar, 128, !ok || idx < 0)) break;
+            if (lane == 0) mbar_arrive(bar_unit_empty(s));
+            const PrefillUnit u = prefill_unit<NQ>(p, idx);
+            const int n_kt = u.n_kt;
+            const int pos = u.p_begin + q * P + (r % P);
+            const bool row_valid = (r < rows_used) && (pos < p.Lq);
+            const int h = u.g * p.G + head_local;
+            // last visible key of this row, and the smallest such bound over the tile's rows
+            const long bound = p.is_causal ? min(static_cast<long>(pos) + off, lk1) : lk1;
+            const int tile_p0 = u.p_begin + q * P;
+            const long tile_min_bound = p.is_causal ? min(static_cast<long>(tile_p0) + off, lk1) : lk1;
+
+            float m_run = -INFINITY;   // running max used for the exponentials (log2 domain)
+            float l_run = 0.0f;        // running sum normalising O (see the exponentials below)
+            float l_exact = 0.0f;      // running sum of the unrounded exponentials (for the LSE)
+            for (int j = 0; j < n_kt; ++j) {
+                // S buffer of this tile, and the phase of its barriers
+                const int buf = (NQ == 2) ? q : (j & 1);
+                const uint32_t ph = static_cast<uint32_t>(NQ == 2 ? tiles + j : (j >> 1)) & 1u;
+                const uint32_t tS = (NQ == 2) ? tS_q : tS_q + (static_cast<uint32_t>(j & 1) << 7);
+                ok = mbar_wait(bar_s_full(buf), ph, abort_flag, &g_attn_err, kDevErrTimeout);
+                if (!ok) break;
+                tc_fence_after_sync();
+                uint32_t sr[128];
+                tmem_ld_32x32b_x32(tS + 0, sr + 0);
+                tmem_ld_32x32b_x32(tS + 32, sr + 32);
+                tmem_ld_32x32b_x32(tS + 64, sr + 64);
+                tmem_ld_32x32b_x32(tS + 96, sr + 96);
+                tmem_wait_ld();
+                reg_fence<128>(sr);
+                float sv[kBN];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) mx[i] = fmax3(s[i], s[8 + i], s[16 + i]);
+                for (int c = 0; c < kBN; ++c) sv[c] = __uint_as_float(sr[c]);
+                const long key0 = static_cast<long>(j) * kBN;
+                const bool masked = key0 + kBN - 1 > tile_min_bound;
+                if (masked) {
+                    // diagonal or ragged tile: mask keys beyond this row's bound
 #pragma unroll
-            for (int c = 24; c < kBN - 8; c += 16)
-#pragma unroll
-                for (int i = 0; i < 8; ++i) mx[i] = fmax3(mx[i], s[c + i], s[c + 8 + i]);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], s[kBN - 8 + i]);
-            const float tmax = fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(fmax3(mx[3], mx[4], mx[5]), mx[6], mx[7]));
-            const float m_tile = tmax * sl2;   // -inf stays -inf
-            float factor = 1.0f;
-            if (m_tile > m_run + kRescaleLog2) {
-                factor = (m_run == -INFINITY) ? 0.0f : ex2_approx(m_run - m_tile);
-                m_run = m_tile;
-                l_run *= factor;
-                l_exact *= factor;
-            }
-            // rescale O_q in TMEM if any row of this warp raised its max (O holds
-            // the sum over tiles < j, settled: see the file comment)
-            if (j > 0 && __any_sync(0xffffffffu, factor != 1.0f)) {
-                if constexpr (NQ == 1) {
-                    // O += P(j-1) V_{j-1} must have landed (at most one P.V is outstanding)
-                    if (!mbar_wait(bar_o_done(1), static_cast<uint32_t>(j - 1) & 1u, abort_flag, &g_attn_err,
-                                   kDevErrTimeout)) {
-                        ok = false;
-                        break;
-                    }
-                    tc_fence_after_sync();
+                    for (int c = 0; c < kBN; ++c)
+                        if (key0 + c > bound) sv[c] = -INFINITY;
                 }
-                const uint64_t f2 = f2_pack(factor, factor);
+                float mx[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) mx[i] = fmax3(sv[i], sv[8 + i], sv[16 + i]);
+#pragma unroll
+                for (int c = 24; c < kBN - 8; c += 16)
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) mx[i] = fmax3(mx[i], sv[c + i], sv[c + 8 + i]);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) mx[i] = fmaxf(mx[i], sv[kBN - 8 + i]);
+                const float tmax =
+                    fmaxf(fmax3(mx[0], mx[1], mx[2]), fmax3(fmax3(mx[3], mx[4], mx[5]), mx[6], mx[7]));
+                const float m_tile = tmax * sl2;   // -inf stays -inf
+                float factor = 1.0f;
+                if (m_tile > m_run + kRescaleLog2) {
+                    factor = (m_run == -INFINITY) ? 0.0f : ex2_approx(m_run - m_tile);
+                    m_run = m_tile;
+                    l_run *= factor;
+                    l_exact *= factor;
+                }
+                // rescale O_q in TMEM if any row of this warp raised its max (O holds
+                // the sum over tiles < j, settled: see the file comment)
+                if (j > 0 && __any_sync(0xffffffffu, factor != 1.0f)) {
+                    if constexpr (NQ == 1) {
+                        // O += P(j-1) V_{j-1} must have landed (at most one P.V is outstanding)
+                        if (!mbar_wait(bar_o_done(1), static_cast<uint32_t>(j - 1) & 1u, abort_flag, &g_attn_err,
+                                       kDevErrTimeout)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after_sync();
+                    }
+                    const uint64_t f2 = f2_pack(factor, factor);
 #pragma unroll 1
-                for (int c = 0; c < D; c += 32) {
-                    uint32_t orr[32];
+                    for (int c = 0; c < D; c += 32) {
+                        uint32_t orr[32];
+                        tmem_ld_32x32b_x32(tO + c, orr);
+                        tmem_wait_ld();
+                        reg_fence<32>(orr);
+#pragma unroll
+                        for (int i = 0; i < 32; i += 2) {
+                            float a0, a1;
+                            f2_unpack(f2_mul(f2_pack(__uint_as_float(orr[i]), __uint_as_float(orr[i + 1])), f2), a0,
+                                      a1);
+                            orr[i] = __float_as_uint(a0);
+                            orr[i + 1] = __float_as_uint(a1);
+                        }
+                        tmem_st_32x32b_x32(tO + c, orr);
+                    }
+                    tmem_wait_st();
+                }
+                // exponentials 2^(s * scale * log2 e - m), the row sum, and P (bf16)
+                // into TMEM in two halves, each handed to the MMA thread at once
+                const float m_sub = (m_run == -INFINITY) ? 0.0f : m_run;
+                const uint64_t sl2x2 = f2_pack(sl2, sl2);
+                const uint64_t negm2 = f2_pack(-m_sub, -m_sub);
+                uint64_t acc_e[2] = {0ull, 0ull};
+                auto exp_half = [&](auto masked_tag, int hf) {
+                    constexpr bool kMasked = decltype(masked_tag)::value;
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int c = hf * 64 + 2 * i;
+                        const uint64_t t = f2_fma(f2_pack(sv[c], sv[c + 1]), sl2x2, negm2);
+                        uint64_t e;
+                        if (!kMasked && (i % 8) < kExpFmaPairsPer8) {
+                            e = exp2_fma_x2(t);
+                        } else {
+                            float t0, t1;
+                            f2_unpack(t, t0, t1);
+                            e = f2_pack(ex2_approx(t0), ex2_approx(t1));
+                        }
+                        float e0, e1;
+                        f2_unpack(e, e0, e1);
+                        pk[i] = pack_bf16x2(e0, e1);
+                        acc_e[i & 1] = f2_add(acc_e[i & 1], e);
+                    }
+                    tmem_st_32x32b_x32(tS + hf * 32, pk);
+                    tmem_wait_st();
+                    tc_fence_before_sync();
+                    __syncwarp();   // every lane's P is in TMEM: one arrival for the warp
+                    if (lane == 0) mbar_arrive(hf == 0 ? bar_p_half(buf) : bar_p_full(buf));
+                };
+                if (masked) {
+                    exp_half(std::true_type{}, 0);
+                    exp_half(std::true_type{}, 1);
+                } else {
+                    exp_half(std::false_type{}, 0);
+                    exp_half(std::false_type{}, 1);
+                }
+                // P reaches the MMA rounded to bf16.  O is normalised by the sum with the
+                // tile's largest P taken as rounded (its exponential is recomputed
+                // exactly as in the loop above): a key that dominates a row then has
+                // its rounding cancel in O / l, which is where rounding P costs most.
+                // The LSE takes the unrounded sum.
+                float d_round = 0.0f;
+                if (tmax != -INFINITY) {
+                    const float pm = ex2_approx(fmaf(tmax, sl2, -m_sub));
+                    d_round = __uint_as_float(pack_bf16x2(pm, 0.0f) << 16) - pm;
+                }
+                float b0, b1;
+                f2_unpack(f2_add(acc_e[0], acc_e[1]), b0, b1);
+                l_run += (b0 + b1) + d_round;
+                l_exact += b0 + b1;
+            }
+
+            // ---- epilogue: O / l -> bf16, staged in shared memory in the TMA box
+            // layout (128-byte swizzle) and written with TMA stores, 64 columns
+            // per store (positions past Lq are clipped by TMA); LSE per row ----
+            bool have_o = ok && n_kt > 0;
+            if (have_o) {
+                have_o = mbar_wait(bar_o_done(q), static_cast<uint32_t>(nu) & 1u, abort_flag, &g_attn_err,
+                                   kDevErrTimeout);
+                ok = have_o;
+                tc_fence_after_sync();
+            }
+            const float inv_l = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
+            const int q_head0 = u.b * p.Hq + u.g * p.G;
+            auto o_cols = [&](int c, uint32_t* ob) {   // 32 columns from c, packed into 16 words
+                uint32_t orr[32];
+                if (have_o) {
                     tmem_ld_32x32b_x32(tO + c, orr);
                     tmem_wait_ld();
                     reg_fence<32>(orr);
+                } else {
 #pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        float a0, a1;
-                        f2_unpack(f2_mul(f2_pack(__uint_as_float(orr[i]), __uint_as_float(orr[i + 1])), f2), a0, a1);
-                        orr[i] = __float_as_uint(a0);
-                        orr[i + 1] = __float_as_uint(a1);
-                    }
-                    tmem_st_32x32b_x32(tO + c, orr);
+                    for (int i = 0; i < 32; ++i) orr[i] = 0u;
                 }
-                tmem_wait_st();
-            }
-            // exponentials 2^(s * scale * log2 e - m), the row sum, and P (bf16)
-            // into TMEM in two halves, each handed to the MMA thread at once
-            const float m_sub = (m_run == -INFINITY) ? 0.0f : m_run;
-            const uint64_t sl2x2 = f2_pack(sl2, sl2);
-            const uint64_t negm2 = f2_pack(-m_sub, -m_sub);
-            uint64_t acc_e[2] = {0ull, 0ull};
-            auto exp_half = [&](auto masked_tag, int h) {
-                constexpr bool kMasked = decltype(masked_tag)::value;
-                uint32_t pk[32];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const int c = h * 64 + 2 * i;
-                    const uint64_t t = f2_fma(f2_pack(s[c], s[c + 1]), sl2x2, negm2);
-                    uint64_t e;
-                    if (!kMasked && (i % 8) < kExpFmaPairsPer8) {
-                        e = exp2_fma_x2(t);
-                    } else {
-                        float t0, t1;
-                        f2_unpack(t, t0, t1);
-                        e = f2_pack(ex2_approx(t0), ex2_approx(t1));
-                    }
-                    float e0, e1;
-                    f2_unpack(e, e0, e1);
-                    pk[i] = pack_bf16x2(e0, e1);
-                    acc_e[i & 1] = f2_add(acc_e[i & 1], e);
-                }
-                tmem_st_32x32b_x32(tS + h * 32, pk);
-                tmem_wait_st();
-                tc_fence_before_sync();
-                __syncwarp();   // every lane's P is in TMEM: one arrival for the warp
-                if (lane == 0) mbar_arrive(h == 0 ? bar_p_half(buf) : bar_p_full(buf));
+                for (int i = 0; i < 16; ++i)
+                    ob[i] = pack_bf16x2(__uint_as_float(orr[2 * i]) * inv_l, __uint_as_float(orr[2 * i + 1]) * inv_l);
             };
-            if (masked) {
-                exp_half(std::true_type{}, 0);
-                exp_half(std::true_type{}, 1);
-            } else {
-                exp_half(std::false_type{}, 0);
-                exp_half(std::false_type{}, 1);
-            }
-            // P reaches the MMA rounded to bf16.  O is normalised by the sum with the
-            // tile's largest P taken as rounded (its exponential is recomputed
-            // exactly as in the loop above): a key that dominates a row then has
-            // its rounding cancel in O / l, which is where rounding P costs most.
-            // The LSE takes the unrounded sum.
-            float d_round = 0.0f;
-            if (tmax != -INFINITY) {
-                const float pm = ex2_approx(fmaf(tmax, sl2, -m_sub));
-                d_round = __uint_as_float(pack_bf16x2(pm, 0.0f) << 16) - pm;
-            }
-            float b0, b1;
-            f2_unpack(f2_add(acc_e[0], acc_e[1]), b0, b1);
-            l_run += (b0 + b1) + d_round;
-            l_exact += b0 + b1;
-        }
-
-        // ---- epilogue: O / l -> bf16 into this Q tile's shared memory (no MMA reads
-        // it any more: the last QK^T precedes the last P.V, which o_done follows),
-        // in the TMA box layout with the 128-byte swizzle, then one TMA store per 64
-        // columns (positions past Lq are clipped by TMA); LSE per row ----
-        bool have_o = ok && n_kt > 0;
-        if (have_o) {
-            have_o = mbar_wait(bar_o_done(q), 0, abort_flag, &g_attn_err, kDevErrTimeout);
-            tc_fence_after_sync();
-        }
-        const float inv_l = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
-        uint8_t* stile = smem + L::kQOff + q * L::kQTileBytes;
+            if constexpr (kPersistent) {
+                // One 64-column staging block per warpgroup: the next unit's Q may
+                // already be landing in the Q tiles.
+                uint8_t* stg = smem + L::kStgOff + q * L::kBlockBytes;
 #pragma unroll 1
-        for (int c = 0; c < D; c += 32) {
-            uint32_t orr[32];
-            if (have_o) {
-                tmem_ld_32x32b_x32(tO + c, orr);
-                tmem_wait_ld();
-                reg_fence<32>(orr);
+                for (int kb = 0; kb < L::kKB; ++kb) {
+                    uint32_t ob[32];
+                    o_cols(kb * 64, ob);
+                    o_cols(kb * 64 + 32, ob + 16);
+                    if (r == 0) tma_store_wait_read();   // the previous store from the block has read it
+                    named_bar_sync(wg_bar, 128);
+                    uint8_t* rowp = stg + r * 128;
+#pragma unroll
+                    for (int i = 0; i < 8; ++i)
+                        *reinterpret_cast<uint4*>(rowp + ((i ^ (r & 7)) << 4)) =
+                            make_uint4(ob[4 * i], ob[4 * i + 1], ob[4 * i + 2], ob[4 * i + 3]);
+                    fence_proxy_async_smem();
+                    named_bar_sync(wg_bar, 128);   // the warpgroup's rows are all staged
+                    if (r == 0) {
+                        tma_store_3d(&tm_o, smem_u32(stg), kb * 64, tile_p0, q_head0);
+                        tma_store_commit();
+                    }
+                }
             } else {
+                // One unit per CTA: the Q tile is free (its last reader, the last
+                // Q K^T, precedes the last P.V, which o_done follows).
+                uint8_t* stile = smem + L::kQOff + q * L::kQTileBytes;
+#pragma unroll 1
+                for (int c = 0; c < D; c += 32) {
+                    uint32_t ob[16];
+                    o_cols(c, ob);
+                    uint8_t* rowp = stile + (c >> 6) * L::kBlockBytes + r * 128;
+                    const int chunk0 = (c & 63) >> 3;   // 16-byte chunk of the 128-byte row: 0 or 4
 #pragma unroll
-                for (int i = 0; i < 32; ++i) orr[i] = 0u;
+                    for (int i = 0; i < 4; ++i)
+                        *reinterpret_cast<uint4*>(rowp + (((chunk0 + i) ^ (r & 7)) << 4)) =
+                            make_uint4(ob[4 * i], ob[4 * i + 1], ob[4 * i + 2], ob[4 * i + 3]);
+                }
+                fence_proxy_async_smem();
+                named_bar_sync(wg_bar, 128);   // the warpgroup's rows are all staged
+                if (r == 0) {
+                    for (int kb = 0; kb < L::kKB; ++kb)
+                        tma_store_3d(&tm_o, smem_u32(stile) + kb * L::kBlockBytes, kb * 64, tile_p0, q_head0);
+                    tma_store_commit();
+                }
             }
-            uint32_t ob[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i)
-                ob[i] = pack_bf16x2(__uint_as_float(orr[2 * i]) * inv_l, __uint_as_float(orr[2 * i + 1]) * inv_l);
-            uint8_t* rowp = stile + (c >> 6) * L::kBlockBytes + r * 128;
-            const int chunk0 = (c & 63) >> 3;   // 16-byte chunk of the 128-byte row: 0 or 4
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-                *reinterpret_cast<uint4*>(rowp + (((chunk0 + i) ^ (r & 7)) << 4)) =
-                    make_uint4(ob[4 * i], ob[4 * i + 1], ob[4 * i + 2], ob[4 * i + 3]);
+            if (row_valid && p.lse != nullptr) {
+                const float lse = (l_exact > 0.0f) ? (m_run + __log2f(l_exact)) * kLn2 : -INFINITY;
+                p.lse[(static_cast<size_t>(u.b) * p.Hq + h) * p.Lq + pos] = lse;
+            }
+            tiles += n_kt;
+            if (n_kt > 0) ++nu;
         }
-        fence_proxy_async_smem();
-        asm volatile("bar.sync %0, 128;" ::"r"(1 + q) : "memory");   // the warpgroup's rows are all staged
-        if (r == 0) {
-            const int q_head0 = b * p.Hq + g * p.G;
-            for (int kb = 0; kb < L::kKB; ++kb)
-                tma_store_3d(&tm_o, smem_u32(stile) + kb * L::kBlockBytes, kb * 64, p_begin + q * P, q_head0);
-            tma_store_commit();
-            tma_store_wait_read();   // the shared memory may be released after this
-        }
-        if (row_valid && p.lse != nullptr) {
-            const float lse = (l_exact > 0.0f) ? (m_run + __log2f(l_exact)) * kLn2 : -INFINITY;
-            p.lse[(static_cast<size_t>(b) * p.Hq + h) * p.Lq + pos] = lse;
-        }
+        if (r == 0) tma_store_wait_all();   // shared memory stays until the stores are done with it
     }
 
     // ---- teardown ----
