@@ -84,6 +84,13 @@ typedef enum {
  * Hkv < 1, Hq % Hkv != 0, non-finite or non-positive scale, or a base
  * address not 16-byte aligned; ATTN_ERR_UNSUPPORTED for D outside {64, 128, 256}
  * or G > 128; ATTN_ERR_CUDA when a launch fails.
+ *
+ * Concurrency: for D = 64 and 128 the kernel is persistent and hands out its
+ * work from a counter in the library's device memory; each launch takes the
+ * next of 256 counters in turn.  Launches on one stream may follow each other
+ * without limit; at most 256 launches may be in flight at the same time
+ * across streams, and a CUDA graph that holds this call must not be replayed
+ * on two streams at once.
  */
 int attn_prefill(const void* q, const void* k, const void* v, void* out, float* lse,
                  int B, int Hq, int Hkv, int Lq, int Lk, int D, float scale, int is_causal,

@@ -120,6 +120,41 @@ def test_deterministic(oracle_mod):
     assert torch.equal(a, b) and torch.equal(la, lb)
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_persistent_counters_reused_and_concurrent(oracle_mod, D):
+    """For D <= 128 one CTA per SM takes work units from a per-launch counter
+    (256 counters in turn, each put back to zero by its launch's last CTA).
+    With 168 units (more than the SMs, so CTAs take several), 600 launches in a
+    row use every counter twice or more, then two streams run launches on
+    different inputs at the same time: every result must equal the first one,
+    which matches the oracle."""
+    B, Hq, Hkv, L = 2, 16, 4, 1300
+    ins = [tuple(t.cuda() for t in W.prefill_inputs(B, Hq, Hkv, L, L, D, seed=40 + i)) for i in range(2)]
+    scale = 1.0 / math.sqrt(D)
+    first = [prefill(*x, scale=scale) for x in ins]
+    torch.cuda.synchronize()
+    q, k, v = (t.cpu() for t in ins[0])
+    ref_o, ref_l = oracle_mod.attention_prefill(q, k, v, scale, True)
+    assert_close(first[0][0], first[0][1], ref_o, ref_l, f"persistent D{D}")
+    out = torch.empty_like(ins[0][0])
+    for _ in range(600):
+        prefill(*ins[0], scale=scale, out=out, want_lse=False)
+    torch.cuda.synchronize()
+    assert torch.equal(out, first[0][0])
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = [torch.empty_like(x[0]) for x in ins]
+    bad = 0
+    for _ in range(20):
+        for i in range(2):
+            with torch.cuda.stream(streams[i]):
+                prefill(*ins[i], scale=scale, out=outs[i], want_lse=False, stream=streams[i])
+        for i in range(2):
+            streams[i].synchronize()
+            bad += int(not torch.equal(outs[i], first[i][0]))
+    assert bad == 0
+    assert device_error(reset=True) == 0
+
+
 def _sample_rows(Lq, extra=()):
     rows = {0, 1, 2, Lq - 1, Lq - 2, Lq // 2}
     for e in (31, 32, 33, 63, 64, 65, 127, 128, 129, 255, 256, 257):
