@@ -385,8 +385,11 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
             int tb = 0;      // ring entries of earlier units
             int tiles = 0;   // key tiles of earlier units (phases of the per-tile barriers)
             int nu = 0;      // earlier units with key tiles
-            auto slot_of = [&](int t) { return (tb + t) % L::kStages; };
-            auto par_of = [&](int t) { return static_cast<uint32_t>((tb + t) / L::kStages) & 1u; };
+            // Ring positions in unsigned arithmetic: this thread's instruction latency
+            // sits on the S -> P -> MMA chain, and signed % and / with a runtime base
+            // cost about 60 cycles per key tile (measured).
+            auto slot_of = [&](int t) { return static_cast<int>(static_cast<unsigned>(tb + t) % L::kStages); };
+            auto par_of = [&](int t) { return (static_cast<unsigned>(tb + t) / L::kStages) & 1u; };
             // Shared-memory descriptors are built once; a k-step only moves the
             // start-address field (bits 0-13, address >> 4), so each MMA issue
             // costs one 64-bit add.
