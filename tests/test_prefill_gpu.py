@@ -155,6 +155,17 @@ def test_persistent_counters_reused_and_concurrent(oracle_mod, D):
     assert device_error(reset=True) == 0
 
 
+@pytest.mark.parametrize("D,Hq,Hkv,causal", [(128, 12, 4, True), (64, 24, 4, True), (128, 12, 4, False),
+                                              (128, 40, 8, True)])
+def test_persistent_many_units_ragged_groups(oracle_mod, D, Hq, Hkv, causal):
+    """G = 3, 6, 5 (the Q tile has padding rows and its TMA box is G x P rows)
+    with several hundred work units, so each persistent CTA runs many units in a
+    row through the same Q tiles and staging block; sampled rows across tiles."""
+    B, L = 4, 2000
+    rows = sorted({0, 1, 41, 42, 43, 83, 84, 85, 127, 128, 255, 256, 1000, 1023, 1024, 1998, 1999})
+    _run(oracle_mod, B, Hq, Hkv, L, L, D, causal, seed=Hq + D, spike=97, rows=rows)
+
+
 def _sample_rows(Lq, extra=()):
     rows = {0, 1, 2, Lq - 1, Lq - 2, Lq // 2}
     for e in (31, 32, 33, 63, 64, 65, 127, 128, 129, 255, 256, 257):
