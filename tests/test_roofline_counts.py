@@ -1,6 +1,5 @@
 """The work counts used for the roofline, checked against closed forms and the
 figures the SDPA / FlashAttention selection guide prints for Qwen3-8B."""
-import math
 
 import pytest
 
