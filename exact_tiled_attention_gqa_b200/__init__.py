@@ -59,6 +59,54 @@ def _check_tensor(name: str, t: torch.Tensor, dtype: torch.dtype, ndim: int) -> 
         raise ValueError(f"{name} must be contiguous")
 
 
+def _check_on(device: torch.device, **tensors) -> None:
+    """Every given tensor (None skipped) lives on `device`."""
+    for name, t in tensors.items():
+        if t is not None and t.device != device:
+            raise ValueError(f"{name} is on {t.device}, but q is on {device}")
+
+
+def _result(name: str, t: Optional[torch.Tensor], dtype: torch.dtype, shape, device: torch.device,
+            want: bool = True) -> Optional[torch.Tensor]:
+    """A caller's output tensor, checked against the shape the call writes, or a new one.
+
+    The library writes exactly `shape` elements through the pointer, so a
+    smaller or differently laid out buffer is refused here rather than
+    overrun on the device."""
+    shape = tuple(int(x) for x in shape)
+    if t is None:
+        return torch.empty(shape, dtype=dtype, device=device) if want else None
+    _check_tensor(name, t, dtype, len(shape))
+    if tuple(t.shape) != shape:
+        raise ValueError(f"{name} must have shape {shape}, got {tuple(t.shape)}")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, but q is on {device}")
+    return t
+
+
+def _workspace(ws: Optional[torch.Tensor], need: int, device: torch.device):
+    """(pointer, size in bytes) of a caller's workspace, or of a new one of `need` bytes."""
+    if ws is None:
+        ws = torch.empty(max(need, 1), dtype=torch.uint8, device=device)
+    if not isinstance(ws, torch.Tensor) or not ws.is_contiguous() or ws.device != device:
+        raise ValueError(f"workspace must be a contiguous tensor on {device}")
+    return ws, ws.numel() * ws.element_size()
+
+
+def _squeezed_results(out, lse, q4: torch.Tensor, want_lse: bool, squeezed: bool):
+    """out / lse for a call whose q was given as [B,Hq,D] and viewed as [B,Hq,1,D]:
+    results the caller passed in that 3-d / 2-d form are viewed the same way."""
+    B, Hq, Lq, D = q4.shape
+    if squeezed:
+        if out is not None:
+            out = _result("out", out, torch.bfloat16, (B, Hq, D), q4.device).unsqueeze(2)
+        if lse is not None:
+            lse = _result("lse", lse, torch.float32, (B, Hq), q4.device).unsqueeze(2)
+    out = _result("out", out, torch.bfloat16, q4.shape, q4.device)
+    lse = _result("lse", lse, torch.float32, (B, Hq, Lq), q4.device, want_lse)
+    return out, lse
+
+
 def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: Optional[float] = None,
             is_causal: bool = True, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
             want_lse: bool = True, stream=None):
@@ -69,16 +117,11 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: Optiona
     Hkv, Lk = k.shape[1], k.shape[2]
     if k.shape[0] != B or k.shape[3] != D or v.shape != k.shape:
         raise ValueError(f"shape mismatch: q {tuple(q.shape)} k {tuple(k.shape)} v {tuple(v.shape)}")
+    _check_on(q.device, k=k, v=v)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
-    if out is None:
-        out = torch.empty_like(q)
-    else:
-        _check_tensor("out", out, torch.bfloat16, 4)
-    if lse is None and want_lse:
-        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
-    elif lse is not None:
-        _check_tensor("lse", lse, torch.float32, 3)
+    out = _result("out", out, torch.bfloat16, q.shape, q.device)
+    lse = _result("lse", lse, torch.float32, (B, Hq, Lq), q.device, want_lse)
     with torch.cuda.device(q.device):
         st = _native.lib().attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Lq, Lk, D,
                                         float(scale), int(bool(is_causal)), _stream_handle(stream))
@@ -111,15 +154,14 @@ def prefill_host(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: Op
         out = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=True)
     if lse is None and want_lse:
         lse = torch.empty((B, Hq, Lq), dtype=torch.float32, pin_memory=True)
-    for name, t in (("out", out), ("lse", lse)):
-        if t is not None and (t.is_cuda or not t.is_contiguous()):
-            raise ValueError(f"{name} must be a contiguous CPU tensor")
+    for name, t, dt, shp in (("out", out, torch.bfloat16, tuple(q.shape)), ("lse", lse, torch.float32, (B, Hq, Lq))):
+        if t is not None and (t.is_cuda or not t.is_contiguous() or t.dtype != dt or tuple(t.shape) != shp):
+            raise ValueError(f"{name} must be a contiguous {dt} CPU tensor of shape {shp}")
     need = prefill_host_scratch_size(B, Hq, Hkv, Lq, Lk, D)
-    if scratch is None:
-        scratch = torch.empty(max(need, 1), dtype=torch.uint8, device=device)
+    scratch, scratch_bytes = _workspace(scratch, need, device)
     with torch.cuda.device(device):
         st = _native.lib().attn_prefill_host(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Lq, Lk,
-                                             D, float(scale), int(bool(is_causal)), _ptr(scratch), scratch.numel(),
+                                             D, float(scale), int(bool(is_causal)), _ptr(scratch), scratch_bytes,
                                              _stream_handle(stream))
     _native.check(st, "attn_prefill_host")
     return out, lse
@@ -141,27 +183,26 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, seqlen
     Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
     if k_cache.shape[0] != B or k_cache.shape[3] != D or v_cache.shape != k_cache.shape or seqlens.shape[0] != B:
         raise ValueError("shape mismatch between q, the caches and seqlens")
+    _check_on(q.device, k_cache=k_cache, v_cache=v_cache, seqlens=seqlens)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
-    if out is None:
-        out = torch.empty_like(q)
-    if lse is None and want_lse:
-        lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
-    need = decode_workspace_size(B, Hq, Hkv, Lmax, D)
-    if workspace is None:
-        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    out = _result("out", out, torch.bfloat16, q.shape, q.device)
+    lse = _result("lse", lse, torch.float32, (B, Hq), q.device, want_lse)
+    workspace, ws_bytes = _workspace(workspace, decode_workspace_size(B, Hq, Hkv, Lmax, D), q.device)
     with torch.cuda.device(q.device):
         st = _native.lib().attn_decode(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(out), _ptr(lse),
-                                       B, Hq, Hkv, Lmax, D, float(scale), _ptr(workspace), workspace.numel(),
+                                       B, Hq, Hkv, Lmax, D, float(scale), _ptr(workspace), ws_bytes,
                                        _stream_handle(stream))
     _native.check(st, "attn_decode")
     return out, lse
 
 
 def decode_partial(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, seqlens: torch.Tensor, *,
-                   scale: Optional[float] = None, workspace: Optional[torch.Tensor] = None, stream=None):
+                   scale: Optional[float] = None, o_part: Optional[torch.Tensor] = None,
+                   lse_part: Optional[torch.Tensor] = None, workspace: Optional[torch.Tensor] = None, stream=None):
     """decode over the cache rows this device holds, results unrounded for decode_merge:
-    (o_part fp32 [B,Hq,D], lse_part fp32 [B,Hq], natural log, -inf where a sequence has no rows here)."""
+    (o_part fp32 [B,Hq,D], lse_part fp32 [B,Hq], natural log, -inf where a sequence has no rows here).
+    o_part / lse_part may be given (e.g. slices of an exchange buffer) and are then written in place."""
     _check_tensor("q", q, torch.bfloat16, 3)
     _check_tensor("k_cache", k_cache, torch.bfloat16, 4)
     _check_tensor("v_cache", v_cache, torch.bfloat16, 4)
@@ -170,17 +211,16 @@ def decode_partial(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
     Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
     if k_cache.shape[0] != B or k_cache.shape[3] != D or v_cache.shape != k_cache.shape or seqlens.shape[0] != B:
         raise ValueError("shape mismatch between q, the caches and seqlens")
+    _check_on(q.device, k_cache=k_cache, v_cache=v_cache, seqlens=seqlens)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
-    o_part = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
-    lse_part = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
-    need = decode_workspace_size(B, Hq, Hkv, Lmax, D)
-    if workspace is None:
-        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    o_part = _result("o_part", o_part, torch.float32, (B, Hq, D), q.device)
+    lse_part = _result("lse_part", lse_part, torch.float32, (B, Hq), q.device)
+    workspace, ws_bytes = _workspace(workspace, decode_workspace_size(B, Hq, Hkv, Lmax, D), q.device)
     with torch.cuda.device(q.device):
         st = _native.lib().attn_decode_partial(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(o_part),
                                                _ptr(lse_part), B, Hq, Hkv, Lmax, D, float(scale), _ptr(workspace),
-                                               workspace.numel(), _stream_handle(stream))
+                                               ws_bytes, _stream_handle(stream))
     _native.check(st, "attn_decode_partial")
     return o_part, lse_part
 
@@ -195,10 +235,9 @@ def decode_merge(o_parts: torch.Tensor, lse_parts: torch.Tensor, *, out: Optiona
     if tuple(lse_parts.shape) != tuple(o_parts.shape[:-1]) or o_parts.dim() < 3:
         raise ValueError("o_parts must be [n, ..., D] and lse_parts [n, ...]")
     rows = lse_parts[0].numel()
-    if out is None:
-        out = torch.empty(o_parts.shape[1:], dtype=torch.bfloat16, device=o_parts.device)
-    if lse is None and want_lse:
-        lse = torch.empty(lse_parts.shape[1:], dtype=torch.float32, device=o_parts.device)
+    _check_on(o_parts.device, lse_parts=lse_parts)
+    out = _result("out", out, torch.bfloat16, o_parts.shape[1:], o_parts.device)
+    lse = _result("lse", lse, torch.float32, lse_parts.shape[1:], o_parts.device, want_lse)
     with torch.cuda.device(o_parts.device):
         st = _native.lib().attn_decode_merge(_ptr(o_parts), _ptr(lse_parts), n, rows, D, _ptr(out), _ptr(lse),
                                              _stream_handle(stream))
@@ -223,19 +262,16 @@ def decode_mq(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, seq
     Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
     if k_cache.shape[0] != B or k_cache.shape[3] != D or v_cache.shape != k_cache.shape or seqlens.shape[0] != B:
         raise ValueError("shape mismatch between q, the caches and seqlens")
+    _check_on(q.device, k_cache=k_cache, v_cache=v_cache, seqlens=seqlens)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
-    if out is None:
-        out = torch.empty_like(q)
-    if lse is None and want_lse:
-        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
-    need = decode_mq_workspace_size(B, Hq, Hkv, Lq, Lmax, D)
-    if workspace is None:
-        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    out = _result("out", out, torch.bfloat16, q.shape, q.device)
+    lse = _result("lse", lse, torch.float32, (B, Hq, Lq), q.device, want_lse)
+    workspace, ws_bytes = _workspace(workspace, decode_mq_workspace_size(B, Hq, Hkv, Lq, Lmax, D), q.device)
     with torch.cuda.device(q.device):
         st = _native.lib().attn_decode_mq(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(out),
                                           _ptr(lse), B, Hq, Hkv, Lq, Lmax, D, float(scale), _ptr(workspace),
-                                          workspace.numel(), _stream_handle(stream))
+                                          ws_bytes, _stream_handle(stream))
     _native.check(st, "attn_decode_mq")
     return out, lse
 
@@ -273,23 +309,19 @@ def decode_kv8(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, k_
     want_scale = (Hkv,) if fmt == _native.ATTN_KV_E4M3 else (B, Hkv, Lmax, D // 32)
     if tuple(k_scale.shape) != want_scale or tuple(v_scale.shape) != want_scale:
         raise ValueError(f"k_scale / v_scale must have shape {want_scale}")
+    _check_on(q.device, k_cache=k_cache, v_cache=v_cache, k_scale=k_scale, v_scale=v_scale, seqlens=seqlens)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
-    if out is None:
-        out = torch.empty_like(q)
-    if lse is None and want_lse:
-        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
-    need = decode_kv8_workspace_size(B, Hq, Hkv, Lq, Lmax, D)
-    if workspace is None:
-        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    out, lse = _squeezed_results(out, lse, q, want_lse, squeeze)
+    workspace, ws_bytes = _workspace(workspace, decode_kv8_workspace_size(B, Hq, Hkv, Lq, Lmax, D), q.device)
     with torch.cuda.device(q.device):
         st = _native.lib().attn_decode_kv8(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(k_scale), _ptr(v_scale), fmt,
                                            _ptr(seqlens), _ptr(out), _ptr(lse), B, Hq, Hkv, Lq, Lmax, D,
-                                           float(scale), _ptr(workspace), workspace.numel(), _stream_handle(stream))
+                                           float(scale), _ptr(workspace), ws_bytes, _stream_handle(stream))
     _native.check(st, "attn_decode_kv8")
     if squeeze:
-        out = out.squeeze(2) if out.dim() == 4 else out
-        lse = None if lse is None else (lse.squeeze(2) if lse.dim() == 3 else lse)
+        out = out.squeeze(2)
+        lse = None if lse is None else lse.squeeze(2)
     return out, lse
 
 
@@ -326,24 +358,22 @@ def decode_kv8_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tens
     want_scale = (Hkv,) if fmt == _native.ATTN_KV_E4M3 else (n_pages, Hkv, page_size, D // 32)
     if tuple(k_scale.shape) != want_scale or tuple(v_scale.shape) != want_scale:
         raise ValueError(f"k_scale / v_scale must have shape {want_scale}")
+    _check_on(q.device, k_pages=k_pages, v_pages=v_pages, k_scale=k_scale, v_scale=v_scale, block_table=block_table,
+              seqlens=seqlens)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
-    if out is None:
-        out = torch.empty_like(q)
-    if lse is None and want_lse:
-        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    out, lse = _squeezed_results(out, lse, q, want_lse, squeeze)
     need = int(_native.lib().attn_decode_kv8_paged_workspace_size(B, Hq, Hkv, Lq, page_size, max_pages, D))
-    if workspace is None:
-        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    workspace, ws_bytes = _workspace(workspace, need, q.device)
     with torch.cuda.device(q.device):
         st = _native.lib().attn_decode_kv8_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(k_scale), _ptr(v_scale),
                                                  fmt, _ptr(block_table), _ptr(seqlens), _ptr(out), _ptr(lse), B, Hq,
                                                  Hkv, Lq, n_pages, page_size, max_pages, D, float(scale),
-                                                 _ptr(workspace), workspace.numel(), _stream_handle(stream))
+                                                 _ptr(workspace), ws_bytes, _stream_handle(stream))
     _native.check(st, "attn_decode_kv8_paged")
     if squeeze:
-        out = out.squeeze(2) if out.dim() == 4 else out
-        lse = None if lse is None else (lse.squeeze(2) if lse.dim() == 3 else lse)
+        out = out.squeeze(2)
+        lse = None if lse is None else lse.squeeze(2)
     return out, lse
 
 
@@ -367,24 +397,21 @@ def decode_paged(q: torch.Tensor, k_pages: torch.Tensor, v_pages: torch.Tensor, 
     if (k_pages.shape[3] != D or v_pages.shape != k_pages.shape or block_table.shape[0] != B
             or seqlens.shape[0] != B):
         raise ValueError("shape mismatch between q, the page pools, block_table and seqlens")
+    _check_on(q.device, k_pages=k_pages, v_pages=v_pages, block_table=block_table, seqlens=seqlens)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
-    if out is None:
-        out = torch.empty_like(q)
-    if lse is None and want_lse:
-        lse = torch.empty((B, Hq, Lq), dtype=torch.float32, device=q.device)
+    out, lse = _squeezed_results(out, lse, q, want_lse, squeeze)
     need = int(_native.lib().attn_decode_paged_workspace_size(B, Hq, Hkv, Lq, page_size, max_pages, D))
-    if workspace is None:
-        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=q.device)
+    workspace, ws_bytes = _workspace(workspace, need, q.device)
     with torch.cuda.device(q.device):
         st = _native.lib().attn_decode_paged(_ptr(q), _ptr(k_pages), _ptr(v_pages), _ptr(block_table),
                                              _ptr(seqlens), _ptr(out), _ptr(lse), B, Hq, Hkv, Lq, n_pages, page_size,
-                                             max_pages, D, float(scale), _ptr(workspace), workspace.numel(),
+                                             max_pages, D, float(scale), _ptr(workspace), ws_bytes,
                                              _stream_handle(stream))
     _native.check(st, "attn_decode_paged")
     if squeeze:
-        out = out.squeeze(2) if out.dim() == 4 else out
-        lse = None if lse is None else (lse.squeeze(2) if lse.dim() == 3 else lse)
+        out = out.squeeze(2)
+        lse = None if lse is None else lse.squeeze(2)
     return out, lse
 
 
@@ -394,13 +421,18 @@ def decode_noalloc(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor
     library's own fixed scratch (16 MiB per GPU), and `out` (and `lse`, if
     wanted) must be passed in.  Calls on one GPU must not overlap in time."""
     for n, t, dt, nd in (("q", q, torch.bfloat16, 3), ("k_cache", k_cache, torch.bfloat16, 4),
-                         ("v_cache", v_cache, torch.bfloat16, 4), ("seqlens", seqlens, torch.int32, 1),
-                         ("out", out, torch.bfloat16, 3)):
+                         ("v_cache", v_cache, torch.bfloat16, 4), ("seqlens", seqlens, torch.int32, 1)):
         _check_tensor(n, t, dt, nd)
-    if lse is not None:
-        _check_tensor("lse", lse, torch.float32, 2)
     B, Hq, D = q.shape
     Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
+    if k_cache.shape[0] != B or k_cache.shape[3] != D or v_cache.shape != k_cache.shape or seqlens.shape[0] != B:
+        raise ValueError("shape mismatch between q, the caches and seqlens")
+    _check_on(q.device, k_cache=k_cache, v_cache=v_cache, seqlens=seqlens)
+    if out is None:
+        raise ValueError("out must be given: decode_noalloc allocates nothing")
+    _result("out", out, torch.bfloat16, q.shape, q.device)
+    if lse is not None:
+        _result("lse", lse, torch.float32, (B, Hq), q.device)
     if scale is None:
         scale = 1.0 / math.sqrt(D)
     with torch.cuda.device(q.device):

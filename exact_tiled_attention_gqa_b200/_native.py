@@ -21,6 +21,7 @@ ATTN_ERR_CUDA = -4
 ATTN_DEVERR_TIMEOUT = 0x1
 ATTN_DEVERR_SEQLEN = 0x2
 ATTN_DEVERR_PAGE = 0x4
+ATTN_DEVERR_SCHED = 0x8
 ATTN_DECODE_NOALLOC_SCRATCH_BYTES = 16 << 20
 ATTN_KV_E4M3 = 1
 ATTN_KV_Q8_0 = 2
@@ -51,6 +52,8 @@ SIGNATURES = {
                                      _i32, _i32, _i32, _f32, _vp, _sz, _vp]),
     "attn_selftest_kv8_convert": (_i32, [_vp, _vp, _i32, _i32, _vp]),
     "attn_selftest_exp2": (_i32, [_vp, _vp, _i32, _vp]),
+    "attn_selftest_wait": (_i32, [ctypes.c_ulonglong, _vp, _vp]),
+    "attn_prefill_sched_busy": (_i32, [ctypes.POINTER(_i32)]),
     "attn_status_string": (ctypes.c_char_p, [_i32]),
     "attn_last_error": (ctypes.c_char_p, []),
     "attn_device_error": (_i32, [ctypes.POINTER(ctypes.c_uint), _i32]),

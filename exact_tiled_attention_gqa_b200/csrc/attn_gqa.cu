@@ -120,11 +120,14 @@ int ensure_smem(Kernel kernel, int bytes, int* done_mask_per_device) {
 }
 
 // SMs of the current device, and this launch's scheduling counters for a
-// persistent prefill (slots are taken in turn, see g_prefill_sched).
-int device_sms_and_sched(int* n_sm, int** sched) {
+// persistent prefill.  Ordinary launches take the eager slots in turn; a launch
+// being recorded into a CUDA graph (a stream capture) takes the next capture
+// slot instead, which the graph then uses on every replay (see g_prefill_sched).
+int device_sms_and_sched(cudaStream_t stream, int* n_sm, int** sched) {
     static int sms[64];
     static int* sched_base[64];
-    static std::atomic<unsigned> ticket{0};
+    static std::atomic<unsigned> eager_ticket{0};
+    static std::atomic<unsigned> capture_ticket{0};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
@@ -141,8 +144,16 @@ int device_sms_and_sched(int* n_sm, int** sched) {
         __atomic_store_n(&sched_base[dev], b, __ATOMIC_RELEASE);
         __atomic_store_n(&sms[dev], n, __ATOMIC_RELEASE);
     }
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    e = cudaStreamIsCapturing(stream, &cap);
+    if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "cudaStreamIsCapturing: %s", cudaGetErrorString(e));
+    unsigned slot;
+    if (cap == cudaStreamCaptureStatusActive)
+        slot = kPrefillEagerSlots + capture_ticket.fetch_add(1, std::memory_order_relaxed) % kPrefillCaptureSlots;
+    else
+        slot = eager_ticket.fetch_add(1, std::memory_order_relaxed) % kPrefillEagerSlots;
     *n_sm = n;
-    *sched = b + 2 * (ticket.fetch_add(1, std::memory_order_relaxed) % kPrefillSchedSlots);
+    *sched = b + 2 * slot;
     return ATTN_OK;
 }
 
@@ -208,7 +219,7 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
     long long grid = units;
     if (L::kPersistent) {   // one CTA per SM, each taking units until they run out
         int n_sm = 0;
-        if ((st = device_sms_and_sched(&n_sm, &prm.sched)) != ATTN_OK) return st;
+        if ((st = device_sms_and_sched(stream, &n_sm, &prm.sched)) != ATTN_OK) return st;
         grid = std::min<long long>(units, n_sm);
     }
     attn_prefill_sm100_kernel<D, NQ>
@@ -630,10 +641,19 @@ extern "C" size_t attn_decode_workspace_size(int B, int Hq, int Hkv, int Lmax, i
     return decode_layout(B, Hq, Hkv, Lmax, D).total;
 }
 
+namespace attn {
 namespace {
+void* decode_scratch_address(int* status);
+}  // namespace
+}  // namespace attn
+
+namespace {
+// Argument checks and launch shared by attn_decode, attn_decode_partial and
+// attn_decode_noalloc.  With noalloc the workspace arguments are ignored and the
+// split partials go to the library's static scratch array, if they fit.
 int decode_checked(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens, void* out,
                    float* lse, int B, int Hq, int Hkv, int Lmax, int D, float scale, void* workspace,
-                   size_t workspace_bytes, void* stream, bool f32_out) {
+                   size_t workspace_bytes, void* stream, bool f32_out, bool noalloc = false) {
     int st = check_common(q, k_cache, v_cache, out, lse, B, Hq, Hkv, Lmax, Lmax, D, scale, "Lmax", "Lmax");
     if (st != ATTN_OK) return st;
     if (!seqlens && B > 0) return fail(ATTN_ERR_INVALID_ARG, "null seqlens");
@@ -643,11 +663,21 @@ int decode_checked(const void* q, const void* k_cache, const void* v_cache, cons
     if (static_cast<long long>(B) * Hq > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "B*Hq too large");
     if (B == 0) return ok();
     const size_t need = decode_layout(B, Hq, Hkv, Lmax, D).total;
-    if (!workspace || workspace_bytes < need)
-        return fail(ATTN_ERR_WORKSPACE, "decode workspace needs %zu bytes, got %zu", need,
-                    workspace ? workspace_bytes : static_cast<size_t>(0));
-    if (reinterpret_cast<uintptr_t>(workspace) & 255u)
-        return fail(ATTN_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    if (noalloc) {
+        if (need > ATTN_DECODE_NOALLOC_SCRATCH_BYTES)
+            return fail(ATTN_ERR_WORKSPACE,
+                        "attn_decode_noalloc: these sizes need %zu bytes of split partials; the static scratch "
+                        "holds %u (use attn_decode with a caller workspace)",
+                        need, ATTN_DECODE_NOALLOC_SCRATCH_BYTES);
+        workspace = decode_scratch_address(&st);
+        if (st != ATTN_OK) return st;
+    } else {
+        if (!workspace || workspace_bytes < need)
+            return fail(ATTN_ERR_WORKSPACE, "decode workspace needs %zu bytes, got %zu", need,
+                        workspace ? workspace_bytes : static_cast<size_t>(0));
+        if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+            return fail(ATTN_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    }
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     const PagedKV none;
     st = (D == 256)   ? launch_decode<256>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, workspace, s,
@@ -718,6 +748,69 @@ extern "C" int attn_selftest_exp2(const float* x, float* y, int n, void* stream)
     exp2_fma_selftest_kernel<<<(pairs + threads - 1) / threads, threads, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
     const int st = check_launch("exp2_fma_selftest_kernel");
     return st == ATTN_OK ? ok() : st;
+}
+
+namespace attn {
+namespace {
+// The pipelines' bounded wait, made to run out: warp 0 plays a producer that
+// announces 16 bytes on `full` that never arrive (no copy is issued), then waits
+// for the consumer to free the entry (`empty`) with the kernels' 2 s limit;
+// warp 1 plays the consumer and waits on `full` with `limit_ns`.  The consumer's
+// wait gives up, records the timeout and raises the abort flag; the producer's
+// wait then ends through the flag, long before its own limit.  No asynchronous
+// copy is in flight at any point.
+__global__ void wait_selftest_kernel(unsigned long long limit_ns, int* result) {
+    __shared__ __align__(8) uint64_t bars[2];
+    __shared__ int abort_word;
+    volatile int* abort_flag = &abort_word;
+    const uint32_t full = smem_u32(&bars[0]), empty = smem_u32(&bars[1]);
+    if (threadIdx.x == 0) {
+        mbar_init(full, 1);
+        mbar_init(empty, 1);
+        *abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if ((threadIdx.x & 31) != 0) return;
+    const uint64_t t0 = global_timer_ns();
+    bool ok;
+    if (threadIdx.x == 0) {
+        mbar_arrive_expect_tx(full, 16);
+        ok = mbar_wait(empty, 0, abort_flag, &g_attn_err, kDevErrTimeout);
+    } else {
+        ok = mbar_wait(full, 0, abort_flag, &g_attn_err, kDevErrTimeout, limit_ns);
+    }
+    const int role = threadIdx.x >> 5;
+    result[2 * role] = ok ? 1 : 0;
+    const uint64_t us = (global_timer_ns() - t0) / 1000u;
+    result[2 * role + 1] = us > 0x7fffffffull ? 0x7fffffff : static_cast<int>(us);
+}
+}  // namespace
+}  // namespace attn
+
+extern "C" int attn_selftest_wait(unsigned long long limit_ns, int* result, void* stream) {
+    if (!result || (reinterpret_cast<uintptr_t>(result) & 3u))
+        return fail(ATTN_ERR_INVALID_ARG, "result must be a 4-byte aligned device array of 4 ints");
+    if (limit_ns == 0 || limit_ns > kWaitLimitNs)
+        return fail(ATTN_ERR_INVALID_ARG, "limit_ns must be in (0, %llu]", static_cast<unsigned long long>(kWaitLimitNs));
+    wait_selftest_kernel<<<1, 64, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, result);
+    const int st = check_launch("wait_selftest_kernel");
+    return st == ATTN_OK ? ok() : st;
+}
+
+extern "C" int attn_prefill_sched_busy(int* busy) {
+    if (!busy) return fail(ATTN_ERR_INVALID_ARG, "null busy");
+    cudaError_t e = cudaDeviceSynchronize();
+    if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "cudaDeviceSynchronize: %s", cudaGetErrorString(e));
+    static int host[2 * kPrefillSchedSlots];
+    static std::mutex mu;
+    std::lock_guard<std::mutex> lock(mu);
+    e = cudaMemcpyFromSymbol(host, g_prefill_sched, sizeof host);
+    if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "reading the scheduling counters: %s", cudaGetErrorString(e));
+    int n = 0;
+    for (int i = 0; i < 2 * kPrefillSchedSlots; ++i) n += host[i] != 0;
+    *busy = n;
+    return ok();
 }
 
 extern "C" size_t attn_decode_mq_workspace_size(int B, int Hq, int Hkv, int Lq, int Lmax, int D) {
@@ -878,27 +971,8 @@ void* decode_scratch_address(int* status) {
 extern "C" int attn_decode_noalloc(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,
                                    void* out, float* lse, int B, int Hq, int Hkv, int Lmax, int D, float scale,
                                    void* stream) {
-    int st = check_common(q, k_cache, v_cache, out, lse, B, Hq, Hkv, Lmax, Lmax, D, scale, "Lmax", "Lmax");
-    if (st != ATTN_OK) return st;
-    if (!seqlens && B > 0) return fail(ATTN_ERR_INVALID_ARG, "null seqlens");
-    if (reinterpret_cast<uintptr_t>(seqlens) & 3u) return fail(ATTN_ERR_INVALID_ARG, "seqlens must be 4-byte aligned");
-    if (Lmax < 1) return fail(ATTN_ERR_INVALID_ARG, "Lmax must be >= 1");
-    if (Hq / Hkv > 128) return fail(ATTN_ERR_UNSUPPORTED, "decode group size G=%d > 128", Hq / Hkv);
-    if (static_cast<long long>(B) * Hq > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "B*Hq too large");
-    if (B == 0) return ok();
-    const size_t need = decode_layout(B, Hq, Hkv, Lmax, D).total;
-    if (need > ATTN_DECODE_NOALLOC_SCRATCH_BYTES)
-        return fail(ATTN_ERR_WORKSPACE,
-                    "attn_decode_noalloc: these sizes need %zu bytes of split partials; the static scratch holds %u "
-                    "(use attn_decode with a caller workspace)",
-                    need, ATTN_DECODE_NOALLOC_SCRATCH_BYTES);
-    void* scratch = decode_scratch_address(&st);
-    if (st != ATTN_OK) return st;
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    st = (D == 256)   ? launch_decode<256>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, scratch, s)
-         : (D == 128) ? launch_decode<128>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, scratch, s)
-                      : launch_decode<64>(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, scale, scratch, s);
-    return st == ATTN_OK ? ok() : st;
+    return decode_checked(q, k_cache, v_cache, seqlens, out, lse, B, Hq, Hkv, Lmax, D, scale, nullptr, 0, stream,
+                          false, /*noalloc=*/true);
 }
 
 extern "C" size_t attn_decode_kv8_workspace_size(int B, int Hq, int Hkv, int Lq, int Lmax, int D) {

@@ -10,6 +10,7 @@ namespace attn {
 constexpr unsigned int kDevErrTimeout = 0x1u;   // ATTN_DEVERR_TIMEOUT
 constexpr unsigned int kDevErrSeqlen = 0x2u;    // ATTN_DEVERR_SEQLEN
 constexpr unsigned int kDevErrPage = 0x4u;      // ATTN_DEVERR_PAGE
+constexpr unsigned int kDevErrSched = 0x8u;     // ATTN_DEVERR_SCHED
 
 __device__ unsigned int g_attn_err;
 

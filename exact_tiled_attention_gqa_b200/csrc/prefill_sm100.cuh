@@ -137,10 +137,15 @@ struct PrefillSmem {
 };
 
 // Scheduling counters of persistent launches: slot i is {next unit, CTAs
-// done}.  Each launch takes a slot in turn from the host; the last of its CTAs
-// to finish puts both counters back to zero, so a slot is ready for its next
-// launch without a memset.
-constexpr int kPrefillSchedSlots = 256;
+// done}.  Each launch takes a slot from the host; the last of its CTAs to
+// finish puts both counters back to zero, so a slot is ready for its next
+// launch without a memset.  Ordinary launches take the first
+// kPrefillEagerSlots slots in turn; launches recorded into a CUDA graph take
+// the next kPrefillCaptureSlots in turn (a graph keeps its slot for every
+// replay, so the two kinds never share one).
+constexpr int kPrefillEagerSlots = 256;
+constexpr int kPrefillCaptureSlots = 1024;
+constexpr int kPrefillSchedSlots = kPrefillEagerSlots + kPrefillCaptureSlots;
 __device__ int g_prefill_sched[2 * kPrefillSchedSlots];
 
 struct PrefillParams {
@@ -366,11 +371,18 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
             }
             if constexpr (kPersistent) {
                 // This CTA takes no more units.  The last CTA to get here leaves
-                // both counters at zero for the slot's next launch.
+                // both counters at zero for the slot's next launch.  Every CTA
+                // that ran to the end made one claim per unit it ran after its
+                // first, plus one that came back empty, so a launch that had its
+                // counters to itself ends with exactly n_units claims; any other
+                // count means another launch used the same slot at the same time
+                // (units may have been skipped), which is flagged.
                 __threadfence();
                 if (atomicAdd(p.sched + 1, 1) == static_cast<int>(gridDim.x) - 1) {
-                    atomicExch(p.sched, 0);
+                    const int claims = atomicExch(p.sched, 0);
                     atomicExch(p.sched + 1, 0);
+                    if (ok && claims != p.n_units && !(atomicOr(&g_attn_err, 0u) & kDevErrTimeout))
+                        atomicOr(&g_attn_err, kDevErrSched);   // (a timed-out CTA stops claiming early)
                 }
             }
         }

@@ -62,19 +62,21 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     return done != 0;
 }
 
-// A wait that cannot hang: ~2 s of spinning, or an abort raised by another
-// warp of the CTA, ends it with `false`.
+// A wait that cannot hang: ~2 s of spinning (limit_ns), or an abort raised by
+// another warp of the CTA, ends it with `false`.  A wait that runs out of time
+// raises the abort flag itself, so the CTA's other waits end too.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          unsigned int* err_word, unsigned int err_bit) {
+                                          unsigned int* err_word, unsigned int err_bit,
+                                          uint64_t limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (uint32_t spin = 1;; ++spin) {
         if (mbar_try_wait(bar, parity)) return true;
         if ((spin & 63u) == 0) {
             if (*abort_flag) return false;
-            if (global_timer_ns() - t0 > kWaitLimitNs) {
+            if (global_timer_ns() - t0 > limit_ns) {
                 *abort_flag = 1;
                 atomicOr(err_word, err_bit);
                 return false;

@@ -35,6 +35,12 @@
  *     happen before anything is enqueued, so a failed call has no effect.
  *     attn_last_error() gives a one-line description of the last failure on
  *     the calling thread.
+ *   - Per-device state: on first use of a device the library looks up, and
+ *     then keeps for the life of the process, the addresses of its own device
+ *     arrays, kernel attributes, and (attn_prefill_host) two streams and a few
+ *     events.  All of these belong to the device's primary context, so the
+ *     library must not be called again after that context is destroyed
+ *     (cudaDeviceReset, or a reset of the primary context through the driver).
  */
 #ifndef ATTN_GQA_H
 #define ATTN_GQA_H
@@ -86,11 +92,20 @@ typedef enum {
  * or G > 128; ATTN_ERR_CUDA when a launch fails.
  *
  * Concurrency: for D = 64 and 128 the kernel is persistent and hands out its
- * work from a counter in the library's device memory; each launch takes the
- * next of 256 counters in turn.  Launches on one stream may follow each other
- * without limit; at most 256 launches may be in flight at the same time
- * across streams, and a CUDA graph that holds this call must not be replayed
- * on two streams at once.
+ * work from a pair of counters in the library's device memory.  An ordinary
+ * call takes the next of 256 such pairs in turn; a call made while `stream` is
+ * being captured into a CUDA graph takes the next of 1024 further pairs, which
+ * that graph then uses on every replay, so graph replays and ordinary calls
+ * never share counters.  The rules that follow:
+ *   - ordinary calls on one stream may follow each other without limit; at
+ *     most 256 ordinary calls may be in flight at the same time across streams;
+ *   - a graph holding this call must not be replayed while it is still
+ *     running (e.g. on two streams at once), and two graphs whose captures of
+ *     this call lie a multiple of 1024 captures apart must not run at the
+ *     same time.
+ * A launch that finds its counters used by another launch at the same time
+ * sets ATTN_DEVERR_SCHED in the device error word (its results may then be
+ * incomplete).
  */
 int attn_prefill(const void* q, const void* k, const void* v, void* out, float* lse,
                  int B, int Hq, int Hkv, int Lq, int Lk, int D, float scale, int is_causal,
@@ -403,6 +418,31 @@ int attn_selftest_kv8_convert(const uint16_t* codes, uint32_t* out, int n, int k
  */
 int attn_selftest_exp2(const float* x, float* y, int n, void* stream);
 
+/*
+ * attn_selftest_wait -- diagnostic: makes the kernels' bounded pipeline wait
+ * run out, without touching any real pipeline.  One CTA of two warps: a
+ * "producer" announces bytes on a barrier that never arrive (no copy is
+ * issued) and then waits, with the kernels' usual ~2 s limit, for the
+ * "consumer" to free the entry; the consumer waits on the first barrier with
+ * a limit of limit_ns nanoseconds (0 < limit_ns <= 2e9).  The consumer's wait
+ * gives up, sets ATTN_DEVERR_TIMEOUT in the device error word and raises the
+ * CTA's abort flag, which ends the producer's wait too.
+ *   result: device int[4], written: {producer wait succeeded (0/1), producer
+ *   wait time in us, consumer wait succeeded (0/1), consumer wait time in us}.
+ * Enqueued on `stream`; the caller clears the error word afterwards
+ * (attn_device_error with reset).  Errors: ATTN_ERR_INVALID_ARG, ATTN_ERR_CUDA.
+ */
+int attn_selftest_wait(unsigned long long limit_ns, int* result, void* stream);
+
+/*
+ * attn_prefill_sched_busy -- diagnostic: synchronise the current device and
+ * count the prefill scheduling counters (see attn_prefill, "Concurrency")
+ * that are not zero.  Between launches every counter is zero, also after a
+ * launch that gave up on a wait.  Returns ATTN_OK or ATTN_ERR_CUDA /
+ * ATTN_ERR_INVALID_ARG.
+ */
+int attn_prefill_sched_busy(int* busy);
+
 /* attn_status_string -- a static name for a status code; never NULL. */
 const char* attn_status_string(int status);
 
@@ -418,6 +458,8 @@ const char* attn_last_error(void);
 #define ATTN_DEVERR_TIMEOUT 0x1u  /* a pipeline wait gave up after ~2 s */
 #define ATTN_DEVERR_SEQLEN  0x2u  /* a seqlens value was outside [0, Lmax] */
 #define ATTN_DEVERR_PAGE    0x4u  /* a block_table entry was outside [0, n_pages) */
+#define ATTN_DEVERR_SCHED   0x8u  /* a prefill launch shared its scheduling counters with another
+                                     launch running at the same time (see attn_prefill) */
 
 /*
  * attn_device_error -- synchronise the current device, copy its error word

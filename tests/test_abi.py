@@ -219,3 +219,25 @@ def test_decode_partial_and_merge_reject(lib):
         ("q", A), ("k", A), ("v", A), ("sl", A), ("o", A), ("l", A), ("B", 2), ("Hq", 8), ("Hkv", 2), ("Lmax", 64),
         ("D", 128), ("scale", 0.1), ("ws", A), ("wsb", 1 << 30))], None)
     assert p(l=NULL) == -1 and p(D=96) == -2 and p(ws=NULL) == -3 and p(B=0) == 0
+
+
+def test_decode_noalloc_rejects_before_any_gpu_work(lib):
+    """The no-alloc decode shares attn_decode's checks, and refuses sizes whose
+    partials do not fit its static scratch before it looks the scratch up."""
+    f = lambda **kw: lib.attn_decode_noalloc(*[kw.get(n, d) for n, d in (
+        ("q", A), ("k", A), ("v", A), ("sl", A), ("out", A), ("lse", NULL), ("B", 2), ("Hq", 8), ("Hkv", 2),
+        ("Lmax", 64), ("D", 128), ("scale", 0.1))], None)
+    assert f(sl=NULL) == -1 and f(Lmax=0) == -1 and f(Hq=5) == -1 and f(k=NULL) == -1 and f(scale=0.0) == -1
+    assert f(D=96) == -2 and f(Hq=256, Hkv=1) == -2
+    assert f(B=0) == 0
+    # Hq 64 at 131072 cached rows for 64 sequences: far more partials than the 16 MiB scratch
+    assert lib.attn_decode_workspace_size(64, 64, 8, 131072, 128) > _native.ATTN_DECODE_NOALLOC_SCRATCH_BYTES
+    assert f(B=64, Hq=64, Hkv=8, Lmax=131072) == -3
+    assert b"static scratch" in lib.attn_last_error()
+
+
+def test_diagnostics_reject(lib):
+    assert lib.attn_selftest_wait(0, A, None) == -1
+    assert lib.attn_selftest_wait(1000, NULL, None) == -1
+    assert lib.attn_selftest_wait(3_000_000_000, A, None) == -1
+    assert lib.attn_prefill_sched_busy(None) == -1

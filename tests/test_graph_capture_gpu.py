@@ -56,3 +56,40 @@ def test_capture_and_replay_step():
     want = (p_out, p_lse, d_out, d_lse, k_out, k_lse)
     assert all(torch.equal(a, b) for a, b in zip(got, want))
     del g
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_captured_prefill_and_ordinary_calls_do_not_share_counters(D):
+    """A captured prefill keeps one pair of scheduling counters for every replay.
+    Ordinary calls cycle through their own 256 pairs, so even with more than 256
+    of them running on a second stream while the graph is replayed on a first,
+    no launch shares counters with another: every replay gives the captured
+    call's exact result, every ordinary call its own, and the device error word
+    (which a shared counter would flag) stays clear."""
+    dev = torch.device("cuda")
+    qa, ka, va = (t.to(dev) for t in W.prefill_inputs(1, 16, 4, 1500, 1500, D, seed=11))
+    qb, kb, vb = (t.to(dev) for t in W.prefill_inputs(1, 16, 4, 1100, 1100, D, seed=12))
+    want_a, _ = attn.prefill(qa, ka, va)
+    want_b, _ = attn.prefill(qb, kb, vb)
+    torch.cuda.synchronize()
+    out_a = torch.empty_like(qa)
+    sa, sb = torch.cuda.Stream(), torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=sa):
+        attn.prefill(qa, ka, va, out=out_a, want_lse=False, stream=sa)
+    snaps = []
+    outs_b = [torch.empty_like(qb) for _ in range(4)]
+    n_b = 0
+    for i in range(40):
+        with torch.cuda.stream(sa):
+            g.replay()
+            snaps.append(out_a.clone())
+        with torch.cuda.stream(sb):
+            for _ in range(8):   # 320 ordinary calls in all: every ordinary slot used more than once
+                attn.prefill(qb, kb, vb, out=outs_b[n_b % 4], want_lse=False, stream=sb)
+                n_b += 1
+    torch.cuda.synchronize()
+    assert attn.device_error(reset=True) == 0
+    assert all(torch.equal(s, want_a) for s in snaps)
+    assert all(torch.equal(o, want_b) for o in outs_b)
+    del g
