@@ -46,6 +46,9 @@ from exact_tiled_attention_gqa_b200 import workloads as W          # noqa: E402
 METRIC = "prefill TFLOP/s & decode HBM GB/s (frac. of roofline), Qwen3-8B GQA shapes"
 PREFILL = W.QWEN_PREFILL_8K_B4
 DECODE = W.QWEN_DECODE
+PREFILL_WORKLOADS = {"qwen3_8b_b4_l8192": W.QWEN_PREFILL_8K_B4, "qwen3_8b_b1_l4096": W.QWEN_PREFILL_4K,
+                     "chunked_16k": W.CHUNKED_16K, "chunked_32k": W.CHUNKED_32K, "hd64_b4_l8192": W.HD64_PREFILL,
+                     "hd256_b2_l8192": W.HD256_PREFILL}
 
 
 def parse():
@@ -68,6 +71,8 @@ def parse():
                     help="with --only decode: the cache element format (8-bit caches use attn_decode_kv8)")
     ap.add_argument("--decode-group", type=int, default=None,
                     help="profiling aid: with --only decode, use the group-size sweep shape with this G")
+    ap.add_argument("--prefill-workload", choices=sorted(PREFILL_WORKLOADS), default="qwen3_8b_b4_l8192",
+                    help="profiling aid: with --only prefill, the prefill workload to time")
     ap.add_argument("--no-sweeps", action="store_true",
                     help="skip the other workloads (group-size decode sweep, other prefill shapes)")
     return ap.parse_args()
@@ -78,7 +83,8 @@ def parse():
 # --------------------------------------------------------------------------
 class ClockSampler:
     """Polls SM clock, power and throttle reasons through NVML every ~10 ms
-    while the timed region runs (nvidia-smi's 100 ms loop is the fallback)."""
+    while the timed region runs.  Without NVML the line's clocks record says
+    why and holds no samples."""
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
 
@@ -146,6 +152,12 @@ def run_ours(args, rank, world, local_rank):
     import exact_tiled_attention_gqa_b200 as attn
     from exact_tiled_attention_gqa_b200 import build
 
+    global PREFILL
+    if args.prefill_workload != "qwen3_8b_b4_l8192":
+        if args.only != "prefill":
+            raise SystemExit("--prefill-workload applies to --only prefill")
+        PREFILL = PREFILL_WORKLOADS[args.prefill_workload]
+
     build.build()
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
@@ -204,7 +216,8 @@ def run_ours(args, rank, world, local_rank):
 
     def call_prefill():
         if do_pre:
-            attn.prefill(q, k, v, is_causal=True, out=p_out, lse=p_lse, stream=stream)
+            attn.prefill(q, k, v, scale=PREFILL.scale, is_causal=PREFILL.is_causal, out=p_out, lse=p_lse,
+                         stream=stream)
 
     def call_decode():
         if do_dec and kv8:
@@ -291,6 +304,11 @@ def run_ours(args, rank, world, local_rank):
     h2d = (hq.numel() + hk.numel() + hv.numel() + hdq.numel()) * 2
     d2h = (ho.numel() + hdo.numel()) * 2 + (hl.numel() + hdl.numel()) * 4
 
+    kvp_line = None
+    if args.only is None:
+        kvp_line = run_kv_parallel(attn, dev, stream, rank, world, args.seed, max(3, args.steps // 4), 2,
+                                   max_over_ranks, barrier)
+
     cpu_line = None
     if rank == 0 and not args.no_cpu_baseline and args.only is None:
         cpu_line = cpu_baseline(args, q_h, k_h, v_h, dq.cpu(), dk, dv, seqlens_host)
@@ -350,6 +368,7 @@ def run_ours(args, rank, world, local_rank):
                         "out pipelined by the library); decode: pinned q in, attn_decode, pinned out/lse back, "
                         "KV cache resident"},
         "gpu_launches": 3 * args.steps,
+        "kv_parallel": kvp_line,
         "sweeps": sweeps,
         "clocks": clocks,
     }
@@ -358,6 +377,53 @@ def run_ours(args, rank, world, local_rank):
     return line
 
 
+def run_kv_parallel(attn, dev, stream, rank, world, seed, steps, warmup, max_over_ranks, barrier):
+    """KV-parallel decode of the Qwen3-8B decode batch (the NVIDIA attention page,
+    "Parameter four: parallelism"): every rank holds a 1/world share of each
+    sequence's cached rows, so the batch is fixed as ranks are added (strong
+    scaling).  A step is attn_decode_partial on the local rows, an all-gather of
+    the fp32 partials over NCCL, and attn_decode_merge (multigpu.KVParallelDecode).
+    At one GPU the step is the partial and the merge, with no exchange."""
+    from exact_tiled_attention_gqa_b200.multigpu import KVParallelDecode, kv_shard_rows, shard_seqlens
+    shape = DECODE
+    gcpu = torch.Generator().manual_seed(seed + 4242)   # the same sequences and queries on every rank
+    sl = torch.randint(shape.seqlen_lo, shape.seqlen_hi + 1, (shape.B,), generator=gcpu).to(torch.int32)
+    q = torch.randn((shape.B, shape.Hq, shape.D), generator=gcpu).to(torch.bfloat16).to(dev)
+    rows = kv_shard_rows(shape.Lmax, rank, world)
+    g = torch.Generator(device=dev)
+    g.manual_seed(seed + 77 + rank)
+    k = torch.empty((shape.B, shape.Hkv, len(rows), shape.D), dtype=torch.bfloat16, device=dev)
+    v = torch.empty_like(k)
+    for cache in (k, v):
+        for b in range(shape.B):
+            cache[b].copy_(torch.randn(cache[b].shape, generator=g, device=dev).to(torch.bfloat16))
+    ws = torch.empty(attn.decode_workspace_size(shape.B, shape.Hq, shape.Hkv, len(rows), shape.D), dtype=torch.uint8,
+                     device=dev)
+    kvp = KVParallelDecode(q, k, v, shard_seqlens(sl, rows).to(dev), scale=shape.scale, workspace=ws)
+    for _ in range(warmup):
+        kvp.step()
+    torch.cuda.synchronize()
+    barrier()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for e0, e1 in ev:
+        e0.record(stream)
+        kvp.step()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    ms = max_over_ranks(sum(e0.elapsed_time(e1) for e0, e1 in ev) / steps)
+    by = RL.decode_bytes(sl.tolist(), shape.B, shape.Hq, shape.Hkv, shape.D)
+    peak_b = float(RL.measured_peaks()["hbm_gbs"])
+    del kvp, k, v, ws
+    torch.cuda.empty_cache()
+    return {"workload": shape.name + f", cache rows split over {world} GPU(s)", "n_gpus": world,
+            "scaling": "strong", "ms_per_step": round(ms, 4), "value": round(by / ms / 1e6, 1), "unit": "GB/s",
+            "bytes_per_step": by, "frac_of_measured_hbm_per_gpu": round(by / ms / 1e6 / world / peak_b, 4),
+            "exchange": (f"all-gather of fp32 partials over NCCL, {shape.B * shape.Hq * (shape.D + 1) * 4} bytes "
+                         "per rank" if world > 1 else "none (one GPU)")}
+
+
+_L2_FLUSH = None
 _L2_FLUSH = None
 
 

@@ -11,7 +11,12 @@ import ctypes
 import os
 import threading
 
-from .build import LIB_PATH
+from .build import DEBUG_LIB_PATH, LIB_PATH
+
+# ATTN_GQA_DEBUG_BOUNDS=1 in the environment loads the bounds-checking build of
+# the same sources instead (build.py, debug_bounds=True); tests use it.
+if os.environ.get("ATTN_GQA_DEBUG_BOUNDS") == "1":
+    LIB_PATH = DEBUG_LIB_PATH
 
 ATTN_OK = 0
 ATTN_ERR_INVALID_ARG = -1
@@ -22,6 +27,7 @@ ATTN_DEVERR_TIMEOUT = 0x1
 ATTN_DEVERR_SEQLEN = 0x2
 ATTN_DEVERR_PAGE = 0x4
 ATTN_DEVERR_SCHED = 0x8
+ATTN_DEVERR_BOUNDS = 0x10
 ATTN_DECODE_NOALLOC_SCRATCH_BYTES = 16 << 20
 ATTN_KV_E4M3 = 1
 ATTN_KV_Q8_0 = 2

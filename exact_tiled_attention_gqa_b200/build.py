@@ -19,6 +19,10 @@ ROOT = os.path.dirname(PKG_DIR)
 CSRC = os.path.join(PKG_DIR, "csrc")
 LIB_NAME = "libattn_gqa_sm100.so"
 LIB_PATH = os.path.join(PKG_DIR, LIB_NAME)
+# The same sources built with -DATTN_DEBUG_BOUNDS=1: the kernels check their
+# unit mapping, ring positions, TMA coordinates and output indices and report a
+# violation as ATTN_DEVERR_BOUNDS (a checking build for tests, not for speed).
+DEBUG_LIB_PATH = os.path.join(PKG_DIR, "libattn_gqa_sm100_debug_bounds.so")
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 
@@ -34,10 +38,10 @@ def sources() -> list:
                   [os.path.join(ROOT, "include", "attn_gqa.h")])
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB_PATH):
+def up_to_date(path: str = LIB_PATH) -> bool:
+    if not os.path.exists(path):
         return False
-    t = os.path.getmtime(LIB_PATH)
+    t = os.path.getmtime(path)
     return all(os.path.getmtime(s) <= t for s in sources())
 
 
@@ -72,12 +76,14 @@ def check_ptxas_report(report: str) -> dict:
     return {k: tuple(v) for k, v in kernels.items()}
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB_PATH
-    tmp = LIB_PATH + f".tmp{os.getpid()}"
+def build(force: bool = False, verbose: bool = False, debug_bounds: bool = False) -> str:
+    path = DEBUG_LIB_PATH if debug_bounds else LIB_PATH
+    if not force and up_to_date(path):
+        return path
+    tmp = path + f".tmp{os.getpid()}"
     cmd = [_nvcc(), "-std=c++17", "-O3", "-lineinfo", *ARCH_FLAGS, "-Xcompiler", "-fPIC", "-shared",
-           "-Xptxas", "-v", os.path.join(CSRC, "attn_gqa.cu"), "-o", tmp]
+           "-Xptxas", "-v", *(["-DATTN_DEBUG_BOUNDS=1"] if debug_bounds else []),
+           os.path.join(CSRC, "attn_gqa.cu"), "-o", tmp]
     res = subprocess.run(cmd, capture_output=True, text=True)
     if res.returncode != 0:
         raise RuntimeError(f"nvcc failed:\n{res.stdout}\n{res.stderr}")
@@ -89,9 +95,9 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if verbose:
         for name, (regs, spill) in sorted(kernels.items()):
             print(f"{regs:4d} regs {spill:6d} B spill  {name}")
-    os.replace(tmp, LIB_PATH)
-    return LIB_PATH
+    os.replace(tmp, path)
+    return path
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="-v" in sys.argv, debug_bounds="--debug-bounds" in sys.argv))

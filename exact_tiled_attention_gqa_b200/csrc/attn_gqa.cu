@@ -227,23 +227,42 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
     return check_launch("attn_prefill_sm100_kernel");
 }
 
-// Cache rows per decode split, a power of two in [256, 4096].
-//  - mma.sync split kernel: the largest that still gives about four waves of
-//    CTAs on a 148-SM part (1184 CTAs).
-//  - tcgen05 kernel: the largest (down to 512) that still gives one CTA per SM.
-//    Its CTAs carry more setup and each split adds a partial for the combine
-//    to merge, so long splits win: measured on B200 at 131072 cached rows,
-//    G = 64 took 0.148 / 0.122 / 0.106 ms with 1024 / 2048 / 4096-row splits.
-// D = 256 always takes the tcgen05 kernel: a 256-wide O per row does not fit
-// the mma.sync kernel's registers.
+// Cache rows per decode split (always a multiple of 64, the tile height).
+//  - mma.sync split kernel: the largest power of two in [256, 4096] that still
+//    gives about four waves of CTAs on a 148-SM part (1184 CTAs).
+//  - tcgen05 kernel (D = 256, or more than 16 query rows per KV head): its CTAs
+//    carry more setup than the split kernel's (TMEM, the Q tile, a partial per
+//    row for the combine), so splits are long, and the split length balances
+//    the waves: of the multiples of 64 in [512, 8192], the one that minimises
+//    waves x (rows per split + 512), with waves = splits / CTA slots rounded up
+//    (148 SMs x 2 CTAs for D <= 128, x 1 for D = 256) and the split count taken
+//    at Lmax.  At 131072 cached rows and G = 64 (8 sequences, one KV head) this
+//    gives 3584-row splits, 296 CTAs, two on every SM; 4096-row splits gave
+//    256 CTAs, so 40 SMs ran one CTA while the rest ran two.
+// The result depends only on the arguments (workspace sizes do too).
 bool decode_uses_tc(int D, int rows_per_group) { return D == 256 || rows_per_group > 16; }
 
-int decode_chunk(int B, int Hkv, int Lmax, bool tc_path) {
-    const long long target = tc_path ? 148LL : 148LL * 2 * 4;
-    const int min_chunk = tc_path ? 512 : 256;
-    int chunk = 4096;
-    while (chunk > min_chunk && static_cast<long long>(B) * Hkv * ((Lmax + chunk - 1) / chunk) < target) chunk >>= 1;
-    return chunk;
+int decode_chunk(int B, int Hkv, int Lmax, bool tc_path, int D) {
+    const long long groups = static_cast<long long>(B) * Hkv;
+    if (!tc_path) {
+        int chunk = 4096;
+        while (chunk > 256 && groups * ((Lmax + chunk - 1) / chunk) < 148LL * 2 * 4) chunk >>= 1;
+        return chunk;
+    }
+    const long long slots = 148LL * (D <= 128 ? 2 : 1);
+    int best = 512;
+    long long best_cost = -1;
+    for (int c = 512; c <= 8192; c += 64) {
+        const long long splits = (Lmax + c - 1) / c;
+        const long long waves = (groups * splits + slots - 1) / slots;
+        const long long cost = waves * (c + 512);
+        if (best_cost < 0 || cost < best_cost) {   // ties keep the shorter split (more parallel partials)
+            best_cost = cost;
+            best = c;
+        }
+        if (splits == 1) break;   // longer splits change nothing
+    }
+    return best;
 }
 
 size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
@@ -255,7 +274,7 @@ struct DecodeLayout {
 
 DecodeLayout decode_layout(int B, int Hq, int Hkv, int Lmax, int D, int Lq = 1, bool kv8 = false) {
     DecodeLayout d;
-    d.chunk = decode_chunk(B, Hkv, Lmax, !kv8 && decode_uses_tc(D, (Hq / Hkv) * Lq));
+    d.chunk = decode_chunk(B, Hkv, Lmax, !kv8 && decode_uses_tc(D, (Hq / Hkv) * Lq), D);
     d.n_splits = (Lmax + d.chunk - 1) / d.chunk;
     const size_t rows = static_cast<size_t>(B) * Hq * Lq * d.n_splits;
     d.o_bytes = align256(rows * D * sizeof(float));

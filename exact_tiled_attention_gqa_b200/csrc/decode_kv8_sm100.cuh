@@ -135,6 +135,7 @@ __device__ __forceinline__ void kv8_produce(const CUtensorMap* tm_k, const CUten
             row = key0 % p.page_size;
             outer = page * p.Hkv + g;
         }
+        decode_check_tile(p, row, outer);
         if (!mbar_wait(bar_empty(s), (round & 1u) ^ 1u, abort_flag, &g_attn_err, kDevErrTimeout)) break;
         mbar_arrive_expect_tx(bar_full(s), L::kStageTx);
         const uint32_t dst = ring + s * L::kStageBytes;
@@ -456,6 +457,7 @@ __global__ void __maxnreg__(200)
             acc += sm_o[(ww * 16 + rr) * D + d] * sc;
         }
         const size_t prow = (group_row0 + row) * p.n_splits + split;
+        decode_check_prow(p, prow);
         p.o_part[prow * D + d] = (Lsum > 0.0f) ? acc * vscale / Lsum : 0.0f;
         if (d == 0) p.lse_part[prow] = (Lsum > 0.0f) ? M + __log2f(Lsum) : -INFINITY;
     }
@@ -786,6 +788,7 @@ __global__ void __launch_bounds__(kDecThreads, kv8t_min_blocks<NR>())
             acc += sm_o[(w * 16 + row) * D + d] * sc;
         }
         const size_t prow = (group_row0 + row) * p.n_splits + split;
+        decode_check_prow(p, prow);
         p.o_part[prow * D + d] = (Lsum > 0.0f) ? acc * vscale / Lsum : 0.0f;
         if (d == 0) p.lse_part[prow] = (Lsum > 0.0f) ? M + __log2f(Lsum) : -INFINITY;
     }

@@ -86,6 +86,20 @@ __device__ __forceinline__ int decode_seqlen(const DecodeParams& p, int b) {
     return n;
 }
 
+// (debug builds) a tile starting at cache row `row` of slab `outer` lies in the
+// view TMA reads: [B * Hkv, Lmax] rows, or [n_pages * Hkv, page_size] when paged
+__device__ __forceinline__ void decode_check_tile(const DecodeParams& p, int row, int outer) {
+    const int rows = p.block_table ? p.page_size : p.Lmax;
+    const long long outers = p.block_table ? static_cast<long long>(p.n_pages) * p.Hkv
+                                           : static_cast<long long>(p.B) * p.Hkv;
+    ATTN_CHECK(row >= 0 && row < rows && outer >= 0 && outer < outers);
+}
+
+// (debug builds) a partial row index lies in [B * Hq * Lq * n_splits)
+__device__ __forceinline__ void decode_check_prow(const DecodeParams& p, size_t prow) {
+    ATTN_CHECK(prow < static_cast<size_t>(p.B) * p.Hq * p.Lq * p.n_splits);
+}
+
 // KPW = cache rows of each 64-row tile handled by one compute warp (16, 32 or 64).
 // A group's query rows are the G heads x Lq new tokens, head-major (row r = head
 // r / Lq, token r % Lq), which is also their order in q, out and lse.
@@ -146,6 +160,7 @@ __global__ void __maxnreg__(200)
                     row = key0 % p.page_size;
                     outer = page * p.Hkv + g;
                 }
+                decode_check_tile(p, row, outer);
                 if (!mbar_wait(bar_empty(s), (round & 1u) ^ 1u, abort_flag, &g_attn_err, kDevErrTimeout)) break;
                 mbar_arrive_expect_tx(bar_full(s), L::kStageBytes);
                 const uint32_t dst = ring + s * L::kStageBytes;
@@ -381,6 +396,7 @@ __global__ void __maxnreg__(200)
             acc += sm_o[(ww * 16 + rr) * D + d] * sc;
         }
         const size_t prow = (group_row0 + row) * p.n_splits + split;
+        decode_check_prow(p, prow);
         p.o_part[prow * D + d] = (Lsum > 0.0f) ? acc / Lsum : 0.0f;
         if (d == 0) p.lse_part[prow] = (Lexact > 0.0f) ? M + __log2f(Lexact) : -INFINITY;
     }
@@ -400,6 +416,7 @@ __global__ void __launch_bounds__(128)
     const int b = row / (p.Hq * p.Lq);
     const int seqlen = decode_seqlen(p, b);
     const int n_valid = (seqlen + p.chunk - 1) / p.chunk;
+    ATTN_CHECK(n_valid >= 0 && n_valid <= p.n_splits);
     const float* lp = p.lse_part + static_cast<size_t>(row) * p.n_splits;
     const float* op = p.o_part + static_cast<size_t>(row) * p.n_splits * D;
     constexpr int kPer = D / 32;

@@ -70,7 +70,8 @@ struct DecodeTcSmem {
     // q_full, full[S], empty[S], s_full[2], p_full[2], o_ready, o_done, drain
     static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 3;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem base, abort flag
-    static constexpr int kBytes = kMiscOff + 16;
+    static constexpr int kTagOff = kMiscOff + 16;             // debug builds: ring entry -> item index
+    static constexpr int kBytes = kTagOff + 4 * kStages;
     static constexpr int kAlloc = kBytes + 1024;
     static_assert(kAlloc <= 232448, "dynamic shared memory per CTA");
     static_assert(kStages >= 4, "ring too shallow");
@@ -109,6 +110,8 @@ __global__ void __launch_bounds__(kDtcThreads, DecodeTcSmem<D>::kCtasPerSm)
     const uint32_t bar_drain = bar_o_ready + 16u;
     uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
+    // (debug builds) the ring position the producer put in each entry, checked by the MMA warp
+    volatile int* ring_tag = reinterpret_cast<volatile int*>(smem + L::kTagOff);
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q_full, 1);
@@ -179,6 +182,9 @@ __global__ void __launch_bounds__(kDtcThreads, DecodeTcSmem<D>::kCtasPerSm)
                     row = key0 % p.page_size;
                     outer = page * p.Hkv + g;
                 }
+                decode_check_tile(p, row, outer);
+                ATTN_CHECK(j >= 0 && j < n_tiles);
+                if (ATTN_DEBUG_BOUNDS) ring_tag[s] = t;
                 mbar_arrive_expect_tx(bar_full(s), L::kHalfBytes);
                 const CUtensorMap* map = is_v ? &tm_v : &tm_k;
                 const uint32_t dst = sKV + s * L::kHalfBytes;
@@ -208,7 +214,9 @@ __global__ void __launch_bounds__(kDtcThreads, DecodeTcSmem<D>::kCtasPerSm)
         const uint64_t dV0 = umma_sdesc_sw128(sKV, L::kHalfBlockBytes, 1024);
         constexpr uint64_t kSlotStep = L::kHalfBytes >> 4;
         auto wait_item = [&](int it) {
-            return mbar_wait(bar_full(slot_of(it)), par_of(it), abort_flag, &g_attn_err, kDevErrTimeout);
+            const bool got = mbar_wait(bar_full(slot_of(it)), par_of(it), abort_flag, &g_attn_err, kDevErrTimeout);
+            if (got) ATTN_CHECK(ring_tag[slot_of(it)] == it);   // (debug builds) the entry holds that item
+            return got;
         };
         // S(j) = Q K_j^T into buffer j % 2 (N = 64 cache rows)
         auto qk = [&](int j) {
@@ -407,6 +415,7 @@ __global__ void __launch_bounds__(kDtcThreads, DecodeTcSmem<D>::kCtasPerSm)
         const bool row_valid = r < R;
         const float inv_l = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
         const size_t prow = (group_row0 + static_cast<size_t>(row_valid ? r : 0)) * p.n_splits + split;
+        decode_check_prow(p, prow);
         float* dst = p.o_part + prow * D;
 #pragma unroll 1
         for (int c = 0; c < D; c += 32) {

@@ -115,6 +115,9 @@ struct PrefillSmem {
     // NQ = 2 CTAs are persistent and take work units from a counter; an NQ = 1
     // CTA takes one unit (its shared memory has no room for the O staging block)
     static constexpr bool kPersistent = (kNQ == 2);
+    // D = 64: S0 | S1 | O0 | O1 take 384 TMEM columns, so P gets columns of its
+    // own (P0 at 384, P1 at 448) instead of overwriting S; see the file comment
+    static constexpr bool kSplitP = (D == 64);
     // ring entries: whole K or V tiles, or half tiles (32 KB each) for D = 256
     static constexpr int kItemsPerTile = (D == 256) ? 2 : 1;
     static constexpr int kItemBytes = kKVTileBytes / kItemsPerTile;
@@ -127,10 +130,11 @@ struct PrefillSmem {
     static constexpr int kStgOff = kKVOff + kStages * kItemBytes;
     static constexpr int kBarOff = kStgOff + (kPersistent ? kNQ * kBlockBytes : 0);
     // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_half[2], p_full[2], o_done[2], drain,
-    //           q_empty, unit_full[2], unit_empty[2]
-    static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 2 + 1 + 1 + 2 + 2;
+    //           q_empty, unit_full[2], unit_empty[2], s_free[2], pv_done[2]
+    static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 2 + 1 + 1 + 2 + 2 + 2 + 2;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;   // tmem base, abort flag, two unit slots (int each)
-    static constexpr int kBytes = kMiscOff + 16;
+    static constexpr int kTagOff = kMiscOff + 16;             // debug builds: ring entry -> item index
+    static constexpr int kBytes = kTagOff + 4 * kStages;
     static constexpr int kAlloc = kBytes + 1024;              // slack to align the base to 1 KiB
     static_assert(kAlloc <= 232448, "dynamic shared memory per CTA");
     static_assert(kStgOff % 1024 == 0, "swizzled TMA blocks start on 1 KiB");
@@ -204,6 +208,7 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
     using L = PrefillSmem<D>;
     static_assert(L::kNQ == NQ, "Q tiles per CTA follow from D");
     constexpr bool kPersistent = L::kPersistent;
+    constexpr bool kSplitP = L::kSplitP;
     constexpr int kThreads = prefill_threads<NQ>();
     constexpr int kProducerWarp = 4 * NQ;
     constexpr int kMmaWarp = 4 * NQ + 1;
@@ -233,9 +238,14 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
     const uint32_t bar_q_empty = bar0 + 8u * (10 + 2 * L::kStages);
     auto bar_unit_full = [&](int s) { return bar0 + 8u * (11 + 2 * L::kStages + s); };
     auto bar_unit_empty = [&](int s) { return bar0 + 8u * (13 + 2 * L::kStages + s); };
+    // (split P only) the softmax has read S_q into registers / O_q += P_q V has completed
+    auto bar_s_free = [&](int q) { return bar0 + 8u * (15 + 2 * L::kStages + q); };
+    auto bar_pv_done = [&](int q) { return bar0 + 8u * (17 + 2 * L::kStages + q); };
     uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
     volatile int* unit_slot = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 8);
+    // (debug builds) the ring position the producer put in each entry, checked by the MMA thread
+    volatile int* ring_tag = reinterpret_cast<volatile int*>(smem + L::kTagOff);
 
     if (threadIdx.x == 0) {
         mbar_init(bar_q_full, 1);
@@ -251,6 +261,8 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
             mbar_init(bar_o_done(q), 1);
             mbar_init(bar_unit_full(q), 1);
             mbar_init(bar_unit_empty(q), kUnitReaders);
+            mbar_init(bar_s_free(q), 4);   // one arrival per softmax warp
+            mbar_init(bar_pv_done(q), 1);
         }
         mbar_init(bar_drain, 1);
         *abort_flag = 0;
@@ -309,6 +321,9 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
                 mbar_arrive(bar_unit_full(s));
                 if (!have) break;
                 const PrefillUnit u = prefill_unit<NQ>(p, idx);
+                ATTN_CHECK(idx >= 0 && u.b >= 0 && u.b < p.B && u.g >= 0 && u.g < p.Hkv && u.p_begin >= 0 &&
+                           u.p_begin < p.Lq && u.p_begin % (NQ * P) == 0 && u.n_kt >= 0 &&
+                           u.n_kt <= (p.Lk + kBN - 1) / kBN);
                 // The next unit is taken once this one's loads are all issued (about
                 // two key tiles before its MMAs end), not earlier: a CTA that claimed
                 // its next unit at the start of a long one would hold it back from SMs
@@ -326,6 +341,7 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
                     if (!ok) break;
                 }
                 const int q_head0 = u.b * p.Hq + u.g * p.G;
+                ATTN_CHECK(q_head0 >= 0 && q_head0 + p.G <= p.B * p.Hq);
                 mbar_arrive_expect_tx(bar_q_full, q_bytes);
                 for (int q = 0; q < NQ; ++q)
                     for (int kb = 0; kb < L::kKB; ++kb)
@@ -339,11 +355,14 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
                     const uint32_t round = static_cast<uint32_t>(t / L::kStages);
                     ok = mbar_wait(bar_kv_empty(st), (round & 1u) ^ 1u, abort_flag, &g_attn_err, kDevErrTimeout);
                     if (!ok) break;
-                    mbar_arrive_expect_tx(bar_kv_full(st), L::kItemBytes);
                     bool is_v;
                     int j;
                     ring_tile<NQ>(i / L::kItemsPerTile, u.n_kt, is_v, j);
                     const int kb0 = (i % L::kItemsPerTile) * L::kItemKB;
+                    ATTN_CHECK(j >= 0 && j < u.n_kt && kv_row >= 0 && kv_row < p.B * p.Hkv &&
+                               (kb0 + L::kItemKB) * 64 <= D);
+                    if (ATTN_DEBUG_BOUNDS) ring_tag[st] = t;
+                    mbar_arrive_expect_tx(bar_kv_full(st), L::kItemBytes);
                     const CUtensorMap* map = is_v ? &tm_v : &tm_k;
                     for (int kb = 0; kb < L::kItemKB; ++kb)
                         tma_load_3d(sKV + st * L::kItemBytes + kb * L::kBlockBytes, map, bar_kv_full(st),
@@ -394,6 +413,7 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
             constexpr uint32_t kIdescPV = umma_idesc_bf16_f32(kBM, D, true);
             const uint32_t tS[2] = {tmem + 0u, tmem + 128u};
             const uint32_t tO[2] = {tmem + 256u, tmem + 256u + D};
+            const uint32_t tP[2] = {kSplitP ? tmem + 384u : tS[0], kSplitP ? tmem + 448u : tS[1]};
             int tb = 0;      // ring entries of earlier units
             int tiles = 0;   // key tiles of earlier units (phases of the per-tile barriers)
             int nu = 0;      // earlier units with key tiles
@@ -402,6 +422,8 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
             // cost about 60 cycles per key tile (measured).
             auto slot_of = [&](int t) { return static_cast<int>(static_cast<unsigned>(tb + t) % L::kStages); };
             auto par_of = [&](int t) { return (static_cast<unsigned>(tb + t) / L::kStages) & 1u; };
+            // (debug builds) the entry holds the item this thread expects there
+            auto check_item = [&](int t) { ATTN_CHECK(ring_tag[slot_of(t)] == tb + t); };
             // Shared-memory descriptors are built once; a k-step only moves the
             // start-address field (bits 0-13, address >> 4), so each MMA issue
             // costs one 64-bit add.
@@ -425,7 +447,7 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
 #pragma unroll
                 for (int k4 = 0; k4 < kBN / 32; ++k4) {
                     const int kk = half * (kBN / 32) + k4;
-                    umma_ts(tO[q], tS[q] + kk * 8, b0 + static_cast<uint64_t>((kk * 2048) >> 4), kIdescPV,
+                    umma_ts(tO[q], tP[q] + kk * 8, b0 + static_cast<uint64_t>((kk * 2048) >> 4), kIdescPV,
                             (acc || kk > 0) ? 1u : 0u);
                 }
             };
@@ -452,8 +474,59 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
                 const int n_kt = prefill_unit<NQ>(p, idx).n_kt;
                 if (n_kt == 0) continue;
                 ok = mbar_wait(bar_q_full, static_cast<uint32_t>(nu) & 1u, abort_flag, &g_attn_err, kDevErrTimeout);
-              if constexpr (NQ == 2) {
+              if constexpr (kSplitP) {
+                // P has TMEM columns of its own: S_q(j+1) = Q_q K_{j+1}^T is issued as soon
+                // as the softmax has read S_q(j) into registers, and O_q += P_q(j) V_j once
+                // P_q(j) is in TMEM, so the next tile's scores are ready when the softmax
+                // finishes this one.  pv_done_q tells the softmax when P_q and O_q are free.
                 if (ok) ok = mbar_wait(bar_kv_full(slot_of(0)), par_of(0), abort_flag, &g_attn_err, kDevErrTimeout);
+                if (ok) check_item(0);
+                if (ok) {
+                    tc_fence_after_sync();
+                    issue_qk(0, 0);
+                    umma_commit(bar_s_full(0));
+                    issue_qk(1, 0);
+                    umma_commit(bar_s_full(1));
+                    if (n_kt == 1) umma_commit(bar_q_empty);
+                    umma_commit(bar_kv_empty(slot_of(0)));
+                }
+                for (int j = 0; j < n_kt && ok; ++j) {
+                    const int tv = 2 * j + 1, tk = 2 * j + 2;
+                    const bool last = (j + 1 == n_kt);
+                    const uint32_t ph = static_cast<uint32_t>(tiles + j) & 1u;
+                    ok = mbar_wait(bar_kv_full(slot_of(tv)), par_of(tv), abort_flag, &g_attn_err, kDevErrTimeout);
+                    if (ok) check_item(tv);
+                    if (ok && !last)
+                        ok = mbar_wait(bar_kv_full(slot_of(tk)), par_of(tk), abort_flag, &g_attn_err, kDevErrTimeout);
+                    if (ok && !last) check_item(tk);
+                    if (ok && !last) {
+                        ok = mbar_wait(bar_s_free(0), ph, abort_flag, &g_attn_err, kDevErrTimeout);
+                        if (ok) {
+                            tc_fence_after_sync();
+                            issue_qk(0, tk);
+                            umma_commit(bar_s_full(0));
+                        }
+                    }
+                    ok = ok && pv_tile(0, tv, j);
+                    if (!ok) break;
+                    umma_commit(bar_pv_done(0));
+                    if (!last) {
+                        ok = mbar_wait(bar_s_free(1), ph, abort_flag, &g_attn_err, kDevErrTimeout);
+                        if (!ok) break;
+                        tc_fence_after_sync();
+                        issue_qk(1, tk);
+                        umma_commit(bar_s_full(1));
+                        if (j + 2 == n_kt) umma_commit(bar_q_empty);   // the unit's last reads of Q
+                        umma_commit(bar_kv_empty(slot_of(tk)));
+                    }
+                    ok = pv_tile(1, tv, j);
+                    if (!ok) break;
+                    umma_commit(bar_pv_done(1));
+                    umma_commit(bar_kv_empty(slot_of(tv)));
+                }
+              } else if constexpr (NQ == 2) {
+                if (ok) ok = mbar_wait(bar_kv_full(slot_of(0)), par_of(0), abort_flag, &g_attn_err, kDevErrTimeout);
+                if (ok) check_item(0);
                 if (ok) {
                     tc_fence_after_sync();
                     issue_qk(0, 0);
@@ -468,8 +541,10 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
                     const bool last = (j + 1 == n_kt);
                     // operands first (normally long landed), so only the P waits sit on the chain
                     ok = mbar_wait(bar_kv_full(slot_of(tv)), par_of(tv), abort_flag, &g_attn_err, kDevErrTimeout);
+                    if (ok) check_item(tv);
                     if (ok && !last)
                         ok = mbar_wait(bar_kv_full(slot_of(tk)), par_of(tk), abort_flag, &g_attn_err, kDevErrTimeout);
+                    if (ok && !last) check_item(tk);
                     ok = ok && pv_tile(0, tv, j);
                     if (!ok) break;
                     if (last) umma_commit(bar_o_done(0));
@@ -494,7 +569,10 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
                 constexpr uint32_t kIdescPVh = umma_idesc_bf16_f32(kBM, 128, true);
                 const uint32_t tOq = tmem + 256u;
                 auto wait_item = [&](int it) {
-                    return mbar_wait(bar_kv_full(slot_of(it)), par_of(it), abort_flag, &g_attn_err, kDevErrTimeout);
+                    const bool got =
+                        mbar_wait(bar_kv_full(slot_of(it)), par_of(it), abort_flag, &g_attn_err, kDevErrTimeout);
+                    if (got) check_item(it);
+                    return got;
                 };
                 // S(j) into buffer j % 2, K_j in two half entries (columns 0-127, 128-255)
                 auto qk = [&](int j) {
@@ -575,6 +653,7 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t tS_q = tmem + (q ? 128u : 0u) + lane_off;
         const uint32_t tO = tmem + 256u + (q ? static_cast<uint32_t>(D) : 0u) + lane_off;
+        const uint32_t tP_q = kSplitP ? tmem + (q ? 448u : 384u) + lane_off : tS_q;
         const int head_local = r / P;
         const long off = static_cast<long>(p.Lk) - static_cast<long>(p.Lq);
         const long lk1 = static_cast<long>(p.Lk) - 1;
@@ -623,10 +702,28 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
                 tmem_ld_32x32b_x32(tS + 96, sr + 96);
                 tmem_wait_ld();
                 reg_fence<128>(sr);
+                if constexpr (kSplitP) {   // S_q is in registers: the next Q K^T may overwrite it
+                    tc_fence_before_sync();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(bar_s_free(q));
+                }
+                // (split P) O_q += P_q(j-1) V_{j-1} must have completed before O_q is
+                // rescaled or P_q(j) overwrites P_q(j-1)
+                bool pv_prev_done = !kSplitP || j == 0;
+                auto wait_pv_prev = [&]() {
+                    if (pv_prev_done) return true;
+                    pv_prev_done = true;
+                    if (!mbar_wait(bar_pv_done(q), static_cast<uint32_t>(tiles + j - 1) & 1u, abort_flag,
+                                   &g_attn_err, kDevErrTimeout))
+                        return false;
+                    tc_fence_after_sync();
+                    return true;
+                };
                 float sv[kBN];
 #pragma unroll
                 for (int c = 0; c < kBN; ++c) sv[c] = __uint_as_float(sr[c]);
                 const long key0 = static_cast<long>(j) * kBN;
+                ATTN_CHECK(key0 < p.Lk);
                 const bool masked = key0 + kBN - 1 > tile_min_bound;
                 if (masked) {
                     // diagonal or ragged tile: mask keys beyond this row's bound
@@ -656,6 +753,10 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
                 // rescale O_q in TMEM if any row of this warp raised its max (O holds
                 // the sum over tiles < j, settled: see the file comment)
                 if (j > 0 && __any_sync(0xffffffffu, factor != 1.0f)) {
+                    if (!wait_pv_prev()) {
+                        ok = false;
+                        break;
+                    }
                     if constexpr (NQ == 1) {
                         // O += P(j-1) V_{j-1} must have landed (at most one P.V is outstanding)
                         if (!mbar_wait(bar_o_done(1), static_cast<uint32_t>(j - 1) & 1u, abort_flag, &g_attn_err,
@@ -710,12 +811,16 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
                         pk[i] = pack_bf16x2(e0, e1);
                         acc_e[i & 1] = f2_add(acc_e[i & 1], e);
                     }
-                    tmem_st_32x32b_x32(tS + hf * 32, pk);
+                    tmem_st_32x32b_x32((kSplitP ? tP_q : tS) + hf * 32, pk);
                     tmem_wait_st();
                     tc_fence_before_sync();
                     __syncwarp();   // every lane's P is in TMEM: one arrival for the warp
                     if (lane == 0) mbar_arrive(hf == 0 ? bar_p_half(buf) : bar_p_full(buf));
                 };
+                if (!wait_pv_prev()) {
+                    ok = false;
+                    break;
+                }
                 if (masked) {
                     exp_half(std::true_type{}, 0);
                     exp_half(std::true_type{}, 1);
@@ -744,13 +849,17 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
             // per store (positions past Lq are clipped by TMA); LSE per row ----
             bool have_o = ok && n_kt > 0;
             if (have_o) {
-                have_o = mbar_wait(bar_o_done(q), static_cast<uint32_t>(nu) & 1u, abort_flag, &g_attn_err,
-                                   kDevErrTimeout);
+                // the unit's last P.V has completed: o_done, or (split P) its pv_done
+                have_o = kSplitP ? mbar_wait(bar_pv_done(q), static_cast<uint32_t>(tiles + n_kt - 1) & 1u,
+                                             abort_flag, &g_attn_err, kDevErrTimeout)
+                                 : mbar_wait(bar_o_done(q), static_cast<uint32_t>(nu) & 1u, abort_flag, &g_attn_err,
+                                             kDevErrTimeout);
                 ok = have_o;
                 tc_fence_after_sync();
             }
             const float inv_l = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
             const int q_head0 = u.b * p.Hq + u.g * p.G;
+            ATTN_CHECK(tile_p0 >= 0 && q_head0 >= 0 && q_head0 + p.G <= p.B * p.Hq);
             auto o_cols = [&](int c, uint32_t* ob) {   // 32 columns from c, packed into 16 words
                 uint32_t orr[32];
                 if (have_o) {
@@ -811,6 +920,7 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
                     tma_store_commit();
                 }
             }
+            ATTN_CHECK(!row_valid || (h >= 0 && h < p.Hq && pos >= 0 && pos < p.Lq));
             if (row_valid && p.lse != nullptr) {
                 const float lse = (l_exact > 0.0f) ? (m_run + __log2f(l_exact)) * kLn2 : -INFINITY;
                 p.lse[(static_cast<size_t>(u.b) * p.Hq + h) * p.Lq + pos] = lse;

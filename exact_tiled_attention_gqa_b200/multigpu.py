@@ -58,21 +58,63 @@ def shard_seqlens(seqlens: torch.Tensor, rows: range) -> torch.Tensor:
     return (seqlens.to(torch.int64) - rows.start).clamp(0, len(rows)).to(torch.int32)
 
 
-def decode_kv_parallel(q: torch.Tensor, k_shard: torch.Tensor, v_shard: torch.Tensor, seqlens_shard: torch.Tensor,
-                       group=None, partial_fn=None, merge_fn=None):
-    """One new token per sequence against a cache split by rows over the ranks of `group`.
+class KVParallelDecode:
+    """Decode with the cache split by rows over the ranks of `group` (KV parallelism).
 
-    q [B,Hq,D] (the same on every rank); k_shard / v_shard [B,Hkv,rows,D] this rank's rows;
-    seqlens_shard int32 [B] the valid rows of each sequence in this shard (shard_seqlens).
-    Every rank returns the full result (out [B,Hq,D] bf16, lse [B,Hq]).  partial_fn / merge_fn
-    default to the library's attn_decode_partial / attn_decode_merge.
+    Every rank holds a contiguous share of each sequence's cached rows
+    (kv_shard_rows / shard_seqlens) and the same query rows.  One step:
+      1. attention over this rank's rows (attn_decode_partial), written straight
+         into this rank's slice of the exchange buffers;
+      2. an all-gather of the fp32 partials (B * Hq * (D + 1) * 4 bytes per rank);
+      3. the log-sum-exp merge of all ranks' partials (attn_decode_merge).
+    Every rank ends with the full result.  The buffers are allocated once, so a
+    step allocates nothing and every rank makes the same collective calls in the
+    same order.  partial_fn(q, k, v, seqlens, o_out, lse_out) and
+    merge_fn(o_all, lse_all, out, lse) default to the library's kernels; the
+    tests substitute the fp64 oracle to check the exchange on CPU ranks.
     """
-    import torch.distributed as dist
-    from . import decode_merge, decode_partial
-    o, lse = (partial_fn or decode_partial)(q, k_shard, v_shard, seqlens_shard)
-    world = dist.get_world_size(group)
-    o_all = [torch.empty_like(o) for _ in range(world)]
-    l_all = [torch.empty_like(lse) for _ in range(world)]
-    dist.all_gather(o_all, o.contiguous(), group=group)
-    dist.all_gather(l_all, lse.contiguous(), group=group)
-    return (merge_fn or decode_merge)(torch.stack(o_all), torch.stack(l_all))
+
+    def __init__(self, q: torch.Tensor, k_shard: torch.Tensor, v_shard: torch.Tensor, seqlens_shard: torch.Tensor,
+                 *, scale=None, group=None, partial_fn=None, merge_fn=None, workspace=None):
+        import torch.distributed as dist
+        B, Hq, D = q.shape
+        self.q, self.k, self.v, self.sl = q, k_shard, v_shard, seqlens_shard
+        self.scale, self.group = scale, group
+        self.distributed = dist.is_available() and dist.is_initialized()
+        self.world = dist.get_world_size(group) if self.distributed else 1
+        self.rank = dist.get_rank(group) if self.distributed else 0
+        self.o_all = torch.empty((self.world, B, Hq, D), dtype=torch.float32, device=q.device)
+        self.lse_all = torch.empty((self.world, B, Hq), dtype=torch.float32, device=q.device)
+        self.out = torch.empty((B, Hq, D), dtype=q.dtype, device=q.device)
+        self.lse = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+        self.workspace = workspace
+        self._partial = partial_fn or self._library_partial
+        self._merge = merge_fn or self._library_merge
+
+    def _library_partial(self, q, k, v, sl, o_out, lse_out):
+        from . import decode_partial
+        decode_partial(q, k, v, sl, scale=self.scale, o_part=o_out, lse_part=lse_out, workspace=self.workspace)
+
+    def _library_merge(self, o_all, lse_all, out, lse):
+        from . import decode_merge
+        decode_merge(o_all, lse_all, out=out, lse=lse)
+
+    def step(self):
+        """One decode step; returns (out [B,Hq,D], lse [B,Hq]) -- buffers reused by the next step."""
+        import torch.distributed as dist
+        self._partial(self.q, self.k, self.v, self.sl, self.o_all[self.rank], self.lse_all[self.rank])
+        if self.world > 1:
+            dist.all_gather(list(self.o_all.unbind(0)), self.o_all[self.rank], group=self.group)
+            dist.all_gather(list(self.lse_all.unbind(0)), self.lse_all[self.rank], group=self.group)
+        self._merge(self.o_all, self.lse_all, self.out, self.lse)
+        return self.out, self.lse
+
+
+def decode_kv_parallel(q: torch.Tensor, k_shard: torch.Tensor, v_shard: torch.Tensor, seqlens_shard: torch.Tensor,
+                       group=None, partial_fn=None, merge_fn=None, scale=None):
+    """One new token per sequence against a cache split by rows over the ranks of `group`:
+    one KVParallelDecode step.  q [B,Hq,D] (the same on every rank); k_shard / v_shard
+    [B,Hkv,rows,D] this rank's rows; seqlens_shard int32 [B] the valid rows of each sequence
+    in this shard (shard_seqlens).  Every rank returns the full result (out, lse)."""
+    return KVParallelDecode(q, k_shard, v_shard, seqlens_shard, scale=scale, group=group, partial_fn=partial_fn,
+                            merge_fn=merge_fn).step()

@@ -460,6 +460,9 @@ const char* attn_last_error(void);
 #define ATTN_DEVERR_PAGE    0x4u  /* a block_table entry was outside [0, n_pages) */
 #define ATTN_DEVERR_SCHED   0x8u  /* a prefill launch shared its scheduling counters with another
                                      launch running at the same time (see attn_prefill) */
+#define ATTN_DEVERR_BOUNDS  0x10u /* only in the library built with -DATTN_DEBUG_BOUNDS=1: a work-unit
+                                     mapping, ring position, TMA coordinate or output index fell
+                                     outside its tensor (a checking build for tests) */
 
 /*
  * attn_device_error -- synchronise the current device, copy its error word
