@@ -27,8 +27,8 @@ import torch
 from . import _native
 from ._native import AttnError
 
-__all__ = ["prefill", "prefill_host", "decode", "decode_partial", "decode_merge", "decode_mq", "decode_paged", "decode_noalloc", "decode_kv8",
-           "decode_kv8_paged", "prefill_host_scratch_size", "decode_workspace_size", "decode_mq_workspace_size",
+__all__ = ["prefill", "prefill_host", "decode", "decode_partial", "decode_merge", "decode_merge_peers", "kvp_signal",
+           "kvp_wait", "decode_mq", "decode_paged", "decode_noalloc", "decode_kv8", "decode_kv8_paged", "prefill_host_scratch_size", "decode_workspace_size", "decode_mq_workspace_size",
            "decode_kv8_workspace_size", "device_error", "AttnError", "library_path"]
 
 
@@ -242,6 +242,52 @@ def decode_merge(o_parts: torch.Tensor, lse_parts: torch.Tensor, *, out: Optiona
         st = _native.lib().attn_decode_merge(_ptr(o_parts), _ptr(lse_parts), n, rows, D, _ptr(out), _ptr(lse),
                                              _stream_handle(stream))
     _native.check(st, "attn_decode_merge")
+    return out, lse
+
+
+def _ptr_array(t: torch.Tensor, name: str) -> torch.Tensor:
+    if not isinstance(t, torch.Tensor) or not t.is_cuda or t.dtype != torch.int64 or t.dim() != 1 \
+            or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous 1-d int64 CUDA tensor of device pointers")
+    return t
+
+
+def kvp_signal(flag_ptrs: torch.Tensor, value: int, *, stream=None) -> None:
+    """Store `value` to each flag whose address is in flag_ptrs (int64 device tensor of
+    pointers), with release semantics, after this stream's earlier work is visible."""
+    _ptr_array(flag_ptrs, "flag_ptrs")
+    with torch.cuda.device(flag_ptrs.device):
+        st = _native.lib().attn_kvp_signal(_ptr(flag_ptrs), flag_ptrs.numel(), int(value) & 0xFFFFFFFF,
+                                           _stream_handle(stream))
+    _native.check(st, "attn_kvp_signal")
+
+
+def kvp_wait(flags: torch.Tensor, value: int, *, stream=None) -> None:
+    """Make the stream wait until every flag (uint32 storage, given as an int32 tensor) has reached `value`."""
+    _check_tensor("flags", flags, torch.int32, 1)
+    with torch.cuda.device(flags.device):
+        st = _native.lib().attn_kvp_wait(_ptr(flags), flags.numel(), int(value) & 0xFFFFFFFF,
+                                         _stream_handle(stream))
+    _native.check(st, "attn_kvp_wait")
+
+
+def decode_merge_peers(o_ptrs: torch.Tensor, lse_ptrs: torch.Tensor, ready: torch.Tensor, value: int, rows: int,
+                       D: int, *, out: torch.Tensor, lse: Optional[torch.Tensor] = None, stream=None):
+    """decode_merge over parts that stay where they were computed: part p's O at o_ptrs[p]
+    ([rows, D] fp32) and LSE at lse_ptrs[p] ([rows]), read once ready[p] has reached `value`."""
+    _ptr_array(o_ptrs, "o_ptrs")
+    _ptr_array(lse_ptrs, "lse_ptrs")
+    _check_tensor("ready", ready, torch.int32, 1)
+    if o_ptrs.numel() != lse_ptrs.numel() or ready.numel() != o_ptrs.numel():
+        raise ValueError("o_ptrs, lse_ptrs and ready must have one entry per part")
+    _check_tensor("out", out, torch.bfloat16, out.dim())
+    if out.numel() != rows * D or (lse is not None and lse.numel() != rows):
+        raise ValueError("out must hold rows * D values and lse rows values")
+    with torch.cuda.device(out.device):
+        st = _native.lib().attn_decode_merge_peers(_ptr(o_ptrs), _ptr(lse_ptrs), _ptr(ready), int(value) & 0xFFFFFFFF,
+                                                   o_ptrs.numel(), rows, D, _ptr(out), _ptr(lse),
+                                                   _stream_handle(stream))
+    _native.check(st, "attn_decode_merge_peers")
     return out, lse
 
 

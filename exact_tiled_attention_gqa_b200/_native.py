@@ -43,6 +43,9 @@ SIGNATURES = {
     "attn_decode": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _sz, _vp]),
     "attn_decode_partial": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _sz, _vp]),
     "attn_decode_merge": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp]),
+    "attn_kvp_signal": (_i32, [_vp, _i32, ctypes.c_uint, _vp]),
+    "attn_kvp_wait": (_i32, [_vp, _i32, ctypes.c_uint, _vp]),
+    "attn_decode_merge_peers": (_i32, [_vp, _vp, _vp, ctypes.c_uint, _i32, _i32, _i32, _vp, _vp, _vp]),
     "attn_decode_mq_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32]),
     "attn_decode_mq": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _sz,
                               _vp]),

@@ -746,6 +746,45 @@ extern "C" int attn_decode_merge(const float* o_parts, const float* lse_parts, i
     return st == ATTN_OK ? ok() : st;
 }
 
+extern "C" int attn_kvp_signal(unsigned int* const* flag_ptrs, int n, unsigned int value, void* stream) {
+    if (n < 0 || (n > 0 && !flag_ptrs)) return fail(ATTN_ERR_INVALID_ARG, "bad flag pointer array");
+    if (n == 0) return ok();
+    attn_kvp_signal_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(flag_ptrs, n, value);
+    const int st = check_launch("attn_kvp_signal_kernel");
+    return st == ATTN_OK ? ok() : st;
+}
+
+extern "C" int attn_kvp_wait(const unsigned int* flags, int n, unsigned int value, void* stream) {
+    if (n < 0 || (n > 0 && !flags) || (reinterpret_cast<uintptr_t>(flags) & 3u))
+        return fail(ATTN_ERR_INVALID_ARG, "bad flags array");
+    if (n == 0) return ok();
+    attn_kvp_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(flags, n, value);
+    const int st = check_launch("attn_kvp_wait_kernel");
+    return st == ATTN_OK ? ok() : st;
+}
+
+extern "C" int attn_decode_merge_peers(const float* const* o_ptrs, const float* const* lse_ptrs,
+                                       const unsigned int* ready, unsigned int value, int n_parts, int rows, int D,
+                                       void* out, float* lse, void* stream) {
+    if (n_parts < 1 || rows < 0) return fail(ATTN_ERR_INVALID_ARG, "n_parts must be >= 1 and rows >= 0");
+    if (D != 64 && D != 128 && D != 256) return fail(ATTN_ERR_UNSUPPORTED, "head dim D=%d (built: 64, 128, 256)", D);
+    if (rows == 0) return ok();
+    if (!o_ptrs || !lse_ptrs || !ready || !out) return fail(ATTN_ERR_INVALID_ARG, "null pointer array, flags or out");
+    if (!aligned16(out) || (reinterpret_cast<uintptr_t>(ready) & 3u) || (lse && (reinterpret_cast<uintptr_t>(lse) & 3u)))
+        return fail(ATTN_ERR_INVALID_ARG, "out must be 16-byte aligned, ready and lse 4-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const unsigned grid = static_cast<unsigned>((rows + 3) / 4);
+    auto* o = static_cast<__nv_bfloat16*>(out);
+    if (D == 256)
+        attn_decode_merge_peers_kernel<256><<<grid, 128, 0, s>>>(o_ptrs, lse_ptrs, ready, value, n_parts, rows, o, lse);
+    else if (D == 128)
+        attn_decode_merge_peers_kernel<128><<<grid, 128, 0, s>>>(o_ptrs, lse_ptrs, ready, value, n_parts, rows, o, lse);
+    else
+        attn_decode_merge_peers_kernel<64><<<grid, 128, 0, s>>>(o_ptrs, lse_ptrs, ready, value, n_parts, rows, o, lse);
+    const int st = check_launch("attn_decode_merge_peers_kernel");
+    return st == ATTN_OK ? ok() : st;
+}
+
 namespace attn {
 namespace {
 __global__ void exp2_fma_selftest_kernel(const float* x, float* y, int n) {

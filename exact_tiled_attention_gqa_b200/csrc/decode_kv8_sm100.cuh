@@ -697,28 +697,47 @@ __global__ void __launch_bounds__(kDecThreads, kv8t_min_blocks<NR>())
         }
         // ---- O^T += V^T P^T ----
         // cache rows past the valid length may hold anything (NaN codes or scales included)
-        const bool k0v = !tail || key_lo < k_end, k8v = !tail || key_hi < k_end;
         const int vk = key_off + 2 * tq;           // this lane's V rows: vk, vk+1, vk+8, vk+9
         const int vabs = tile_key0 + 2 * tq;
         const bool v0 = !tail || vabs < k_end, v1 = !tail || vabs + 1 < k_end;
         const bool v8 = !tail || vabs + 8 < k_end, v9 = !tail || vabs + 9 < k_end;
-        uint32_t pb[NR][2];   // P^T B fragments (E4M3: one set for all column blocks)
-        if constexpr (FMT == kKvFmtE4M3) {
+        // P^T B fragments, transposed once per tile: after the transpose this lane
+        // holds cache rows vk, vk + 1 (fragment 0) and vk + 8, vk + 9 (fragment 1),
+        // the rows whose V codes it loads.  q8_0 scales P per row and column
+        // block, so each block multiplies the fragments by those rows' V scales.
+        uint32_t pt[NR][2];
 #pragma unroll
-            for (int j = 0; j < NR; ++j) {
-                pb[j][0] = movmatrix_trans(pack_f16x2(sacc[j][0], sacc[j][1]));
-                pb[j][1] = movmatrix_trans(pack_f16x2(sacc[j][2], sacc[j][3]));
-            }
+        for (int j = 0; j < NR; ++j) {
+            pt[j][0] = movmatrix_trans(pack_f16x2(sacc[j][0], sacc[j][1]));
+            pt[j][1] = movmatrix_trans(pack_f16x2(sacc[j][2], sacc[j][3]));
         }
+        // q8_0: the V scales of those rows, one word (two blocks) at a time; zero for
+        // rows past the valid length (their scales may be NaN)
+        const uint32_t* vsw = reinterpret_cast<const uint32_t*>(vs_tile);
+        uint32_t w0s = 0u, w1s = 0u, w8s = 0u, w9s = 0u;
+        uint32_t pb[NR][2];
 #pragma unroll
         for (int c = 0; c < kBlk; ++c) {
             if constexpr (FMT == kKvFmtQ8_0) {
-                const float s_lo = k0v ? __half2float(vs_tile[(key_off + grp) * kBlk + c]) : 0.0f;
-                const float s_hi = k8v ? __half2float(vs_tile[(key_off + grp + 8) * kBlk + c]) : 0.0f;
+                if ((c & 1) == 0) {
+                    constexpr int kW = kBlk / 2;   // scale words per row
+                    w0s = v0 ? vsw[vk * kW + (c >> 1)] : 0u;
+                    w1s = v1 ? vsw[(vk + 1) * kW + (c >> 1)] : 0u;
+                    w8s = v8 ? vsw[(vk + 8) * kW + (c >> 1)] : 0u;
+                    w9s = v9 ? vsw[(vk + 9) * kW + (c >> 1)] : 0u;
+                }
+                const uint32_t sel = (c & 1) ? 0x7632u : 0x5410u;
+                const uint32_t s01 = prmt(w0s, w1s, sel), s89 = prmt(w8s, w9s, sel);
 #pragma unroll
                 for (int j = 0; j < NR; ++j) {
-                    pb[j][0] = movmatrix_trans(pack_f16x2(sacc[j][0] * s_lo, sacc[j][1] * s_lo));
-                    pb[j][1] = movmatrix_trans(pack_f16x2(sacc[j][2] * s_hi, sacc[j][3] * s_hi));
+                    pb[j][0] = hmul2(pt[j][0], s01);
+                    pb[j][1] = hmul2(pt[j][1], s89);
+                }
+            } else {
+#pragma unroll
+                for (int j = 0; j < NR; ++j) {
+                    pb[j][0] = pt[j][0];
+                    pb[j][1] = pt[j][1];
                 }
             }
             const int col = c * 32 + 4 * grp;

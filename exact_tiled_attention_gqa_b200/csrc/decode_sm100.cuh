@@ -513,4 +513,107 @@ __global__ void __launch_bounds__(128)
     if (lse != nullptr && lane == 0) lse[row] = (Lsum > 0.0f) ? M + __logf(Lsum) : -INFINITY;
 }
 
+// ---------------------------------------------------------------------------
+// KV parallelism with the exchange fused into the merge.  Each GPU writes its
+// partial results into its own memory; the merge on every GPU then reads all
+// parts where they lie (plain loads: this GPU's memory, or a peer's over
+// NVLink), instead of first copying them with an all-gather.  Flags order the
+// steps, each a 32-bit epoch counter compared wraparound-safely:
+//   ready[p]    part p is complete (set by part p's GPU after its partial)
+//   consumed[p] GPU p has finished reading every part of that epoch (set after
+//               its merge), so a part's buffer may be overwritten next epoch.
+// Every wait is bounded: after kWaitLimitNs it sets ATTN_DEVERR_TIMEOUT and the
+// kernel skips its work instead of hanging.
+// ---------------------------------------------------------------------------
+
+__device__ __forceinline__ uint32_t ld_acquire_sys(const unsigned int* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ void st_release_sys(unsigned int* p, uint32_t v) {
+    asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+// flag has reached `value` (epochs only grow; compared modulo 2^32)
+__device__ __forceinline__ bool epoch_reached(uint32_t flag, uint32_t value) {
+    return static_cast<int32_t>(flag - value) >= 0;
+}
+
+// One thread waits until flags[0 .. n) have all reached `value`; false after the time limit.
+__device__ __forceinline__ bool wait_flags(const unsigned int* flags, int n, uint32_t value) {
+    const uint64_t t0 = global_timer_ns();
+    for (int i = 0; i < n; ++i) {
+        while (!epoch_reached(ld_acquire_sys(flags + i), value)) {
+            if (global_timer_ns() - t0 > kWaitLimitNs) {
+                atomicOr(&g_attn_err, kDevErrTimeout);
+                return false;
+            }
+            __nanosleep(64);
+        }
+    }
+    return true;
+}
+
+// flag_ptrs[i] <- value for i < n, after everything this GPU wrote before this
+// kernel (in stream order) is visible system-wide.
+__global__ void attn_kvp_signal_kernel(unsigned int* const* flag_ptrs, int n, uint32_t value) {
+    __threadfence_system();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) st_release_sys(flag_ptrs[i], value);
+}
+
+__global__ void attn_kvp_wait_kernel(const unsigned int* flags, int n, uint32_t value) {
+    if (threadIdx.x == 0) wait_flags(flags, n, value);
+}
+
+// attn_decode_merge_kernel over parts reached through pointers: part p's O at
+// o_ptrs[p] ([rows][D] fp32) and LSE at lse_ptrs[p] ([rows]), read only after
+// ready[p] has reached `value`.
+template <int D>
+__global__ void __launch_bounds__(128)
+    attn_decode_merge_peers_kernel(const float* const* o_ptrs, const float* const* lse_ptrs,
+                                   const unsigned int* ready, uint32_t value, int n_parts, int rows,
+                                   __nv_bfloat16* out, float* lse) {
+    __shared__ int go;
+    if (threadIdx.x == 0) go = wait_flags(ready, n_parts, value) ? 1 : 0;
+    __syncthreads();
+    if (!go) return;
+    const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= rows) return;
+    constexpr int kPer = D / 32;
+    float M = -INFINITY;
+    // parts are read at L2 (.cg): the same addresses held last epoch's values
+    for (int q = lane; q < n_parts; q += 32) M = fmaxf(M, __ldcg(lse_ptrs[q] + row));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float acc[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) acc[i] = 0.0f;
+    float Lsum = 0.0f;
+    for (int q0 = 0; q0 < n_parts; q0 += 32) {
+        const int q = q0 + lane;
+        const float ls = (q < n_parts) ? __ldcg(lse_ptrs[q] + row) : -INFINITY;
+        const float wl = (ls == -INFINITY) ? 0.0f : ex2_approx((ls - M) * kLog2e);
+        Lsum += wl;
+        const int cnt = min(32, n_parts - q0);
+        for (int i = 0; i < cnt; ++i) {
+            const float w = __shfl_sync(0xffffffffu, wl, i);
+            const float* src = o_ptrs[q0 + i] + static_cast<size_t>(row) * D + lane * kPer;
+#pragma unroll
+            for (int c = 0; c < kPer; c += 2) {
+                const float2 v = __ldcg(reinterpret_cast<const float2*>(src + c));
+                acc[c] = fmaf(w, v.x, acc[c]);
+                acc[c + 1] = fmaf(w, v.y, acc[c + 1]);
+            }
+        }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, o);
+    const float inv = (Lsum > 0.0f) ? 1.0f / Lsum : 0.0f;
+    __nv_bfloat16* o = out + static_cast<size_t>(row) * D + lane * kPer;
+#pragma unroll
+    for (int i = 0; i < kPer; i += 2) *reinterpret_cast<uint32_t*>(o + i) = pack_bf16x2(acc[i] * inv, acc[i + 1] * inv);
+    if (lse != nullptr && lane == 0) lse[row] = (Lsum > 0.0f) ? M + __logf(Lsum) : -INFINITY;
+}
+
 }  // namespace attn

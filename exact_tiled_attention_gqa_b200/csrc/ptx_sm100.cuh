@@ -420,6 +420,13 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
     return r;
 }
 
+// packed f16x2 product, round to nearest even
+__device__ __forceinline__ uint32_t hmul2(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
 // two fp32 -> packed f16x2 (lo in bits 0-15), round to nearest even
 __device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
     uint32_t r;

@@ -219,6 +219,46 @@ int attn_decode_merge(const float* o_parts, const float* lse_parts, int n_parts,
                       void* out, float* lse, void* stream);
 
 /*
+ * attn_kvp_signal / attn_kvp_wait / attn_decode_merge_peers -- the same KV
+ * parallelism with the exchange fused into the merge: each device leaves its
+ * attn_decode_partial results in its own memory, and the merge on every device
+ * reads all parts where they lie -- its own memory or a peer's, over NVLink,
+ * with plain loads -- instead of all-gathering them first.  Epoch flags order
+ * the steps; an epoch is a 32-bit counter that grows by one per step, and a
+ * flag "has reached" a value when (int32_t)(flag - value) >= 0.
+ *
+ * One step, epoch e, on device r of n (ready and consumed are n-entry uint32
+ * arrays in device r's memory, zero before the first step):
+ *   1. attn_kvp_wait(consumed, n, e - 1)   (steps after the first) -- every
+ *      device has finished reading this device's previous parts
+ *   2. attn_decode_partial into this device's part buffers
+ *   3. attn_kvp_signal({&ready_on_device_p[r] for p < n}, n, e)
+ *   4. attn_decode_merge_peers(o_ptrs, lse_ptrs, ready, e, n, ...)
+ *   5. attn_kvp_signal({&consumed_on_device_p[r] for p < n}, n, e)
+ * all on one stream.  Every pointer must be valid in the calling process
+ * (peer memory mapped into it, e.g. through CUDA IPC or symmetric memory).
+ *
+ * attn_kvp_signal: after everything enqueued before it on `stream` is visible
+ *   system-wide, stores `value` to *flag_ptrs[i] (i < n) with release
+ *   semantics.  flag_ptrs: device array of n device pointers.
+ * attn_kvp_wait: makes `stream` wait until flags[0 .. n) (device array) have
+ *   all reached `value`.
+ * attn_decode_merge_peers: attn_decode_merge with part p's O at o_ptrs[p]
+ *   ([rows, D] fp32) and its LSE at lse_ptrs[p] ([rows] fp32, natural log),
+ *   device arrays of n_parts pointers; each CTA first waits until ready[0 ..
+ *   n_parts) have reached `value`.  out [rows, D] bf16 16-byte aligned, lse
+ *   [rows] fp32 or NULL.
+ * Every wait gives up after about 2 s, sets ATTN_DEVERR_TIMEOUT and lets the
+ * kernel end (the merge then leaves out and lse unwritten).  Errors:
+ * ATTN_ERR_INVALID_ARG, ATTN_ERR_UNSUPPORTED (D), ATTN_ERR_CUDA; n == 0 or
+ * rows == 0 returns ATTN_OK.
+ */
+int attn_kvp_signal(unsigned int* const* flag_ptrs, int n, unsigned int value, void* stream);
+int attn_kvp_wait(const unsigned int* flags, int n, unsigned int value, void* stream);
+int attn_decode_merge_peers(const float* const* o_ptrs, const float* const* lse_ptrs, const unsigned int* ready,
+                            unsigned int value, int n_parts, int rows, int D, void* out, float* lse, void* stream);
+
+/*
  * attn_decode_mq_workspace_size -- bytes of scratch attn_decode_mq needs for
  * these sizes.  Depends only on the arguments; 0 for sizes it would reject.
  */

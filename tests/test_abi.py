@@ -241,3 +241,14 @@ def test_diagnostics_reject(lib):
     assert lib.attn_selftest_wait(1000, NULL, None) == -1
     assert lib.attn_selftest_wait(3_000_000_000, A, None) == -1
     assert lib.attn_prefill_sched_busy(None) == -1
+
+
+def test_fused_merge_calls_reject(lib):
+    assert lib.attn_kvp_signal(NULL, 2, 1, None) == -1
+    assert lib.attn_kvp_signal(NULL, 0, 1, None) == 0
+    assert lib.attn_kvp_wait(NULL, 2, 1, None) == -1
+    assert lib.attn_kvp_wait(ctypes.c_void_p(0x10002), 2, 1, None) == -1
+    f = lambda **kw: lib.attn_decode_merge_peers(*[kw.get(n, d) for n, d in (
+        ("o", A), ("l", A), ("r", A), ("v", 1), ("n", 2), ("rows", 8), ("D", 128), ("out", A), ("lse", NULL))], None)
+    assert f(n=0) == -1 and f(rows=-1) == -1 and f(D=96) == -2 and f(rows=0) == 0
+    assert f(o=NULL) == -1 and f(r=NULL) == -1 and f(out=ctypes.c_void_p(0x10008)) == -1
