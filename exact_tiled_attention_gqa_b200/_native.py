@@ -60,7 +60,6 @@ SIGNATURES = {
     "attn_decode_kv8_paged": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32,
                                      _i32, _i32, _i32, _f32, _vp, _sz, _vp]),
     "attn_selftest_kv8_convert": (_i32, [_vp, _vp, _i32, _i32, _vp]),
-    "attn_selftest_exp2": (_i32, [_vp, _vp, _i32, _vp]),
     "attn_selftest_wait": (_i32, [ctypes.c_ulonglong, _vp, _vp]),
     "attn_prefill_sched_busy": (_i32, [ctypes.POINTER(_i32)]),
     "attn_status_string": (ctypes.c_char_p, [_i32]),

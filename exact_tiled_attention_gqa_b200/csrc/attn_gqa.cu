@@ -230,26 +230,32 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
 // Cache rows per decode split (always a multiple of 64, the tile height).
 //  - mma.sync split kernel: the largest power of two in [256, 4096] that still
 //    gives about four waves of CTAs on a 148-SM part (1184 CTAs).
-//  - tcgen05 kernel (D = 256, or more than 16 query rows per KV head): its CTAs
+//  - tcgen05 kernel, D <= 128 (more than 16 query rows per KV head): its CTAs
 //    carry more setup than the split kernel's (TMEM, the Q tile, a partial per
 //    row for the combine), so splits are long, and the split length balances
 //    the waves: of the multiples of 64 in [512, 8192], the one that minimises
-//    waves x (rows per split + 512), with waves = splits / CTA slots rounded up
-//    (148 SMs x 2 CTAs for D <= 128, x 1 for D = 256) and the split count taken
-//    at Lmax.  At 131072 cached rows and G = 64 (8 sequences, one KV head) this
-//    gives 3584-row splits, 296 CTAs, two on every SM; 4096-row splits gave
-//    256 CTAs, so 40 SMs ran one CTA while the rest ran two.
+//    waves x (rows per split + 512), with waves = splits / (148 SMs x 2 CTAs)
+//    rounded up and the split count taken at Lmax.  Measured on B200 at 131072
+//    cached rows: G = 32 got 7296-row splits (288 CTAs, one wave) and went from
+//    0.179 to 0.169 ms against 4096-row splits (512 CTAs); G = 64 (3584-row
+//    splits, 296 CTAs) was unchanged.
+//  - tcgen05 kernel, D = 256 (one CTA per SM): the largest power of two in
+//    [512, 4096] that still gives 148 CTAs (the balanced rule above, at one CTA
+//    per SM, made the head-dim-256 decode batch 8 % slower: with lengths spread
+//    over [1024, 32768] the split count at Lmax says little about real waves).
 // The result depends only on the arguments (workspace sizes do too).
 bool decode_uses_tc(int D, int rows_per_group) { return D == 256 || rows_per_group > 16; }
 
 int decode_chunk(int B, int Hkv, int Lmax, bool tc_path, int D) {
     const long long groups = static_cast<long long>(B) * Hkv;
-    if (!tc_path) {
+    if (!tc_path || D == 256) {
+        const long long target = tc_path ? 148LL : 148LL * 2 * 4;
+        const int min_chunk = tc_path ? 512 : 256;
         int chunk = 4096;
-        while (chunk > 256 && groups * ((Lmax + chunk - 1) / chunk) < 148LL * 2 * 4) chunk >>= 1;
+        while (chunk > min_chunk && groups * ((Lmax + chunk - 1) / chunk) < target) chunk >>= 1;
         return chunk;
     }
-    const long long slots = 148LL * (D <= 128 ? 2 : 1);
+    const long long slots = 148LL * 2;
     int best = 512;
     long long best_cost = -1;
     for (int c = 512; c <= 8192; c += 64) {
@@ -785,28 +791,6 @@ extern "C" int attn_decode_merge_peers(const float* const* o_ptrs, const float* 
     return st == ATTN_OK ? ok() : st;
 }
 
-namespace attn {
-namespace {
-__global__ void exp2_fma_selftest_kernel(const float* x, float* y, int n) {
-    const int i = 2 * (blockIdx.x * blockDim.x + threadIdx.x);
-    if (i >= n) return;
-    const float x0 = x[i], x1 = (i + 1 < n) ? x[i + 1] : 0.0f;
-    float y0, y1;
-    f2_unpack(exp2_fma_x2(f2_pack(x0, x1)), y0, y1);
-    y[i] = y0;
-    if (i + 1 < n) y[i + 1] = y1;
-}
-}  // namespace
-}  // namespace attn
-
-extern "C" int attn_selftest_exp2(const float* x, float* y, int n, void* stream) {
-    if (n < 0 || (n > 0 && (!x || !y))) return fail(ATTN_ERR_INVALID_ARG, "bad selftest arguments");
-    if (n == 0) return ok();
-    const int threads = 256, pairs = (n + 1) / 2;
-    exp2_fma_selftest_kernel<<<(pairs + threads - 1) / threads, threads, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
-    const int st = check_launch("exp2_fma_selftest_kernel");
-    return st == ATTN_OK ? ok() : st;
-}
 
 namespace attn {
 namespace {

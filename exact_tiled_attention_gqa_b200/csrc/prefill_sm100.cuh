@@ -63,11 +63,8 @@
 // arrive in two halves, in the order the MMAs use them (K0 K1 V0 K2 V1 ...),
 // and the P.V product is issued as two N = 128 halves of O.
 //
-// The exponentials of an unmasked tile can be split between the MUFU unit
-// (ex2.approx) and the FMA pipe (a cubic after range reduction, see
-// exp2_fma_x2; kExpFmaPairsPer8 below, off by default as measured).
-// Scale-and-subtract, sums and O rescales use packed f32x2 instructions,
-// maxima a 3-input max.
+// The exponentials run on the MUFU unit (ex2.approx).  Scale-and-subtract,
+// sums and O rescales use packed f32x2 instructions, maxima a 3-input max.
 //
 // Online softmax, in the log2 domain (x2 = x * scale * log2 e): per row a
 // running max m and sum l.  The max used for the exponentials is only raised
@@ -76,8 +73,6 @@
 // is the same exact quantity -- O = sum_j 2^(s2_j - m) v_j / sum_j 2^(s2_j - m)
 // holds for any m -- and the O rescale in TMEM is skipped on most tiles.
 #pragma once
-
-#include <type_traits>
 
 #include "ptx_sm100.cuh"
 #include "device_error.cuh"
@@ -95,22 +90,6 @@ static_assert(2 * kSoftmaxRegs + kControlRegs == 3 * kPrefillLaunchRegs, "regist
 constexpr int kBM = 128;               // rows per Q tile (MMA M)
 constexpr int kBN = 128;               // keys per K/V tile
 constexpr float kRescaleLog2 = 8.0f;
-// Of every 8 pairs of exponentials in an unmasked tile, this many are computed
-// on the FMA pipe (exp2_fma_x2) and the rest on the MUFU unit.  Measured on
-// B200: 0 is fastest for this kernel (the softmax is latency-bound, not MUFU
-// throughput-bound: each Q tile's softmax waits on its own S / P / MMA chain),
-// so the FMA-pipe exponential is built and tested but off by default.
-#ifndef ATTN_EXP_FMA_PAIRS_PER_8
-#define ATTN_EXP_FMA_PAIRS_PER_8 0
-#endif
-// The softmax hands P_q to the MMA thread in this many parts (2 or 4) per key
-// tile, each as soon as its exponentials are in TMEM, so that O_q += P_q V_j can
-// start on the first keys while the rest are computed (two-Q-tile kernels).
-#ifndef ATTN_P_PARTS
-#define ATTN_P_PARTS 2
-#endif
-static_assert(ATTN_P_PARTS == 2 || ATTN_P_PARTS == 4, "P is handed over in 2 or 4 parts");
-constexpr int kExpFmaPairsPer8 = ATTN_EXP_FMA_PAIRS_PER_8;
 
 template <int D>
 struct PrefillSmem {
@@ -137,8 +116,8 @@ struct PrefillSmem {
     static constexpr int kStgOff = kKVOff + kStages * kItemBytes;
     static constexpr int kBarOff = kStgOff + (kPersistent ? kNQ * kBlockBytes : 0);
     // barriers: q_full, kv_full[S], kv_empty[S], s_full[2], p_half[2], p_full[2], o_done[2], drain,
-    //           q_empty, unit_full[2], unit_empty[2], s_free[2], pv_done[2], p_mid[2][2]
-    static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 2 + 1 + 1 + 2 + 2 + 2 + 2 + 4;
+    //           q_empty, unit_full[2], unit_empty[2], s_free[2], pv_done[2]
+    static constexpr int kNumBars = 1 + 2 * kStages + 2 + 2 + 2 + 2 + 1 + 1 + 2 + 2 + 2 + 2;
     static constexpr int kMiscOff = kBarOff + kNumBars * 8;   // tmem base, abort flag, two unit slots (int each)
     static constexpr int kTagOff = kMiscOff + 16;             // debug builds: ring entry -> item index
     static constexpr int kBytes = kTagOff + 4 * kStages;
@@ -248,12 +227,8 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
     // (split P only) the softmax has read S_q into registers / O_q += P_q V has completed
     auto bar_s_free = [&](int q) { return bar0 + 8u * (15 + 2 * L::kStages + q); };
     auto bar_pv_done = [&](int q) { return bar0 + 8u * (17 + 2 * L::kStages + q); };
-    // P_q handed over in kPParts parts: part 0 on p_half, the last on p_full, the
-    // middle ones (kPParts = 4) on p_mid
-    constexpr int kPParts = (NQ == 2) ? ATTN_P_PARTS : 2;
-    auto bar_p_part = [&](int q, int i) {
-        return i == 0 ? bar_p_half(q) : i == kPParts - 1 ? bar_p_full(q) : bar0 + 8u * (18 + 2 * L::kStages + 2 * q + i);
-    };
+    // P_q (or, for NQ = 1, S buffer q's P) is handed over in two halves: keys 0-63 on p_half, 64-127 on p_full
+    auto bar_p_part = [&](int q, int half) { return half == 0 ? bar_p_half(q) : bar_p_full(q); };
     uint32_t* tmem_base_ptr = reinterpret_cast<uint32_t*>(smem + L::kMiscOff);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 4);
     volatile int* unit_slot = reinterpret_cast<volatile int*>(smem + L::kMiscOff + 8);
@@ -276,7 +251,6 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
             mbar_init(bar_unit_empty(q), kUnitReaders);
             mbar_init(bar_s_free(q), 4);   // one arrival per softmax warp
             mbar_init(bar_pv_done(q), 1);
-            for (int i = 1; i + 1 < kPParts; ++i) mbar_init(bar_p_part(q, i), 4);
         }
         mbar_init(bar_drain, 1);
         *abort_flag = 0;
@@ -455,25 +429,24 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
                 }
             };
             // O_q += P_q V : M=128, N=D, K=128 keys in steps of 16 (8 TMEM columns of P);
-            // part i of kPParts covers keys 128 i / kPParts .. (P columns 64 i / kPParts ..)
-            auto issue_pv = [&](int q, int t, bool acc, int part) {
-                constexpr int kSteps = (kBN / 16) / kPParts;
+            // `half` 0 covers keys 0-63 (P columns 0-31), half 1 keys 64-127
+            auto issue_pv = [&](int q, int t, bool acc, int half) {
                 const uint64_t b0 = dV0 + static_cast<uint64_t>(slot_of(t)) * kSlotStep;
 #pragma unroll
-                for (int k4 = 0; k4 < kSteps; ++k4) {
-                    const int kk = part * kSteps + k4;
+                for (int k4 = 0; k4 < kBN / 32; ++k4) {
+                    const int kk = half * (kBN / 32) + k4;
                     umma_ts(tO[q], tP[q] + kk * 8, b0 + static_cast<uint64_t>((kk * 2048) >> 4), kIdescPV,
                             (acc || kk > 0) ? 1u : 0u);
                 }
             };
-            // every part of O_q += P_q(j) V_j, each as soon as the softmax has released it
+            // both halves of O_q += P_q(j) V_j, each as soon as the softmax has released it
             auto pv_tile = [&](int q, int t, int j) {
                 const uint32_t ph = static_cast<uint32_t>(tiles + j) & 1u;
 #pragma unroll
-                for (int part = 0; part < kPParts; ++part) {
-                    if (!mbar_wait(bar_p_part(q, part), ph, abort_flag, &g_attn_err, kDevErrTimeout)) return false;
+                for (int half = 0; half < 2; ++half) {
+                    if (!mbar_wait(bar_p_part(q, half), ph, abort_flag, &g_attn_err, kDevErrTimeout)) return false;
                     tc_fence_after_sync();
-                    issue_pv(q, t, part > 0 || j > 0, part);
+                    issue_pv(q, t, half > 0 || j > 0, half);
                 }
                 return true;
             };
@@ -806,33 +779,19 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
                 const uint64_t sl2x2 = f2_pack(sl2, sl2);
                 const uint64_t negm2 = f2_pack(-m_sub, -m_sub);
                 uint64_t acc_e[2] = {0ull, 0ull};
-                // (NQ = 1 always uses two parts: the D = 256 MMA thread waits on p_half / p_full)
-                constexpr int kParts = (NQ == 2) ? kPParts : 2;
-                constexpr int kPairs = 64 / kParts;   // exponential pairs (P columns) per part
-                auto exp_half = [&](auto masked_tag, int hf) {
-                    constexpr bool kMasked = decltype(masked_tag)::value;
-                    uint32_t pk[kPairs];
+                auto exp_half = [&](int hf) {
+                    uint32_t pk[32];
 #pragma unroll
-                    for (int i = 0; i < kPairs; ++i) {
-                        const int c = hf * 2 * kPairs + 2 * i;
+                    for (int i = 0; i < 32; ++i) {
+                        const int c = hf * 64 + 2 * i;
                         const uint64_t t = f2_fma(f2_pack(sv[c], sv[c + 1]), sl2x2, negm2);
-                        uint64_t e;
-                        if (!kMasked && (i % 8) < kExpFmaPairsPer8) {
-                            e = exp2_fma_x2(t);
-                        } else {
-                            float t0, t1;
-                            f2_unpack(t, t0, t1);
-                            e = f2_pack(ex2_approx(t0), ex2_approx(t1));
-                        }
-                        float e0, e1;
-                        f2_unpack(e, e0, e1);
+                        float t0, t1;
+                        f2_unpack(t, t0, t1);
+                        const float e0 = ex2_approx(t0), e1 = ex2_approx(t1);
                         pk[i] = pack_bf16x2(e0, e1);
-                        acc_e[i & 1] = f2_add(acc_e[i & 1], e);
+                        acc_e[i & 1] = f2_add(acc_e[i & 1], f2_pack(e0, e1));
                     }
-                    if constexpr (kPairs == 32)
-                        tmem_st_32x32b_x32((kSplitP ? tP_q : tS) + hf * kPairs, pk);
-                    else
-                        tmem_st_32x32b_x16((kSplitP ? tP_q : tS) + hf * kPairs, pk);
+                    tmem_st_32x32b_x32((kSplitP ? tP_q : tS) + hf * 32, pk);
                     tmem_wait_st();
                     tc_fence_before_sync();
                     __syncwarp();   // every lane's P is in TMEM: one arrival for the warp
@@ -842,13 +801,8 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
                     ok = false;
                     break;
                 }
-                if (masked) {
-#pragma unroll
-                    for (int part = 0; part < kParts; ++part) exp_half(std::true_type{}, part);
-                } else {
-#pragma unroll
-                    for (int part = 0; part < kParts; ++part) exp_half(std::false_type{}, part);
-                }
+                exp_half(0);
+                exp_half(1);
                 // P reaches the MMA rounded to bf16.  O is normalised by the sum with the
                 // tile's largest P taken as rounded (its exponential is recomputed
                 // exactly as in the loop above): a key that dominates a row then has

@@ -323,39 +323,6 @@ __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
     return r;
 }
 
-// 2^t for two lanes on the FMA pipe (the MUFU unit is the softmax's scarce
-// resource).  Range reduction: j = round(t) by the 1.5 * 2^23 shift trick
-// (a round-to-nearest add leaves j in the low mantissa bits), f = t - j in
-// [-1/2, 1/2]; then 2^f ~= c0 + c1 f + c2 f^2 + c3 f^3, the cubic that
-// minimises the maximum relative error on [-1/2, 1/2] (Lawson's algorithm;
-// csrc/fit_exp2_poly.py), max relative error 7.5e-5 in fp32; finally 2^j is
-// added to the exponent field.  Valid for t in [-126, 8] (callers clamp; in
-// [-126, -125] the result nears the subnormal range and the error grows to
-// about 1.5e-4, irrelevant next to the row max's 2^0 .. 2^8);
-// masked lanes (t = -inf) must use the MUFU path, which returns exactly 0.
-constexpr float kExp2C0 = 0x1.fff692p-1f;
-constexpr float kExp2C1 = 0x1.62f31ap-1f;
-constexpr float kExp2C2 = 0x1.f0de1ap-3f;
-constexpr float kExp2C3 = 0x1.c3f760p-5f;
-constexpr float kRoundShift = 12582912.0f;   // 1.5 * 2^23
-
-__device__ __forceinline__ uint64_t exp2_fma_x2(uint64_t t) {
-    float t0, t1;
-    f2_unpack(t, t0, t1);
-    t = f2_pack(fmaxf(t0, -126.0f), fmaxf(t1, -126.0f));
-    const uint64_t shift = f2_pack(kRoundShift, kRoundShift);
-    const uint64_t tj = f2_add(t, shift);
-    const uint64_t f = f2_sub(t, f2_sub(tj, shift));
-    uint64_t p = f2_fma(f, f2_pack(kExp2C3, kExp2C3), f2_pack(kExp2C2, kExp2C2));
-    p = f2_fma(p, f, f2_pack(kExp2C1, kExp2C1));
-    p = f2_fma(p, f, f2_pack(kExp2C0, kExp2C0));
-    float p0, p1, j0, j1;
-    f2_unpack(p, p0, p1);
-    f2_unpack(tj, j0, j1);
-    return f2_pack(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(j0) << 23)),
-                   __uint_as_float(__float_as_uint(p1) + (__float_as_uint(j1) << 23)));
-}
-
 // two fp32 -> packed bf16x2 (lo in bits 0-15), round to nearest even
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     uint32_t r;

@@ -450,15 +450,6 @@ int attn_decode_kv8_paged(const void* q, const void* k_pages, const void* v_page
 int attn_selftest_kv8_convert(const uint16_t* codes, uint32_t* out, int n, int kv_format, void* stream);
 
 /*
- * attn_selftest_exp2 -- diagnostic: y[i] = the prefill softmax's FMA-pipe
- * approximation of 2^x[i] (range reduction plus a minimax cubic; relative
- * error about 7.5e-5 for x in [-125, 8], below 2e-4 for x in [-126, -125]
- * where the result nears the subnormal range; inputs below -126 are clamped
- * to -126).  x and y are device arrays of n floats; enqueued on `stream`.
- */
-int attn_selftest_exp2(const float* x, float* y, int n, void* stream);
-
-/*
  * attn_selftest_wait -- diagnostic: makes the kernels' bounded pipeline wait
  * run out, without touching any real pipeline.  One CTA of two warps: a
  * "producer" announces bytes on a barrier that never arrive (no copy is

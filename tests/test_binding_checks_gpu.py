@@ -76,5 +76,7 @@ def test_squeezed_decode_results(dev):
     o, l = attn.decode_paged(q, kp, kp, table, sl, out=out, lse=lse)
     torch.cuda.synchronize()
     assert o.data_ptr() == out.data_ptr() and l.data_ptr() == lse.data_ptr() and o.shape == q.shape
-    with pytest.raises(ValueError, match="out must have shape"):
+    with pytest.raises(ValueError, match="out must"):
         attn.decode_paged(q, kp, kp, table, sl, out=_bf(2, 8, 1, 64, dev=dev))
+    with pytest.raises(ValueError, match="out must have shape"):
+        attn.decode_paged(q, kp, kp, table, sl, out=_bf(2, 8, 64, dev=dev))
