@@ -77,15 +77,6 @@ struct DecodeTcSmem {
     static_assert(kStages >= 4, "ring too shallow");
 };
 
-// Per-SM counters that rotate where a CTA puts its query rows (see row0 below).
-__device__ unsigned int g_dtc_sm_turn[256];
-
-__device__ __forceinline__ uint32_t sm_id() {
-    uint32_t id;
-    asm volatile("mov.u32 %0, %%smid;" : "=r"(id));
-    return id;
-}
-
 template <int D>
 __global__ void __launch_bounds__(kDtcThreads, DecodeTcSmem<D>::kCtasPerSm)
     attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -104,19 +95,6 @@ __global__ void __launch_bounds__(kDtcThreads, DecodeTcSmem<D>::kCtasPerSm)
     const int n_tiles = (k_end - k_begin + kDtcBN - 1) / kDtcBN;
     const int R = p.G * p.Lq;          // query rows of the group (<= 128)
     const size_t group_row0 = (static_cast<size_t>(b) * p.Hq + static_cast<size_t>(g) * p.G) * p.Lq;
-    // The rows occupy TMEM lanes row0 .. row0 + R - 1, and lane quarter w is only
-    // reachable from warps with w = warp % 4, which run on SM sub-partition w.  When
-    // R fills at most half the tile (G >= 32 at one token), CTAs sharing an SM take
-    // turns over the free positions (a per-SM counter), so their softmax warps run
-    // on different sub-partitions instead of all on the first ones.
-    __shared__ int row0_s;
-    if (threadIdx.x == 0) {
-        const int span = R <= 32 ? 32 : R <= 64 ? 64 : 128;
-        row0_s = (span < 128) ? static_cast<int>(atomicAdd(&g_dtc_sm_turn[sm_id() & 255], 1u) % (128 / span)) * span
-                              : 0;
-    }
-    __syncthreads();
-    const int row0 = row0_s;
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t sQ = base + L::kQOff;
@@ -153,12 +131,11 @@ __global__ void __launch_bounds__(kDtcThreads, DecodeTcSmem<D>::kCtasPerSm)
     }
     // query rows R .. 127 are not loaded: make them zero (finite) for the MMA
     if (R < 128) {
+        const int pad = (128 - R) * 128;
         for (int kb = 0; kb < L::kKB; ++kb) {
-            uint8_t* blk = smem + L::kQOff + kb * L::kQBlockBytes;
-            for (int i = threadIdx.x * 16; i < 128 * 128; i += kDtcThreads * 16) {
-                const int row = i >> 7;
-                if (row < row0 || row >= row0 + R) *reinterpret_cast<uint4*>(blk + i) = make_uint4(0, 0, 0, 0);
-            }
+            uint8_t* blk = smem + L::kQOff + kb * L::kQBlockBytes + R * 128;
+            for (int i = threadIdx.x * 16; i < pad; i += kDtcThreads * 16)
+                *reinterpret_cast<uint4*>(blk + i) = make_uint4(0, 0, 0, 0);
         }
         fence_proxy_async_smem();
     }
@@ -186,8 +163,7 @@ __global__ void __launch_bounds__(kDtcThreads, DecodeTcSmem<D>::kCtasPerSm)
             tma_prefetch_desc(&tm_v);
             mbar_arrive_expect_tx(bar_q_full, static_cast<uint32_t>(L::kKB * R * 128));
             for (int kb = 0; kb < L::kKB; ++kb)
-                tma_load_3d(sQ + kb * L::kQBlockBytes + row0 * 128, &tm_q, bar_q_full, kb * 64,
-                            static_cast<int>(group_row0), 0);
+                tma_load_3d(sQ + kb * L::kQBlockBytes, &tm_q, bar_q_full, kb * 64, static_cast<int>(group_row0), 0);
             int issued = 0;
             for (int t = 0; t < n_items; ++t) {
                 const int s = slot_of(t);
@@ -307,12 +283,11 @@ __global__ void __launch_bounds__(kDtcThreads, DecodeTcSmem<D>::kCtasPerSm)
         __syncwarp();
     } else {
         // ================= softmax warpgroup (thread = row = TMEM lane) =================
-        const int lane_row = threadIdx.x;        // TMEM lane 0..127
-        const int r = lane_row - row0;           // query row of the group (valid when 0 <= r < R)
+        const int r = threadIdx.x;               // 0..127
         const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
         const uint32_t tOr = tO + lane_off;
         // keys this row may see: below min(k_end, seqlen - Lq + token + 1)
-        const int lim = min(k_end, seqlen - p.Lq + (r >= 0 ? r : 0) % p.Lq + 1);
+        const int lim = min(k_end, seqlen - p.Lq + r % p.Lq + 1);
         const int lim_lo = min(k_end, seqlen - p.Lq + 1);
         const float sl2 = p.scale_log2;
         const uint64_t sl2x2 = f2_pack(sl2, sl2);
@@ -322,7 +297,7 @@ __global__ void __launch_bounds__(kDtcThreads, DecodeTcSmem<D>::kCtasPerSm)
         // A warp whose 32 rows are all padding (row >= R) only keeps the pipeline
         // moving: its P rows are never read into a real output row (the MMA keeps
         // rows apart), so it skips the softmax and just signals.
-        const bool idle_warp = warp * 32 + 31 < row0 || warp * 32 >= row0 + R;
+        const bool idle_warp = warp * 32 >= R;
         bool ok = true;
         for (int j = 0; j < n_tiles; ++j) {
             const int buf = j & 1;
@@ -437,7 +412,7 @@ __global__ void __launch_bounds__(kDtcThreads, DecodeTcSmem<D>::kCtasPerSm)
             have_o = mbar_wait(bar_o_done, 0, abort_flag, &g_attn_err, kDevErrTimeout);
             tc_fence_after_sync();
         }
-        const bool row_valid = r >= 0 && r < R;
+        const bool row_valid = r < R;
         const float inv_l = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
         const size_t prow = (group_row0 + static_cast<size_t>(row_valid ? r : 0)) * p.n_splits + split;
         decode_check_prow(p, prow);
