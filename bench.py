@@ -306,8 +306,8 @@ def run_ours(args, rank, world, local_rank):
 
     kvp_line = None
     if args.only is None:
-        kvp_line = run_kv_parallel(attn, dev, stream, rank, world, args.seed, max(3, args.steps // 4), 2,
-                                   max_over_ranks, barrier)
+        kvp_line = run_kv_parallel(attn, dev, stream, rank, world, args.seed, max(3, args.steps // 4),
+                                   max(3, args.warmup), max_over_ranks, barrier)
 
     cpu_line = None
     if rank == 0 and not args.no_cpu_baseline and args.only is None:

@@ -14,7 +14,6 @@
 #include <cstdint>
 #include <cstdio>
 #include <mutex>
-#include <utility>
 
 #include "../../include/attn_gqa.h"
 #include "decode_kv8_sm100.cuh"
@@ -156,25 +155,6 @@ int device_sms_and_sched(cudaStream_t stream, int* n_sm, int** sched) {
     *n_sm = n;
     *sched = b + 2 * slot;
     return ATTN_OK;
-}
-
-// Launch `kernel` as a programmatic dependent of the grid before it in `stream`:
-// it may be scheduled while that grid still runs, and waits (griddepcontrol.wait)
-// for the grid's results before reading them.
-template <typename... ExpTypes, typename... ActTypes>
-cudaError_t launch_dependent(void (*kernel)(ExpTypes...), unsigned grid, unsigned block, cudaStream_t stream,
-                             ActTypes&&... args) {
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(block);
-    cfg.dynamicSmemBytes = 0;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kernel, std::forward<ActTypes>(args)...);
 }
 
 int check_launch(const char* what) {
@@ -406,8 +386,7 @@ int launch_decode_kv8(const void* q, const void* kc, const void* vc, const void*
         st = launch_decode_kv8_split<D, 64, FMT>(tk, tv, tks, tvs, prm, stream);
     if (st != ATTN_OK) return st;
     const int n_rows = B * Hq * Lq;
-    launch_dependent(attn_decode_combine_kernel<D>, static_cast<unsigned>((n_rows + 3) / 4), 128u, stream, prm, out,
-                     lse);
+    attn_decode_combine_kernel<D><<<(n_rows + 3) / 4, 128, 0, stream>>>(prm, out, lse);
     return check_launch("attn_decode_combine_kernel");
 }
 
@@ -469,11 +448,9 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
     if (st != ATTN_OK) return st;
     const int rows = B * Hq * Lq;
     if (f32_out)
-        launch_dependent(attn_decode_combine_kernel<D, true>, static_cast<unsigned>((rows + 3) / 4), 128u, stream, prm,
-                         out, lse);
+        attn_decode_combine_kernel<D, true><<<(rows + 3) / 4, 128, 0, stream>>>(prm, out, lse);
     else
-        launch_dependent(attn_decode_combine_kernel<D>, static_cast<unsigned>((rows + 3) / 4), 128u, stream, prm, out,
-                         lse);
+        attn_decode_combine_kernel<D><<<(rows + 3) / 4, 128, 0, stream>>>(prm, out, lse);
     return check_launch("attn_decode_combine_kernel");
 }
 

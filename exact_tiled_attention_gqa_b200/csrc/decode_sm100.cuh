@@ -115,8 +115,6 @@ __global__ void __maxnreg__(200)
     const uint32_t base = (raw_base + 1023u) & ~1023u;
     uint8_t* smem = smem_raw + (base - raw_base);
 
-    // the split combine may be scheduled now; it waits for this grid's partials
-    if (threadIdx.x == 0) pdl_launch_dependents();
     const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int seqlen = decode_seqlen(p, b);
     const int k_begin = split * p.chunk;
@@ -412,7 +410,6 @@ __global__ void __maxnreg__(200)
 template <int D, bool F32 = false>
 __global__ void __launch_bounds__(128)
     attn_decode_combine_kernel(const DecodeParams p, void* out_ptr, float* lse) {
-    pdl_wait();   // launched as a programmatic dependent of the split kernel
     const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= p.B * p.Hq * p.Lq) return;

@@ -87,8 +87,6 @@ __global__ void __launch_bounds__(kDtcThreads, DecodeTcSmem<D>::kCtasPerSm)
     const uint32_t base = (raw_base + 1023u) & ~1023u;
     uint8_t* smem = smem_raw + (base - raw_base);
 
-    // the split combine may be scheduled now; it waits for this grid's partials
-    if (threadIdx.x == 0) pdl_launch_dependents();
     const int split = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int seqlen = decode_seqlen(p, b);
     const int k_begin = split * p.chunk;

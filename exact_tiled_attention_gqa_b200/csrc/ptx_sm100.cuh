@@ -86,18 +86,6 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 }
 
 // -------------------------------------------------------------------------
-// programmatic dependent launch (the decode kernels and their split combine)
-// -------------------------------------------------------------------------
-// Let the grid that follows this one in the stream (launched with programmatic
-// stream serialisation) be scheduled now; it waits in pdl_wait for our results.
-__device__ __forceinline__ void pdl_launch_dependents() {
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-}
-// Wait until the grid this one depends on has completed and its writes are
-// visible (returns at once when there is no such grid).
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-
-// -------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor), no multicast
 // -------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
