@@ -157,6 +157,17 @@ int device_sms_and_sched(cudaStream_t stream, int* n_sm, int** sched) {
     return ATTN_OK;
 }
 
+// The split combine: one warp per row (four rows per CTA) when rows have few
+// splits, four warps per row when they have more than 16 (their reads then take
+// four times fewer dependent rounds).
+template <int D, bool F32>
+void launch_combine(const DecodeParams& prm, void* out, float* lse, int rows, cudaStream_t stream) {
+    if (prm.n_splits > 16)
+        attn_decode_combine_kernel<D, F32, 4><<<rows, 128, 0, stream>>>(prm, out, lse);
+    else
+        attn_decode_combine_kernel<D, F32, 1><<<(rows + 3) / 4, 128, 0, stream>>>(prm, out, lse);
+}
+
 int check_launch(const char* what) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString(e));
@@ -386,7 +397,7 @@ int launch_decode_kv8(const void* q, const void* kc, const void* vc, const void*
         st = launch_decode_kv8_split<D, 64, FMT>(tk, tv, tks, tvs, prm, stream);
     if (st != ATTN_OK) return st;
     const int n_rows = B * Hq * Lq;
-    attn_decode_combine_kernel<D><<<(n_rows + 3) / 4, 128, 0, stream>>>(prm, out, lse);
+    launch_combine<D, false>(prm, out, lse, n_rows, stream);
     return check_launch("attn_decode_combine_kernel");
 }
 
@@ -448,9 +459,9 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
     if (st != ATTN_OK) return st;
     const int rows = B * Hq * Lq;
     if (f32_out)
-        attn_decode_combine_kernel<D, true><<<(rows + 3) / 4, 128, 0, stream>>>(prm, out, lse);
+        launch_combine<D, true>(prm, out, lse, rows, stream);
     else
-        attn_decode_combine_kernel<D><<<(rows + 3) / 4, 128, 0, stream>>>(prm, out, lse);
+        launch_combine<D, false>(prm, out, lse, rows, stream);
     return check_launch("attn_decode_combine_kernel");
 }
 

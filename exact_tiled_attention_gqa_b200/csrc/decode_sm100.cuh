@@ -402,24 +402,29 @@ __global__ void __maxnreg__(200)
     }
 }
 
-// One warp per query row: out = sum_s 2^(lse_s - lse) O_s,  lse = log2 sum_s 2^lse_s.
-// The 32 lanes read the splits' LSEs together (one split each); each lane then
-// sums its D / 32 columns over the splits, the loads unrolled so that several
-// are in flight (a row with 64-256 splits is otherwise one dependent load per split).
+// out = sum_s 2^(lse_s - lse) O_s,  lse = log2 sum_s 2^lse_s, per query row.
+// WPR warps per row (1: four rows per CTA; 4: one row per CTA, for rows with many
+// splits).  Every warp of a row finds the max over all the row's splits (the 32
+// lanes read LSEs together); warp w then takes splits w, w + WPR, w + 2 WPR, ...,
+// each lane summing its D / 32 columns with the partial loads unrolled 8 deep, so
+// a row's splits are read in WPR times fewer dependent rounds; the warps' sums
+// meet in shared memory.
 // F32: out is fp32 [rows, D] instead of bf16 (a partial result that is merged later).
-template <int D, bool F32 = false>
+template <int D, bool F32 = false, int WPR = 1>
 __global__ void __launch_bounds__(128)
     attn_decode_combine_kernel(const DecodeParams p, void* out_ptr, float* lse) {
-    const int row = blockIdx.x * 4 + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (row >= p.B * p.Hq * p.Lq) return;
+    static_assert(WPR == 1 || WPR == 4, "one or four warps per row");
+    constexpr int kPer = D / 32;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row = blockIdx.x * (4 / WPR) + warp / WPR;
+    const int sub = warp % WPR;
+    if (row >= p.B * p.Hq * p.Lq) return;   // (uniform over a CTA when WPR = 4)
     const int b = row / (p.Hq * p.Lq);
     const int seqlen = decode_seqlen(p, b);
     const int n_valid = (seqlen + p.chunk - 1) / p.chunk;
     ATTN_CHECK(n_valid >= 0 && n_valid <= p.n_splits);
     const float* lp = p.lse_part + static_cast<size_t>(row) * p.n_splits;
     const float* op = p.o_part + static_cast<size_t>(row) * p.n_splits * D;
-    constexpr int kPer = D / 32;
     float M = -INFINITY;
     for (int s = lane; s < n_valid; s += 32) M = fmaxf(M, lp[s]);
 #pragma unroll
@@ -428,17 +433,17 @@ __global__ void __launch_bounds__(128)
 #pragma unroll
     for (int i = 0; i < kPer; ++i) acc[i] = 0.0f;
     float Lsum = 0.0f;
-    for (int s0 = 0; s0 < n_valid; s0 += 32) {
-        const int s = s0 + lane;
+    for (int base = 0; base < n_valid; base += 32 * WPR) {
+        const int s = base + lane * WPR + sub;   // this lane's split of the round
         const float ls = (s < n_valid) ? lp[s] : -INFINITY;
         const float wl = (ls == -INFINITY) ? 0.0f : ex2_approx(ls - M);   // this lane's split weight
         Lsum += wl;
-        const int cnt = min(32, n_valid - s0);
-        const float* ob = op + static_cast<size_t>(s0) * D + lane * kPer;
+        const int cnt = min(32, (n_valid - base - sub + WPR - 1) / WPR);   // this warp's splits this round
+        const float* ob = op + static_cast<size_t>(base + sub) * D + lane * kPer;
 #pragma unroll 8
         for (int i = 0; i < cnt; ++i) {
             const float w = __shfl_sync(0xffffffffu, wl, i);
-            const float* src = ob + static_cast<size_t>(i) * D;
+            const float* src = ob + static_cast<size_t>(i) * WPR * D;
 #pragma unroll
             for (int c = 0; c < kPer; c += 2) {
                 const float2 v = *reinterpret_cast<const float2*>(src + c);
@@ -449,6 +454,21 @@ __global__ void __launch_bounds__(128)
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, o);
+    if constexpr (WPR > 1) {
+        __shared__ float red_acc[WPR][D];
+        __shared__ float red_l[WPR];
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) red_acc[sub][lane * kPer + i] = acc[i];
+        if (lane == 0) red_l[sub] = Lsum;
+        __syncthreads();
+        if (sub != 0) return;
+#pragma unroll
+        for (int w = 1; w < WPR; ++w) {
+#pragma unroll
+            for (int i = 0; i < kPer; ++i) acc[i] += red_acc[w][lane * kPer + i];
+            Lsum += red_l[w];
+        }
+    }
     const float inv = (Lsum > 0.0f) ? 1.0f / Lsum : 0.0f;
     if constexpr (F32) {
         float* o = static_cast<float*>(out_ptr) + static_cast<size_t>(row) * D + lane * kPer;

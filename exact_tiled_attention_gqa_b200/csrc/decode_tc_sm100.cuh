@@ -32,8 +32,8 @@
 //    caches with 64-row pages work), filled in the order the MMAs use them
 //    (K_0 K_1 V_0 K_2 V_1 ..., ring_order.cuh).
 //
-// The softmax reads S twice from TMEM (row max, then the exponentials).  Warps
-// whose 32 rows are all padding only keep the pipeline moving.  Cache rows past
+// The softmax reads a tile's S from TMEM once into registers (row max, then the
+// exponentials).  Warps whose 32 rows are all padding only keep the pipeline moving.  Cache rows past
 // the split's valid length may hold anything (NaN included); P is 0 there but
 // 0 * NaN is NaN, so the MMA warp zeroes those V rows in shared memory first.
 #pragma once
@@ -313,26 +313,24 @@ __global__ void __launch_bounds__(kDtcThreads, DecodeTcSmem<D>::kCtasPerSm)
             const uint32_t tSr = tS[buf] + lane_off;
             const int key0 = k_begin + j * kDtcBN;
             const bool masked = key0 + kDtcBN > lim_lo;
-            // pass 1: the row max of this tile
+            // the tile's 64 scores of this row, read from TMEM once
+            uint32_t v[kDtcBN];
+            tmem_ld_32x32b_x32(tSr, v);
+            tmem_ld_32x32b_x32(tSr + 32, v + 32);
+            tmem_wait_ld();
+            reg_fence<kDtcBN>(v);
+            if (masked) {
+#pragma unroll
+                for (int i = 0; i < kDtcBN; ++i)
+                    if (key0 + i >= lim) v[i] = __float_as_uint(-INFINITY);
+            }
             float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-#pragma unroll 1
-            for (int c = 0; c < kDtcBN; c += 32) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(tSr + c, v);
-                tmem_wait_ld();
-                reg_fence<32>(v);
-                if (masked) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (key0 + c + i >= lim) v[i] = __float_as_uint(-INFINITY);
-                }
-#pragma unroll
-                for (int i = 0; i < 32; i += 8) {
-                    mx0 = fmax3(mx0, __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
-                    mx1 = fmax3(mx1, __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
-                    mx2 = fmax3(mx2, __uint_as_float(v[i + 4]), __uint_as_float(v[i + 5]));
-                    mx3 = fmax3(mx3, __uint_as_float(v[i + 6]), __uint_as_float(v[i + 7]));
-                }
+            for (int i = 0; i < kDtcBN; i += 8) {
+                mx0 = fmax3(mx0, __uint_as_float(v[i]), __uint_as_float(v[i + 1]));
+                mx1 = fmax3(mx1, __uint_as_float(v[i + 2]), __uint_as_float(v[i + 3]));
+                mx2 = fmax3(mx2, __uint_as_float(v[i + 4]), __uint_as_float(v[i + 5]));
+                mx3 = fmax3(mx3, __uint_as_float(v[i + 6]), __uint_as_float(v[i + 7]));
             }
             const float m_tile = fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * sl2;
             float factor = 1.0f;
@@ -368,26 +366,17 @@ __global__ void __launch_bounds__(kDtcThreads, DecodeTcSmem<D>::kCtasPerSm)
                 }
                 tmem_wait_st();
             }
-            // pass 2: exponentials, row sums, P (bf16) over the S columns already read
+            // exponentials, row sums, P (bf16) over the S columns already read
             const float m_sub = (m_run == -INFINITY) ? 0.0f : m_run;
             const uint64_t negm2 = f2_pack(-m_sub, -m_sub);
             uint64_t acc_r = 0ull, acc_e = 0ull;
-#pragma unroll 1
-            for (int c = 0; c < kDtcBN; c += 32) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(tSr + c, v);
-                tmem_wait_ld();
-                reg_fence<32>(v);
-                if (masked) {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i)
-                        if (key0 + c + i >= lim) v[i] = __float_as_uint(-INFINITY);
-                }
+            for (int c = 0; c < kDtcBN; c += 32) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const uint64_t t =
-                        f2_fma(f2_pack(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), sl2x2, negm2);
+                    const uint64_t t = f2_fma(f2_pack(__uint_as_float(v[c + 2 * i]), __uint_as_float(v[c + 2 * i + 1])),
+                                              sl2x2, negm2);
                     float t0, t1;
                     f2_unpack(t, t0, t1);
                     const float e0 = ex2_approx(t0), e1 = ex2_approx(t1);

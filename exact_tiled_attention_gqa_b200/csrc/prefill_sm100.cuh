@@ -44,7 +44,11 @@
 // NQ = 1 (D = 256) the two buffers alternate between key tiles (S(j) in buffer
 // j mod 2) and O takes [256, 512).  P (bf16, two per column) overwrites the
 // first 64 columns of its S buffer once the softmax has read S, and feeds
-// O += P V_j as the TMEM A operand.
+// O += P V_j as the TMEM A operand -- except at D = 64, where O0 and O1 end at
+// column 384 and P_q gets columns of its own (P0 at 384, P1 at 448): there the
+// softmax signals s_free_q once S_q(j) is in registers, S_q(j+1) = Q_q K_{j+1}^T
+// is issued before O_q += P_q(j) V_j, and pv_done_q (committed after each P.V)
+// tells the softmax when it may overwrite P_q or rescale O_q.
 //
 // Per key tile j the MMA thread issues, in order:
 //   O0 += P0(j) V_j ; S0(j+1) = Q0 K_{j+1}^T ; O1 += P1(j) V_j ; S1(j+1) = Q1 K_{j+1}^T
@@ -52,7 +56,8 @@
 // softmax hands P over in two halves (keys 0-63, then 64-127), and each half of
 // O_q += P_q V_j is issued as soon as its half is in TMEM.
 // A commit after S_q(j+1) also covers O_q += P_q(j) V_j, so when the softmax
-// sees S_q(j+1) its O_q is settled and may be rescaled in place.
+// sees S_q(j+1) its O_q is settled and may be rescaled in place (with P in its
+// own columns, D = 64, the softmax waits on pv_done_q instead).
 //
 // NQ = 1 (D = 256): one Q tile, so the overlap comes from the second S buffer:
 //   S(0) ; S(1) ; then per j:  O += P(j) V_j ; S(j+2) = Q K_{j+2}^T
