@@ -404,17 +404,19 @@ __global__ void __maxnreg__(200)
 
 // out = sum_s 2^(lse_s - lse) O_s,  lse = log2 sum_s 2^lse_s, per query row.
 // WPR warps per row (1: four rows per CTA; 4: one row per CTA, for rows with many
-// splits).  Every warp of a row finds the max over all the row's splits (the 32
-// lanes read LSEs together); warp w then takes splits w, w + WPR, w + 2 WPR, ...,
-// each lane summing its D / 32 columns with the partial loads unrolled 8 deep, so
-// a row's splits are read in WPR times fewer dependent rounds; the warps' sums
-// meet in shared memory.
+// splits).  Warp w of a row takes splits w, w + WPR, w + 2 WPR, ... in chunks of
+// kChunk; lane i holds the LSE of the chunk's split i and every lane D / 32
+// columns of each of its O rows.  All loads of the first chunk -- the row's LSEs
+// for the max, the chunk's LSEs and O rows -- are issued before any of them is
+// used, so a row with up to WPR * kChunk splits costs one round trip to memory.
+// The warps' sums meet in shared memory.
 // F32: out is fp32 [rows, D] instead of bf16 (a partial result that is merged later).
 template <int D, bool F32 = false, int WPR = 1>
 __global__ void __launch_bounds__(128)
     attn_decode_combine_kernel(const DecodeParams p, void* out_ptr, float* lse) {
     static_assert(WPR == 1 || WPR == 4, "one or four warps per row");
-    constexpr int kPer = D / 32;
+    constexpr int kPer = D / 32;                  // columns per lane
+    constexpr int kChunk = (D >= 256) ? 8 : 16;   // splits per warp whose O rows are in registers
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int row = blockIdx.x * (4 / WPR) + warp / WPR;
     const int sub = warp % WPR;
@@ -424,7 +426,31 @@ __global__ void __launch_bounds__(128)
     const int n_valid = (seqlen + p.chunk - 1) / p.chunk;
     ATTN_CHECK(n_valid >= 0 && n_valid <= p.n_splits);
     const float* lp = p.lse_part + static_cast<size_t>(row) * p.n_splits;
-    const float* op = p.o_part + static_cast<size_t>(row) * p.n_splits * D;
+    const float* op = p.o_part + static_cast<size_t>(row) * p.n_splits * D + lane * kPer;
+    float ov[kChunk][kPer];
+    float my_ls;
+    // this warp's chunk from split `base`: lane i's LSE, every lane's columns of the O rows
+    auto load_chunk = [&](int base) {
+        const int sl = base + sub + WPR * lane;
+        my_ls = (lane < kChunk && sl < n_valid) ? lp[sl] : -INFINITY;
+#pragma unroll
+        for (int i = 0; i < kChunk; ++i) {
+            const int s = base + sub + WPR * i;
+            if (s < n_valid) {
+                const float* src = op + static_cast<size_t>(s) * D;
+#pragma unroll
+                for (int c = 0; c < kPer; c += 2) {
+                    const float2 v = *reinterpret_cast<const float2*>(src + c);
+                    ov[i][c] = v.x;
+                    ov[i][c + 1] = v.y;
+                }
+            } else {
+#pragma unroll
+                for (int c = 0; c < kPer; ++c) ov[i][c] = 0.0f;
+            }
+        }
+    };
+    load_chunk(0);
     float M = -INFINITY;
     for (int s = lane; s < n_valid; s += 32) M = fmaxf(M, lp[s]);
 #pragma unroll
@@ -432,24 +458,16 @@ __global__ void __launch_bounds__(128)
     float acc[kPer];
 #pragma unroll
     for (int i = 0; i < kPer; ++i) acc[i] = 0.0f;
-    float Lsum = 0.0f;
-    for (int base = 0; base < n_valid; base += 32 * WPR) {
-        const int s = base + lane * WPR + sub;   // this lane's split of the round
-        const float ls = (s < n_valid) ? lp[s] : -INFINITY;
-        const float wl = (ls == -INFINITY) ? 0.0f : ex2_approx(ls - M);   // this lane's split weight
+    float Lsum = 0.0f;   // lane i: the weights of its splits
+    for (int base = 0; base < n_valid; base += WPR * kChunk) {
+        if (base > 0) load_chunk(base);
+        const float wl = (my_ls == -INFINITY) ? 0.0f : ex2_approx(my_ls - M);   // split weight (lane < kChunk)
         Lsum += wl;
-        const int cnt = min(32, (n_valid - base - sub + WPR - 1) / WPR);   // this warp's splits this round
-        const float* ob = op + static_cast<size_t>(base + sub) * D + lane * kPer;
-#pragma unroll 8
-        for (int i = 0; i < cnt; ++i) {
-            const float w = __shfl_sync(0xffffffffu, wl, i);
-            const float* src = ob + static_cast<size_t>(i) * WPR * D;
 #pragma unroll
-            for (int c = 0; c < kPer; c += 2) {
-                const float2 v = *reinterpret_cast<const float2*>(src + c);
-                acc[c] = fmaf(w, v.x, acc[c]);
-                acc[c + 1] = fmaf(w, v.y, acc[c + 1]);
-            }
+        for (int i = 0; i < kChunk; ++i) {
+            const float w = __shfl_sync(0xffffffffu, wl, i);
+#pragma unroll
+            for (int c = 0; c < kPer; ++c) acc[c] = fmaf(w, ov[i][c], acc[c]);
         }
     }
 #pragma unroll

@@ -783,7 +783,10 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
                 const float m_sub = (m_run == -INFINITY) ? 0.0f : m_run;
                 const uint64_t sl2x2 = f2_pack(sl2, sl2);
                 const uint64_t negm2 = f2_pack(-m_sub, -m_sub);
-                uint64_t acc_e[2] = {0ull, 0ull};
+                // the row sum in independent f32x2 chains: four at D=128 (shorter
+                // dependency chain, measured faster there), two at D=64 (fewer registers)
+                constexpr int kSumChains = (D == 128) ? 4 : 2;
+                uint64_t acc_e[4] = {0ull, 0ull, 0ull, 0ull};
                 auto exp_half = [&](int hf) {
                     uint32_t pk[32];
 #pragma unroll
@@ -794,7 +797,7 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
                         f2_unpack(t, t0, t1);
                         const float e0 = ex2_approx(t0), e1 = ex2_approx(t1);
                         pk[i] = pack_bf16x2(e0, e1);
-                        acc_e[i & 1] = f2_add(acc_e[i & 1], f2_pack(e0, e1));
+                        acc_e[i % kSumChains] = f2_add(acc_e[i % kSumChains], f2_pack(e0, e1));
                     }
                     tmem_st_32x32b_x32((kSplitP ? tP_q : tS) + hf * 32, pk);
                     tmem_wait_st();
@@ -819,7 +822,9 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
                     d_round = __uint_as_float(pack_bf16x2(pm, 0.0f) << 16) - pm;
                 }
                 float b0, b1;
-                f2_unpack(f2_add(acc_e[0], acc_e[1]), b0, b1);
+                f2_unpack(kSumChains == 4 ? f2_add(f2_add(acc_e[0], acc_e[1]), f2_add(acc_e[2], acc_e[3]))
+                                          : f2_add(acc_e[0], acc_e[1]),
+                          b0, b1);
                 l_run += (b0 + b1) + d_round;
                 l_exact += b0 + b1;
             }
