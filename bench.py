@@ -273,10 +273,13 @@ def run_ours(args, rank, world, local_rank):
 
     # ---- end to end through the public API with host buffers ----
     pin = lambda t: t.cpu().pin_memory()
-    hq, hk, hv, hdq = pin(q_h), pin(k_h), pin(v_h), pin(dq)
+    hq, hk, hv, hdq, hsl = pin(q_h), pin(k_h), pin(v_h), pin(dq), pin(dsl)
     ho, hl = torch.empty_like(hq).pin_memory(), torch.empty(p_lse.shape, dtype=torch.float32).pin_memory()
     hdo, hdl = torch.empty_like(hdq).pin_memory(), torch.empty(d_lse.shape, dtype=torch.float32).pin_memory()
     e2e_pre, e2e_dec = [], []
+    ws_host = None if args.only is not None else torch.empty(
+        attn.decode_host_workspace_size(dshape.B, dshape.Hq, dshape.Hkv, dshape.Lmax, dshape.D), dtype=torch.uint8,
+        device=dev)
     # prefill end to end: the host-buffer call, which pipelines copies in, kernels and copies out
     scr = torch.empty(attn.prefill_host_scratch_size(PREFILL.B, PREFILL.Hq, PREFILL.Hkv, PREFILL.Lq, PREFILL.Lk,
                                                      PREFILL.D), dtype=torch.uint8, device=dev)
@@ -285,10 +288,9 @@ def run_ours(args, rank, world, local_rank):
         e[0].record(stream)
         attn.prefill_host(hq, hk, hv, is_causal=True, out=ho, lse=hl, scratch=scr, device=dev, stream=stream)
         e[1].record(stream)
-        dq.copy_(hdq, non_blocking=True)
-        attn.decode(dq, dk, dv, dsl, out=d_out, lse=d_lse, workspace=ws, stream=stream)
-        hdo.copy_(d_out, non_blocking=True)
-        hdl.copy_(d_lse, non_blocking=True)
+        # the host-buffer call: q and seqlens in, decode, out and lse back (bf16 cache: 8-bit caches
+        # only run with --only decode, which has no end-to-end leg)
+        attn.decode_host(hdq, dk, dv, hsl, out=hdo, lse=hdl, workspace=ws_host, stream=stream)
         e[2].record(stream)
         torch.cuda.synchronize()
         if i > 0:   # the first is a warm-up of the copy path
@@ -301,7 +303,7 @@ def run_ours(args, rank, world, local_rank):
                           "prefill_tflops": p_flops / (pre_avg * 1e-3) / 1e12 if do_pre else None,
                           "decode_gbs": d_bytes / (dec_avg * 1e-3) / 1e9 if do_dec else None}), flush=True)
         return None
-    h2d = (hq.numel() + hk.numel() + hv.numel() + hdq.numel()) * 2
+    h2d = (hq.numel() + hk.numel() + hv.numel() + hdq.numel()) * 2 + hsl.numel() * 4
     d2h = (ho.numel() + hdo.numel()) * 2 + (hl.numel() + hdl.numel()) * 4
 
     kvp_line = None
@@ -367,8 +369,8 @@ def run_ours(args, rank, world, local_rank):
                 "decode_gbs": round(world * d_bytes / (e2e_dec_ms * 1e-3) / 1e9, 1),
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "what": "prefill: attn_prefill_host on pinned host q/k/v/out/lse (copies in, kernels and copies "
-                        "out pipelined by the library); decode: pinned q in, attn_decode, pinned out/lse back, "
-                        "KV cache resident"},
+                        "out pipelined by the library); decode: attn_decode_host on pinned host q/seqlens/out/lse "
+                        "(one call: copies in, kernels, copies out), KV cache resident on the device"},
         "gpu_launches": 3 * args.steps,
         "kv_parallel": kvp_line,
         "sweeps": sweeps,

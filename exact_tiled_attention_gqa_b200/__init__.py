@@ -27,7 +27,7 @@ import torch
 from . import _native
 from ._native import AttnError
 
-__all__ = ["prefill", "prefill_host", "decode", "decode_partial", "decode_merge", "decode_merge_peers", "kvp_signal",
+__all__ = ["prefill", "prefill_host", "decode", "decode_host", "decode_host_workspace_size", "decode_partial", "decode_merge", "decode_merge_peers", "kvp_signal",
            "kvp_wait", "decode_mq", "decode_paged", "decode_noalloc", "decode_kv8", "decode_kv8_paged", "prefill_host_scratch_size", "decode_workspace_size", "decode_mq_workspace_size",
            "decode_kv8_workspace_size", "device_error", "AttnError", "library_path"]
 
@@ -59,11 +59,11 @@ def _check_tensor(name: str, t: torch.Tensor, dtype: torch.dtype, ndim: int) -> 
         raise ValueError(f"{name} must be contiguous")
 
 
-def _check_on(device: torch.device, **tensors) -> None:
-    """Every given tensor (None skipped) lives on `device`."""
+def _check_on(device: torch.device, _ref: str = "q", **tensors) -> None:
+    """Every given tensor (None skipped) lives on `device`, the device of the tensor named `_ref`."""
     for name, t in tensors.items():
         if t is not None and t.device != device:
-            raise ValueError(f"{name} is on {t.device}, but q is on {device}")
+            raise ValueError(f"{name} is on {t.device}, but {_ref} is on {device}")
 
 
 def _result(name: str, t: Optional[torch.Tensor], dtype: torch.dtype, shape, device: torch.device,
@@ -194,6 +194,45 @@ def decode(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, seqlen
                                        B, Hq, Hkv, Lmax, D, float(scale), _ptr(workspace), ws_bytes,
                                        _stream_handle(stream))
     _native.check(st, "attn_decode")
+    return out, lse
+
+
+def decode_host_workspace_size(B: int, Hq: int, Hkv: int, Lmax: int, D: int) -> int:
+    return int(_native.lib().attn_decode_host_workspace_size(B, Hq, Hkv, Lmax, D))
+
+
+def decode_host(q: torch.Tensor, k_cache: torch.Tensor, v_cache: torch.Tensor, seqlens: torch.Tensor, *,
+                scale: Optional[float] = None, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                want_lse: bool = True, workspace: Optional[torch.Tensor] = None, stream=None):
+    """decode with q, seqlens, out and lse on the host (CPU tensors, pinned for asynchronous copies) and the
+    caches on the device: one call copies q and seqlens in, decodes and copies the results out.  They are in
+    `out` / `lse` once `stream` (default: the current stream of the caches' device) has passed the call."""
+    for name, t, dt, nd in (("q", q, torch.bfloat16, 3), ("seqlens", seqlens, torch.int32, 1)):
+        if not isinstance(t, torch.Tensor) or t.is_cuda or t.dtype != dt or t.dim() != nd or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous {nd}-d {dt} CPU tensor")
+    _check_tensor("k_cache", k_cache, torch.bfloat16, 4)
+    _check_tensor("v_cache", v_cache, torch.bfloat16, 4)
+    B, Hq, D = q.shape
+    Hkv, Lmax = k_cache.shape[1], k_cache.shape[2]
+    if k_cache.shape[0] != B or k_cache.shape[3] != D or v_cache.shape != k_cache.shape or seqlens.shape[0] != B:
+        raise ValueError("shape mismatch between q, the caches and seqlens")
+    _check_on(k_cache.device, "k_cache", v_cache=v_cache)
+    if scale is None:
+        scale = 1.0 / math.sqrt(D)
+    if out is None:
+        out = torch.empty(q.shape, dtype=torch.bfloat16, pin_memory=True)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, pin_memory=True)
+    for name, t, dt, shp in (("out", out, torch.bfloat16, tuple(q.shape)), ("lse", lse, torch.float32, (B, Hq))):
+        if t is not None and (t.is_cuda or not t.is_contiguous() or t.dtype != dt or tuple(t.shape) != shp):
+            raise ValueError(f"{name} must be a contiguous {dt} CPU tensor of shape {shp}")
+    need = decode_host_workspace_size(B, Hq, Hkv, Lmax, D)
+    workspace, ws_bytes = _workspace(workspace, need, k_cache.device)
+    with torch.cuda.device(k_cache.device):
+        st = _native.lib().attn_decode_host(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(seqlens), _ptr(out),
+                                            _ptr(lse), B, Hq, Hkv, Lmax, D, float(scale), _ptr(workspace), ws_bytes,
+                                            _stream_handle(stream))
+    _native.check(st, "attn_decode_host")
     return out, lse
 
 

@@ -41,6 +41,8 @@ SIGNATURES = {
                                  _vp]),
     "attn_decode_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32]),
     "attn_decode": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _sz, _vp]),
+    "attn_decode_host_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32]),
+    "attn_decode_host": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _sz, _vp]),
     "attn_decode_partial": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _f32, _vp, _sz, _vp]),
     "attn_decode_merge": (_i32, [_vp, _vp, _i32, _i32, _i32, _vp, _vp, _vp]),
     "attn_kvp_signal": (_i32, [_vp, _i32, ctypes.c_uint, _vp]),

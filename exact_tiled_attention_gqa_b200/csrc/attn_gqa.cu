@@ -733,6 +733,68 @@ extern "C" int attn_decode(const void* q, const void* k_cache, const void* v_cac
                           workspace_bytes, stream, false);
 }
 
+namespace {
+// attn_decode_host's workspace: attn_decode's partials, then device copies of
+// q, out, lse and seqlens, each 256-byte aligned.
+struct HostDecodeLayout {
+    size_t q_off, o_off, l_off, s_off, total;
+};
+HostDecodeLayout host_decode_layout(int B, int Hq, int D, size_t partial_bytes) {
+    auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    const size_t rows = static_cast<size_t>(B) * Hq;
+    HostDecodeLayout L;
+    L.q_off = al(partial_bytes);
+    L.o_off = L.q_off + al(rows * D * 2);
+    L.l_off = L.o_off + al(rows * D * 2);
+    L.s_off = L.l_off + al(rows * 4);
+    L.total = L.s_off + al(static_cast<size_t>(B) * 4);
+    return L;
+}
+}  // namespace
+
+extern "C" size_t attn_decode_host_workspace_size(int B, int Hq, int Hkv, int Lmax, int D) {
+    const size_t partial = attn_decode_workspace_size(B, Hq, Hkv, Lmax, D);
+    return partial == 0 ? 0 : host_decode_layout(B, Hq, D, partial).total;
+}
+
+extern "C" int attn_decode_host(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,
+                                void* out, float* lse, int B, int Hq, int Hkv, int Lmax, int D, float scale,
+                                void* workspace, size_t workspace_bytes, void* stream) {
+    int st = check_common(q, k_cache, v_cache, out, lse, B, Hq, Hkv, Lmax, Lmax, D, scale, "Lmax", "Lmax");
+    if (st != ATTN_OK) return st;
+    if (!seqlens && B > 0) return fail(ATTN_ERR_INVALID_ARG, "null seqlens");
+    if (reinterpret_cast<uintptr_t>(seqlens) & 3u) return fail(ATTN_ERR_INVALID_ARG, "seqlens must be 4-byte aligned");
+    if (Lmax < 1) return fail(ATTN_ERR_INVALID_ARG, "Lmax must be >= 1");
+    if (Hq / Hkv > 128) return fail(ATTN_ERR_UNSUPPORTED, "decode group size G=%d > 128", Hq / Hkv);
+    if (static_cast<long long>(B) * Hq > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "B*Hq too large");
+    if (B == 0) return ok();
+    const size_t partial = attn_decode_workspace_size(B, Hq, Hkv, Lmax, D);
+    const HostDecodeLayout L = host_decode_layout(B, Hq, D, partial);
+    if (!workspace || workspace_bytes < L.total)
+        return fail(ATTN_ERR_WORKSPACE, "decode host workspace needs %zu bytes, got %zu", L.total,
+                    workspace ? workspace_bytes : static_cast<size_t>(0));
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u)
+        return fail(ATTN_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    const size_t rows = static_cast<size_t>(B) * Hq;
+    auto copy = [&](void* dst, const void* src, size_t bytes, cudaMemcpyKind kind, const char* what) {
+        const cudaError_t e = cudaMemcpyAsync(dst, src, bytes, kind, s);
+        return e == cudaSuccess ? ATTN_OK : fail(ATTN_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+    };
+    if ((st = copy(ws + L.q_off, q, rows * D * 2, cudaMemcpyHostToDevice, "copy q in")) != ATTN_OK) return st;
+    if ((st = copy(ws + L.s_off, seqlens, static_cast<size_t>(B) * 4, cudaMemcpyHostToDevice, "copy seqlens in")) !=
+        ATTN_OK)
+        return st;
+    float* lse_dev = lse ? reinterpret_cast<float*>(ws + L.l_off) : nullptr;
+    st = decode_checked(ws + L.q_off, k_cache, v_cache, reinterpret_cast<const int32_t*>(ws + L.s_off), ws + L.o_off,
+                        lse_dev, B, Hq, Hkv, Lmax, D, scale, workspace, partial, stream, false);
+    if (st != ATTN_OK) return st;
+    if ((st = copy(out, ws + L.o_off, rows * D * 2, cudaMemcpyDeviceToHost, "copy out")) != ATTN_OK) return st;
+    if (lse && (st = copy(lse, lse_dev, rows * 4, cudaMemcpyDeviceToHost, "copy lse out")) != ATTN_OK) return st;
+    return ok();
+}
+
 extern "C" int attn_decode_partial(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,
                                    float* o_part, float* lse_part, int B, int Hq, int Hkv, int Lmax, int D, float scale,
                                    void* workspace, size_t workspace_bytes, void* stream) {

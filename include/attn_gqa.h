@@ -188,6 +188,38 @@ int attn_decode(const void* q, const void* k_cache, const void* v_cache, const i
                 void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * attn_decode_host_workspace_size / attn_decode_host -- attn_decode for a
+ * caller whose new query rows arrive in, and whose results go back to, HOST
+ * memory, while the KV cache stays resident on the device (a cache is device
+ * state that decode steps append to; the "use_cache" section of the SDPA
+ * guide).  One call copies q and seqlens in, decodes, and copies out and lse
+ * back, all enqueued on `stream` in that order.
+ *
+ *   q        [B, Hq, D]          bf16, HOST memory, read
+ *   k_cache  [B, Hkv, Lmax, D]   bf16, device memory, read (as attn_decode)
+ *   v_cache  [B, Hkv, Lmax, D]   bf16, device memory, read
+ *   seqlens  [B]                 int32, HOST memory, read (values as attn_decode)
+ *   out      [B, Hq, D]          bf16, HOST memory, written
+ *   lse      [B, Hq]             fp32, HOST memory, written; may be NULL
+ *   workspace device memory of attn_decode_host_workspace_size(...) bytes,
+ *            256-byte aligned, owned by the caller: attn_decode's split
+ *            partials followed by device copies of q, out, lse and seqlens
+ *
+ * Page-locked host buffers let the copies run asynchronously; with pageable
+ * memory each copy waits for the host.  Completion: when `stream` has passed
+ * the work this call enqueued, out and lse hold the results; the host buffers
+ * must stay valid until then.  Errors: as attn_decode (checked before anything
+ * is enqueued), ATTN_ERR_WORKSPACE for a missing or small workspace,
+ * ATTN_ERR_INVALID_ARG for a misaligned one, ATTN_ERR_CUDA if a copy cannot
+ * be enqueued.  attn_decode_host_workspace_size returns 0 for sizes
+ * attn_decode would reject and for B == 0.
+ */
+size_t attn_decode_host_workspace_size(int B, int Hq, int Hkv, int Lmax, int D);
+int attn_decode_host(const void* q, const void* k_cache, const void* v_cache, const int32_t* seqlens,
+                     void* out, float* lse, int B, int Hq, int Hkv, int Lmax, int D, float scale,
+                     void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * attn_decode_partial / attn_decode_merge -- decode split across devices by
  * cache rows (the KV parallelism of the NVIDIA attention page, "Parameter
  * four: parallelism"): each device holds a disjoint set of every sequence's

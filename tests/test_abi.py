@@ -210,6 +210,21 @@ def test_prefill_host_rejects(lib):
     assert s(2, 8, 2, 64, 64, 128) > 0 and s(2, 8, 2, 64, 64, 96) == 0 and s(0, 8, 2, 64, 64, 128) == 0
 
 
+def test_decode_host_rejects(lib):
+    f = lambda **kw: lib.attn_decode_host(*[kw.get(n, d) for n, d in (
+        ("q", A), ("k", A), ("v", A), ("sl", A), ("out", A), ("lse", NULL), ("B", 2), ("Hq", 8), ("Hkv", 2),
+        ("Lmax", 64), ("D", 128), ("scale", 0.1), ("ws", A), ("wsb", 1 << 30))], None)
+    assert f(ws=NULL) == -3 and f(wsb=1024) == -3 and f(ws=ctypes.c_void_p(0x10010)) == -1
+    assert f(q=NULL) == -1 and f(sl=NULL) == -1 and f(sl=ctypes.c_void_p(0x10002)) == -1 and f(Lmax=0) == -1
+    assert f(D=96) == -2 and f(Hq=7) == -1 and f(Hq=256, Hkv=1) == -2 and f(B=0) == 0
+    s = lib.attn_decode_host_workspace_size
+    # the partials, then q, out, lse and seqlens, each rounded up to 256 bytes
+    part = lib.attn_decode_workspace_size(2, 8, 2, 64, 128)
+    up = lambda x: (x + 255) // 256 * 256
+    assert s(2, 8, 2, 64, 128) == up(part) + 2 * up(2 * 8 * 128 * 2) + up(2 * 8 * 4) + up(2 * 4)
+    assert s(2, 8, 2, 64, 96) == 0 and s(0, 8, 2, 64, 128) == 0
+
+
 def test_decode_partial_and_merge_reject(lib):
     m = lambda **kw: lib.attn_decode_merge(*[kw.get(n, d) for n, d in (("o", A), ("l", A), ("n", 2), ("rows", 8),
                                                                         ("D", 128), ("out", A), ("lse", NULL))], None)
