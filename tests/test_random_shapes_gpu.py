@@ -1,0 +1,97 @@
+"""Seeded random shapes through prefill and decode, every output element against
+the fp64 oracle.
+
+The cases are drawn once from a fixed numpy seed (the list is the same on every
+run): batch, heads and group size (including group sizes that do not divide
+the 128-row tile), query and key lengths from 1 to a few tiles on either side of
+a tile boundary, head dims 64 / 128 / 256, causal and full attention; decode
+with cache lengths from 0 to Lmax.  They complement the hand-picked edge cases
+of the other parity files with combinations nobody chose.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from exact_tiled_attention_gqa_b200 import decode, device_error, prefill
+from exact_tiled_attention_gqa_b200 import workloads as W
+from parity import assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    device_error(reset=True)
+    yield
+    assert device_error(reset=True) == 0
+
+
+def _near_tile(rng, hi):
+    """A length in [1, hi], often within a few of a multiple of 128."""
+    if rng.random() < 0.5:
+        return int(rng.integers(1, hi + 1))
+    base = 128 * int(rng.integers(1, max(2, hi // 128 + 1)))
+    return int(min(hi, max(1, base + int(rng.integers(-2, 3)))))
+
+
+def _prefill_cases(n=64, seed=20251203):
+    rng = np.random.default_rng(seed)
+    cases = []
+    for i in range(n):
+        D = int(rng.choice([64, 128, 256]))
+        G = int(rng.choice([1, 2, 3, 4, 5, 6, 8, 16, 32]))
+        Hkv = int(rng.integers(1, 4))
+        B = int(rng.integers(1, 3))
+        Lk = _near_tile(rng, 700)
+        Lq = Lk if rng.random() < 0.5 else _near_tile(rng, 700)
+        causal = bool(rng.random() < 0.75)
+        cases.append((B, G * Hkv, Hkv, Lq, Lk, D, causal, seed + i))
+    return cases
+
+
+def _decode_cases(n=48, seed=20251204):
+    rng = np.random.default_rng(seed)
+    cases = []
+    for i in range(n):
+        D = int(rng.choice([64, 128, 256]))
+        G = int(rng.choice([1, 2, 4, 5, 8, 12, 16, 24, 32, 64]))
+        Hkv = int(rng.integers(1, 4))
+        B = int(rng.integers(1, 5))
+        Lmax = _near_tile(rng, 3000)
+        seqlens = [int(x) for x in rng.integers(0, Lmax + 1, size=B)]
+        seqlens[int(rng.integers(0, B))] = Lmax   # one full-length sequence per case
+        cases.append((B, G * Hkv, Hkv, Lmax, D, seqlens, seed + i))
+    return cases
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Lq,Lk,D,causal,seed", _prefill_cases())
+def test_random_prefill(oracle_mod, B, Hq, Hkv, Lq, Lk, D, causal, seed):
+    q, k, v = W.prefill_inputs(B, Hq, Hkv, Lq, Lk, D, seed=seed)
+    scale = 1.0 / math.sqrt(D)
+    out, lse = prefill(q.cuda(), k.cuda(), v.cuda(), scale=scale, is_causal=causal)
+    torch.cuda.synchronize()
+    assert device_error(reset=True) == 0
+    ref_o, ref_l = oracle_mod.attention_prefill(q, k, v, scale, causal)
+    assert_close(out, lse, ref_o, ref_l, f"B{B} Hq{Hq} Hkv{Hkv} Lq{Lq} Lk{Lk} D{D} causal{causal}")
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Lmax,D,seqlens,seed", _decode_cases())
+def test_random_decode(oracle_mod, B, Hq, Hkv, Lmax, D, seqlens, seed):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(B, Hq, D, generator=g).to(torch.bfloat16)
+    k = torch.randn(B, Hkv, Lmax, D, generator=g).to(torch.bfloat16)
+    v = torch.randn(B, Hkv, Lmax, D, generator=g).to(torch.bfloat16)
+    for b, n in enumerate(seqlens):   # rows past a sequence's length are never read
+        k[b, :, n:] = float("nan")
+        v[b, :, n:] = float("nan")
+    sl = torch.tensor(seqlens, dtype=torch.int32)
+    scale = 1.0 / math.sqrt(D)
+    out, lse = decode(q.cuda(), k.cuda(), v.cuda(), sl.cuda(), scale=scale)
+    torch.cuda.synchronize()
+    assert device_error(reset=True) == 0
+    ref_o, ref_l = oracle_mod.attention_decode(q, k, v, sl, scale)
+    assert_close(out, lse, ref_o, ref_l, f"B{B} Hq{Hq} Hkv{Hkv} Lmax{Lmax} D{D} seqlens{seqlens}")
