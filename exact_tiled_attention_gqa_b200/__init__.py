@@ -27,7 +27,7 @@ import torch
 from . import _native
 from ._native import AttnError
 
-__all__ = ["prefill", "prefill_host", "decode", "decode_host", "decode_host_workspace_size", "decode_partial", "decode_merge", "decode_merge_peers", "kvp_signal",
+__all__ = ["prefill", "prefill_workspace_size", "prefill_host", "decode", "decode_host", "decode_host_workspace_size", "decode_partial", "decode_merge", "decode_merge_peers", "kvp_signal",
            "kvp_wait", "decode_mq", "decode_paged", "decode_noalloc", "decode_kv8", "decode_kv8_paged", "prefill_host_scratch_size", "decode_workspace_size", "decode_mq_workspace_size",
            "decode_kv8_workspace_size", "device_error", "AttnError", "library_path"]
 
@@ -107,10 +107,19 @@ def _squeezed_results(out, lse, q4: torch.Tensor, want_lse: bool, squeezed: bool
     return out, lse
 
 
+def prefill_workspace_size(B: int, Hq: int, Hkv: int, Lq: int, Lk: int, D: int, is_causal: bool = True) -> int:
+    return int(_native.lib().attn_prefill_workspace_size(B, Hq, Hkv, Lq, Lk, D, int(bool(is_causal))))
+
+
 def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: Optional[float] = None,
             is_causal: bool = True, out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-            want_lse: bool = True, stream=None):
-    """Exact GQA attention.  q [B,Hq,Lq,D], k/v [B,Hkv,Lk,D] bf16 (CUDA, contiguous)."""
+            want_lse: bool = True, workspace: Optional[torch.Tensor] = None, split: bool = True, stream=None):
+    """Exact GQA attention.  q [B,Hq,Lq,D], k/v [B,Hkv,Lk,D] bf16 (CUDA, contiguous).
+
+    With split (default) the call goes through attn_prefill_ws whenever
+    prefill_workspace_size(...) is non-zero (a launch ending in a part-filled
+    wave of near-equal units), using `workspace` or a new one; split=False is
+    always attn_prefill."""
     for n, t in (("q", q), ("k", k), ("v", v)):
         _check_tensor(n, t, torch.bfloat16, 4)
     B, Hq, Lq, D = q.shape
@@ -123,9 +132,17 @@ def prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, *, scale: Optiona
     out = _result("out", out, torch.bfloat16, q.shape, q.device)
     lse = _result("lse", lse, torch.float32, (B, Hq, Lq), q.device, want_lse)
     with torch.cuda.device(q.device):
-        st = _native.lib().attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Lq, Lk, D,
-                                        float(scale), int(bool(is_causal)), _stream_handle(stream))
-    _native.check(st, "attn_prefill")
+        need = prefill_workspace_size(B, Hq, Hkv, Lq, Lk, D, is_causal) if split and B * Lq * Lk > 0 else 0
+        if need > 0:
+            workspace, ws_bytes = _workspace(workspace, need, q.device)
+            st = _native.lib().attn_prefill_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Lq, Lk,
+                                               D, float(scale), int(bool(is_causal)), _ptr(workspace), ws_bytes,
+                                               _stream_handle(stream))
+            _native.check(st, "attn_prefill_ws")
+        else:
+            st = _native.lib().attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv, Lq, Lk, D,
+                                            float(scale), int(bool(is_causal)), _stream_handle(stream))
+            _native.check(st, "attn_prefill")
     return out, lse
 
 

@@ -184,33 +184,23 @@ __global__ void fill_no_key_rows_kernel(__nv_bfloat16* out, float* lse, size_t r
     }
 }
 
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// The launch's parameters that depend only on the sizes (pointers and the
+// scheduling counters are set by the caller).
 template <int D>
-int launch_prefill(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
-                   int Lq, int Lk, float scale, int is_causal, cudaStream_t stream) {
-    static int smem_done[64];
+PrefillParams prefill_params(int B, int Hq, int Hkv, int Lq, int Lk, float scale, int is_causal) {
     using L = PrefillSmem<D>;
     constexpr int NQ = L::kNQ;
-    const int G = Hq / Hkv;
-    const int P = kBM / G;
-    CUtensorMap tq, tk, tv;
-    int st;
-    if ((st = encode_bf16_3d(&tq, q, D, Lq, static_cast<uint64_t>(B) * Hq, 64, P, G, "q")) != ATTN_OK) return st;
-    if ((st = encode_bf16_3d(&tk, k, D, Lk, static_cast<uint64_t>(B) * Hkv, 64, kBN, 1, "k")) != ATTN_OK) return st;
-    if ((st = encode_bf16_3d(&tv, v, D, Lk, static_cast<uint64_t>(B) * Hkv, 64, kBN, 1, "v")) != ATTN_OK) return st;
-    CUtensorMap to;   // O is written in the same boxes Q is read in
-    if ((st = encode_bf16_3d(&to, out, D, Lq, static_cast<uint64_t>(B) * Hq, 64, P, G, "out")) != ATTN_OK) return st;
-    if ((st = ensure_smem(attn_prefill_sm100_kernel<D, NQ>, L::kAlloc, smem_done)) != ATTN_OK) return st;
-    PrefillParams prm;
-    prm.out = out;
-    prm.lse = lse;
+    PrefillParams prm{};
     prm.B = B;
     prm.Hq = Hq;
     prm.Hkv = Hkv;
     prm.Lq = Lq;
     prm.Lk = Lk;
-    prm.G = G;
-    prm.P = P;
-    prm.n_mblk = (Lq + NQ * P - 1) / (NQ * P);
+    prm.G = Hq / Hkv;
+    prm.P = kBM / prm.G;
+    prm.n_mblk = (Lq + NQ * prm.P - 1) / (NQ * prm.P);
     // Unit order: one band of every group when all of K and V fit in half the
     // L2 (126 MB); otherwise bands of as many groups as fit in 16 MB.  (Bands of
     // 60 MB raised DRAM reads of the Qwen3-8B B4 L8192 prefill from 403 to about
@@ -224,18 +214,104 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
     prm.is_causal = is_causal ? 1 : 0;
     prm.scale_log2 = scale * kLog2e;
     const long long units = static_cast<long long>(B) * Hkv * prm.n_mblk;
-    if (units > 0x7fffffffLL) return fail(ATTN_ERR_UNSUPPORTED, "prefill has too many work units (%lld)", units);
-    prm.n_units = static_cast<int>(units);
+    prm.n_units = units > 0x7fffffffLL ? -1 : static_cast<int>(units);
+    prm.n_full = prm.n_units;
+    prm.n_parts = 1;
+    return prm;
+}
+
+// Key-split tail.  Units are near-equal when every query of a launch sees most
+// keys (chunked prefill: Lq << Lk), and a persistent launch whose unit count is
+// not a multiple of the SM count then ends in a part-filled wave: 256 units on
+// 148 SMs keep 40 SMs idle for half of the launch.  The last (units mod SMs)
+// units of the order are cut into 4 runs of key tiles instead, handed out after
+// the full units, and merged by attn_prefill_merge_kernel.  Only for 1 to 3 full
+// waves (beyond that the tail is a small part of the launch) and only when every
+// unit cut has at least 8 key tiles (2 per part; lighter units cost less than a
+// part's start-up).
+struct PrefillSplit {
+    int n_full = 0, n_items = 0;
+    size_t o_bytes = 0, total = 0;   // partial outputs, then log2-sum-exps
+};
+
+template <int D>
+PrefillSplit prefill_split_plan(const PrefillParams& prm, int n_sm) {
+    using L = PrefillSmem<D>;
+    constexpr int NQ = L::kNQ;
+    PrefillSplit sp;
+    sp.n_full = sp.n_items = prm.n_units;
+    if (!L::kPersistent || prm.n_units <= n_sm || prm.n_units >= 4 * n_sm) return sp;
+    const int R = prm.n_units % n_sm;
+    if (R == 0) return sp;
+    for (int i = prm.n_units - R; i < prm.n_units; ++i)
+        if (prefill_unit<NQ>(prm, i).n_kt < 2 * kPrefillSplitParts) return sp;
+    sp.n_full = prm.n_units - R;
+    sp.n_items = sp.n_full + R * kPrefillSplitParts;
+    const size_t rows = static_cast<size_t>(R) * kPrefillSplitParts * NQ * kBM;
+    sp.o_bytes = align256(rows * D * sizeof(float));
+    sp.total = sp.o_bytes + align256(rows * sizeof(float));
+    return sp;
+}
+
+int device_sm_count(int* n_sm) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(n_sm, cudaDevAttrMultiProcessorCount, dev);
+    return e == cudaSuccess ? ATTN_OK : fail(ATTN_ERR_CUDA, "SM count: %s", cudaGetErrorString(e));
+}
+
+template <int D>
+int launch_prefill(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
+                   int Lq, int Lk, float scale, int is_causal, cudaStream_t stream, bool ws_call = false,
+                   void* workspace = nullptr, size_t workspace_bytes = 0) {
+    static int smem_done[64];
+    using L = PrefillSmem<D>;
+    constexpr int NQ = L::kNQ;
+    const int G = Hq / Hkv;
+    const int P = kBM / G;
+    CUtensorMap tq, tk, tv;
+    int st;
+    if ((st = encode_bf16_3d(&tq, q, D, Lq, static_cast<uint64_t>(B) * Hq, 64, P, G, "q")) != ATTN_OK) return st;
+    if ((st = encode_bf16_3d(&tk, k, D, Lk, static_cast<uint64_t>(B) * Hkv, 64, kBN, 1, "k")) != ATTN_OK) return st;
+    if ((st = encode_bf16_3d(&tv, v, D, Lk, static_cast<uint64_t>(B) * Hkv, 64, kBN, 1, "v")) != ATTN_OK) return st;
+    CUtensorMap to;   // O is written in the same boxes Q is read in
+    if ((st = encode_bf16_3d(&to, out, D, Lq, static_cast<uint64_t>(B) * Hq, 64, P, G, "out")) != ATTN_OK) return st;
+    if ((st = ensure_smem(attn_prefill_sm100_kernel<D, NQ>, L::kAlloc, smem_done)) != ATTN_OK) return st;
+    PrefillParams prm = prefill_params<D>(B, Hq, Hkv, Lq, Lk, scale, is_causal);
+    if (prm.n_units < 0) return fail(ATTN_ERR_UNSUPPORTED, "prefill has too many work units");
+    prm.out = out;
+    prm.lse = lse;
     prm.sched = nullptr;
-    long long grid = units;
+    long long grid = prm.n_units;
+    bool split = false;
     if (L::kPersistent) {   // one CTA per SM, each taking units until they run out
         int n_sm = 0;
         if ((st = device_sms_and_sched(stream, &n_sm, &prm.sched)) != ATTN_OK) return st;
-        grid = std::min<long long>(units, n_sm);
+        if (ws_call) {
+            const PrefillSplit sp = prefill_split_plan<D>(prm, n_sm);
+            if (sp.n_items != prm.n_units) {
+                if (workspace == nullptr || workspace_bytes < sp.total)
+                        return fail(ATTN_ERR_WORKSPACE, "prefill workspace needs %zu bytes, got %zu", sp.total,
+                                workspace ? workspace_bytes : static_cast<size_t>(0));
+                prm.n_full = sp.n_full;
+                prm.n_parts = kPrefillSplitParts;
+                prm.n_units = sp.n_items;
+                prm.part_o = static_cast<float*>(workspace);
+                prm.part_l = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + sp.o_bytes);
+                split = true;
+            }
+        }
+        grid = std::min<long long>(prm.n_units, n_sm);
     }
     attn_prefill_sm100_kernel<D, NQ>
         <<<static_cast<unsigned>(grid), prefill_threads<NQ>(), L::kAlloc, stream>>>(tq, tk, tv, to, prm);
-    return check_launch("attn_prefill_sm100_kernel");
+    if ((st = check_launch("attn_prefill_sm100_kernel")) != ATTN_OK || !split) return st;
+    if constexpr (L::kPersistent) {
+        const long long rows = static_cast<long long>(prm.n_units - prm.n_full) / prm.n_parts * NQ * kBM;
+        attn_prefill_merge_kernel<D, NQ><<<static_cast<unsigned>((rows + 3) / 4), 128, 0, stream>>>(prm);
+        return check_launch("attn_prefill_merge_kernel");
+    }
+    return st;
 }
 
 // Cache rows per decode split (always a multiple of 64, the tile height).
@@ -282,7 +358,6 @@ int decode_chunk(int B, int Hkv, int Lmax, bool tc_path, int D) {
     return best;
 }
 
-size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 struct DecodeLayout {
     int chunk, n_splits;
@@ -490,13 +565,19 @@ int check_common(const void* q, const void* k, const void* v, const void* out, c
 
 using namespace attn;
 
-extern "C" int attn_prefill(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
-                            int Hkv, int Lq, int Lk, int D, float scale, int is_causal, void* stream) {
+namespace {
+// attn_prefill and attn_prefill_ws: checks, empty cases, then the launch (with
+// the key-split tail when a workspace is given and the plan uses one).
+int prefill_checked(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
+                    int Lq, int Lk, int D, float scale, int is_causal, bool ws_call, void* workspace,
+                    size_t workspace_bytes, void* stream) {
     int st = check_common(q, k, v, out, lse, B, Hq, Hkv, Lq, Lk, D, scale, "Lq", "Lk");
     if (st != ATTN_OK) return st;
     if (Hq / Hkv > kBM) return fail(ATTN_ERR_UNSUPPORTED, "group size G=%d > %d", Hq / Hkv, kBM);
     if (static_cast<long long>(B) * Hq > 0x7fffffffLL || static_cast<long long>(B) * Hkv > 0x7fffffffLL)
         return fail(ATTN_ERR_UNSUPPORTED, "B*H too large");
+    if (workspace != nullptr && (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return fail(ATTN_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
     if (B == 0 || Lq == 0) return ok();
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (Lk == 0) {
@@ -505,10 +586,44 @@ extern "C" int attn_prefill(const void* q, const void* k, const void* v, void* o
         st = check_launch("fill_no_key_rows_kernel");
         return st == ATTN_OK ? ok() : st;
     }
-    st = (D == 256)   ? launch_prefill<256>(q, k, v, out, lse, B, Hq, Hkv, Lq, Lk, scale, is_causal, s)
-         : (D == 128) ? launch_prefill<128>(q, k, v, out, lse, B, Hq, Hkv, Lq, Lk, scale, is_causal, s)
-                      : launch_prefill<64>(q, k, v, out, lse, B, Hq, Hkv, Lq, Lk, scale, is_causal, s);
+    st = (D == 256) ? launch_prefill<256>(q, k, v, out, lse, B, Hq, Hkv, Lq, Lk, scale, is_causal, s, ws_call,
+                                          workspace, workspace_bytes)
+         : (D == 128)
+             ? launch_prefill<128>(q, k, v, out, lse, B, Hq, Hkv, Lq, Lk, scale, is_causal, s, ws_call, workspace,
+                                   workspace_bytes)
+             : launch_prefill<64>(q, k, v, out, lse, B, Hq, Hkv, Lq, Lk, scale, is_causal, s, ws_call, workspace,
+                                  workspace_bytes);
     return st == ATTN_OK ? ok() : st;
+}
+}  // namespace
+
+extern "C" int attn_prefill(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
+                            int Hkv, int Lq, int Lk, int D, float scale, int is_causal, void* stream) {
+    return prefill_checked(q, k, v, out, lse, B, Hq, Hkv, Lq, Lk, D, scale, is_causal, false, nullptr, 0, stream);
+}
+
+extern "C" size_t attn_prefill_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int D, int is_causal) {
+    if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Hq / Hkv > kBM || Lq < 1 || Lk < 1 ||
+        (D != 64 && D != 128 && D != 256))
+        return 0;
+    int n_sm = 0;
+    if (device_sm_count(&n_sm) != ATTN_OK) return 0;
+    PrefillSplit sp;
+    if (D == 128) {
+        const PrefillParams prm = prefill_params<128>(B, Hq, Hkv, Lq, Lk, 1.0f, is_causal);
+        if (prm.n_units > 0) sp = prefill_split_plan<128>(prm, n_sm);
+    } else if (D == 64) {
+        const PrefillParams prm = prefill_params<64>(B, Hq, Hkv, Lq, Lk, 1.0f, is_causal);
+        if (prm.n_units > 0) sp = prefill_split_plan<64>(prm, n_sm);
+    }
+    return sp.total;
+}
+
+extern "C" int attn_prefill_ws(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,
+                               int Hkv, int Lq, int Lk, int D, float scale, int is_causal, void* workspace,
+                               size_t workspace_bytes, void* stream) {
+    return prefill_checked(q, k, v, out, lse, B, Hq, Hkv, Lq, Lk, D, scale, is_causal, true, workspace,
+                           workspace_bytes, stream);
 }
 
 namespace attn {

@@ -95,6 +95,7 @@ static_assert(2 * kSoftmaxRegs + kControlRegs == 3 * kPrefillLaunchRegs, "regist
 constexpr int kBM = 128;               // rows per Q tile (MMA M)
 constexpr int kBN = 128;               // keys per K/V tile
 constexpr float kRescaleLog2 = 8.0f;
+constexpr int kPrefillSplitParts = 4;  // runs of key tiles a key-split unit is cut into
 
 template <int D>
 struct PrefillSmem {
@@ -154,12 +155,21 @@ struct PrefillParams {
     int is_causal;
     float scale_log2;   // scale * log2(e)
     int* sched;         // persistent launches: this launch's two counters (zero at launch)
+    // Key-split tail (persistent launches with a workspace): units n_full .. of the
+    // order are each cut into n_parts runs of key tiles; work items n_full + t
+    // (t = split unit * n_parts + part) write fp32 partials to part_o
+    // [t][NQ * 128 rows][D] and log2-sum-exps to part_l [t][NQ * 128], merged by
+    // attn_prefill_merge_kernel.  n_units counts items; n_full == n_units: no split.
+    int n_full, n_parts;
+    float* part_o;
+    float* part_l;
 };
 
-// One work unit: batch b, KV head g, the NQ * P query positions from p_begin,
-// and how many 128-key tiles the latest of them sees.
+// One work item: batch b, KV head g, the NQ * P query positions from p_begin,
+// and the key tiles kt0 .. kt0 + n_kt - 1 it covers (all the latest position
+// sees, unless part >= 0: a run of them, partial results to item slot `part`).
 struct PrefillUnit {
-    int b, g, p_begin, n_kt;
+    int b, g, p_begin, n_kt, kt0, part;
 };
 
 // Unit `idx` of a launch.  Units run band by band: a band is `band`
@@ -168,13 +178,21 @@ struct PrefillUnit {
 // find their K/V there.  Within a band the heaviest (latest) position blocks
 // of all its groups come first: the longest-first order that keeps the tail of
 // a causal launch short, since the last units handed out are the lightest.
+// Items past n_full are the parts of the units n_full .. of this order (the
+// lightest, handed out last), each a contiguous run of about n_kt / n_parts key tiles.
 template <int NQ>
-__device__ __forceinline__ PrefillUnit prefill_unit(const PrefillParams& p, int idx) {
+__host__ __device__ __forceinline__ PrefillUnit prefill_unit(const PrefillParams& p, int idx) {
+    int part = -1, kpart = 0;
+    if (idx >= p.n_full) {
+        part = idx - p.n_full;
+        kpart = part % p.n_parts;
+        idx = p.n_full + part / p.n_parts;
+    }
     const int n_bh = p.B * p.Hkv;
     const int per_band = p.band * p.n_mblk;
     const int k = idx / per_band;
     const int g0 = k * p.band;
-    const int bs = min(p.band, n_bh - g0);   // groups in this band
+    const int bs = (p.band < n_bh - g0) ? p.band : n_bh - g0;   // groups in this band
     const int local = idx - k * per_band;
     const int mblk = p.n_mblk - 1 - local / bs;
     const int bh = g0 + local % bs;
@@ -183,10 +201,17 @@ __device__ __forceinline__ PrefillUnit prefill_unit(const PrefillParams& p, int 
     u.g = bh % p.Hkv;
     u.p_begin = mblk * NQ * p.P;
     const long off = static_cast<long>(p.Lk) - static_cast<long>(p.Lq);
-    const int p_last = min(u.p_begin + NQ * p.P, p.Lq) - 1;
-    const long last_key = p.is_causal ? min(static_cast<long>(p_last) + off, static_cast<long>(p.Lk) - 1)
-                                      : static_cast<long>(p.Lk) - 1;
+    const int p_end = (u.p_begin + NQ * p.P < p.Lq) ? u.p_begin + NQ * p.P : p.Lq;
+    const long lk1 = static_cast<long>(p.Lk) - 1;
+    const long last_key = p.is_causal ? ((p_end - 1 + off < lk1) ? p_end - 1 + off : lk1) : lk1;
     u.n_kt = last_key < 0 ? 0 : static_cast<int>(last_key / kBN) + 1;
+    u.kt0 = 0;
+    u.part = part;
+    if (part >= 0) {
+        const int total = u.n_kt;
+        u.kt0 = kpart * total / p.n_parts;
+        u.n_kt = (kpart + 1) * total / p.n_parts - u.kt0;
+    }
     return u;
 }
 
@@ -315,8 +340,8 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
                 if (!have) break;
                 const PrefillUnit u = prefill_unit<NQ>(p, idx);
                 ATTN_CHECK(idx >= 0 && u.b >= 0 && u.b < p.B && u.g >= 0 && u.g < p.Hkv && u.p_begin >= 0 &&
-                           u.p_begin < p.Lq && u.p_begin % (NQ * P) == 0 && u.n_kt >= 0 &&
-                           u.n_kt <= (p.Lk + kBN - 1) / kBN);
+                           u.p_begin < p.Lq && u.p_begin % (NQ * P) == 0 && u.n_kt >= 0 && u.kt0 >= 0 &&
+                           u.kt0 + u.n_kt <= (p.Lk + kBN - 1) / kBN);
                 // The next unit is taken once this one's loads are all issued (about
                 // two key tiles before its MMAs end), not earlier: a CTA that claimed
                 // its next unit at the start of a long one would hold it back from SMs
@@ -359,7 +384,7 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
                     const CUtensorMap* map = is_v ? &tm_v : &tm_k;
                     for (int kb = 0; kb < L::kItemKB; ++kb)
                         tma_load_3d(sKV + st * L::kItemBytes + kb * L::kBlockBytes, map, bar_kv_full(st),
-                                    (kb0 + kb) * 64, j * kBN, kv_row);
+                                    (kb0 + kb) * 64, (u.kt0 + j) * kBN, kv_row);
                     ++t;
                 }
                 if (!ok) break;
@@ -715,7 +740,7 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
                 float sv[kBN];
 #pragma unroll
                 for (int c = 0; c < kBN; ++c) sv[c] = __uint_as_float(sr[c]);
-                const long key0 = static_cast<long>(j) * kBN;
+                const long key0 = static_cast<long>(u.kt0 + j) * kBN;
                 ATTN_CHECK(key0 < p.Lk);
                 const bool masked = key0 + kBN - 1 > tile_min_bound;
                 if (masked) {
@@ -843,6 +868,35 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
                 tc_fence_after_sync();
             }
             const float inv_l = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
+            if (u.part >= 0) {
+                // a run of the unit's key tiles: O / l in fp32 and the log2-sum-exp to
+                // this item's slot, every row of the tile (attn_prefill_merge_kernel
+                // combines the unit's parts and skips padding rows)
+                ATTN_CHECK(p.part_o != nullptr && u.part < (p.n_units - p.n_full));
+                const size_t prow = (static_cast<size_t>(u.part) * NQ + q) * kBM + r;
+                float* dst = p.part_o + prow * D;
+#pragma unroll 1
+                for (int c = 0; c < D; c += 32) {
+                    uint32_t orr[32];
+                    if (have_o) {
+                        tmem_ld_32x32b_x32(tO + c, orr);
+                        tmem_wait_ld();
+                        reg_fence<32>(orr);
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) orr[i] = 0u;
+                    }
+#pragma unroll
+                    for (int i = 0; i < 32; i += 4)
+                        *reinterpret_cast<float4*>(dst + c + i) =
+                            make_float4(__uint_as_float(orr[i]) * inv_l, __uint_as_float(orr[i + 1]) * inv_l,
+                                        __uint_as_float(orr[i + 2]) * inv_l, __uint_as_float(orr[i + 3]) * inv_l);
+                }
+                p.part_l[prow] = (l_exact > 0.0f) ? m_run + __log2f(l_exact) : -INFINITY;
+                tiles += n_kt;
+                if (n_kt > 0) ++nu;
+                continue;
+            }
             const int q_head0 = u.b * p.Hq + u.g * p.G;
             ATTN_CHECK(tile_p0 >= 0 && q_head0 >= 0 && q_head0 + p.G <= p.B * p.Hq);
             auto o_cols = [&](int c, uint32_t* ob) {   // 32 columns from c, packed into 16 words
@@ -923,6 +977,62 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
         tc_fence_after_sync();
         tmem_dealloc(tmem, 512);
     }
+}
+
+// Merge of the key-split units' parts (PrefillParams: n_full, n_parts, part_o,
+// part_l): out = sum_k 2^(lse_k - lse) O_k and lse = log2 sum_k 2^lse_k (stored
+// as natural log), per query row; one warp per row of a unit's NQ Q tiles, each
+// lane D / 32 columns, all of a row's loads issued before any is used.  Rows
+// past G * P or past Lq are padding: skipped.
+template <int D, int NQ>
+__global__ void __launch_bounds__(128) attn_prefill_merge_kernel(const PrefillParams p) {
+    constexpr int kPer = D / 32;
+    constexpr int kParts = kPrefillSplitParts;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row = blockIdx.x * 4 + warp;                  // over split units x NQ x 128
+    const int n_split = (p.n_units - p.n_full) / kParts;
+    if (row >= n_split * NQ * kBM) return;
+    const int su = row / (NQ * kBM);
+    const int q = (row / kBM) % NQ;
+    const int r = row % kBM;
+    const PrefillUnit u = prefill_unit<NQ>(p, p.n_full + su * kParts);   // b, g, p_begin of the unit
+    const int pos = u.p_begin + q * p.P + r % p.P;
+    if (r >= p.G * p.P || pos >= p.Lq) return;
+    const int h = u.g * p.G + r / p.P;
+    float lk[kParts], ov[kParts][kPer];
+#pragma unroll
+    for (int k = 0; k < kParts; ++k) {
+        const size_t prow = (static_cast<size_t>(su * kParts + k) * NQ + q) * kBM + r;
+        lk[k] = p.part_l[prow];
+        const float* src = p.part_o + prow * D + lane * kPer;
+#pragma unroll
+        for (int i = 0; i < kPer; i += 2) {
+            const float2 v = *reinterpret_cast<const float2*>(src + i);
+            ov[k][i] = v.x;
+            ov[k][i + 1] = v.y;
+        }
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int k = 0; k < kParts; ++k) M = fmaxf(M, lk[k]);
+    float acc[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) acc[i] = 0.0f;
+    float L = 0.0f;
+#pragma unroll
+    for (int k = 0; k < kParts; ++k) {
+        const float w = (lk[k] == -INFINITY) ? 0.0f : ex2_approx(lk[k] - M);
+        L += w;
+#pragma unroll
+        for (int i = 0; i < kPer; ++i) acc[i] = fmaf(w, ov[k][i], acc[i]);
+    }
+    const float inv = (L > 0.0f) ? 1.0f / L : 0.0f;
+    const size_t orow = (static_cast<size_t>(u.b) * p.Hq + h) * p.Lq + pos;
+    ATTN_CHECK(u.b < p.B && h < p.Hq && pos < p.Lq);
+    __nv_bfloat16* o = static_cast<__nv_bfloat16*>(p.out) + orow * D + lane * kPer;
+#pragma unroll
+    for (int i = 0; i < kPer; i += 2) *reinterpret_cast<uint32_t*>(o + i) = pack_bf16x2(acc[i] * inv, acc[i + 1] * inv);
+    if (p.lse != nullptr && lane == 0) p.lse[orow] = (L > 0.0f) ? (M + __log2f(L)) * kLn2 : -INFINITY;
 }
 
 }  // namespace attn

@@ -112,6 +112,35 @@ int attn_prefill(const void* q, const void* k, const void* v, void* out, float* 
                  void* stream);
 
 /*
+ * attn_prefill_workspace_size / attn_prefill_ws -- attn_prefill with a
+ * workspace it may use to even out the end of a launch.
+ *
+ * Same operation, arguments, layouts, limits and results as attn_prefill (the
+ * guide's eager computation, tiled), plus:
+ *   workspace   device memory of attn_prefill_workspace_size(...) bytes,
+ *               256-byte aligned, owned by the caller; may be NULL when that
+ *               size is 0
+ * A launch of D <= 128 takes its work units (a KV group, 2 x 128 query rows)
+ * one wave per SM at a time.  When every query of the launch sees most keys
+ * (chunked prefill, Lq much smaller than Lk) the units are nearly equal, and a
+ * unit count between 1 and 4 waves that is not a multiple of the SM count ends
+ * in a part-filled wave.  attn_prefill_ws then cuts the units of that last
+ * wave into 4 runs of key tiles, writes their normalised fp32 partial results
+ * and log-sum-exps to the workspace and merges them (the single-device form of
+ * the split over keys of the NVIDIA attention page, "Parameter four:
+ * parallelism").  The result is the same attention up to the rounding of the
+ * merge.  attn_prefill_workspace_size returns 0 when no such split applies
+ * (then attn_prefill_ws is attn_prefill); it depends on the sizes and on the
+ * current device's SM count.  Errors: as attn_prefill, plus ATTN_ERR_WORKSPACE
+ * for a workspace smaller than required and ATTN_ERR_INVALID_ARG for a
+ * misaligned one.
+ */
+size_t attn_prefill_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int D, int is_causal);
+int attn_prefill_ws(const void* q, const void* k, const void* v, void* out, float* lse,
+                    int B, int Hq, int Hkv, int Lq, int Lk, int D, float scale, int is_causal,
+                    void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * attn_prefill_host_scratch_size / attn_prefill_host -- attn_prefill with
  * q, k, v, out and lse in HOST memory: the call copies the inputs to the device,
  * computes, and copies the results back, overlapping the three.

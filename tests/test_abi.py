@@ -210,6 +210,16 @@ def test_prefill_host_rejects(lib):
     assert s(2, 8, 2, 64, 64, 128) > 0 and s(2, 8, 2, 64, 64, 96) == 0 and s(0, 8, 2, 64, 64, 128) == 0
 
 
+def test_prefill_ws_rejects(lib):
+    f = lambda **kw: lib.attn_prefill_ws(*[kw.get(n, d) for n, d in (
+        ("q", A), ("k", A), ("v", A), ("out", A), ("lse", NULL), ("B", 1), ("Hq", 8), ("Hkv", 2), ("Lq", 16),
+        ("Lk", 16), ("D", 128), ("scale", 0.1), ("causal", 1), ("ws", NULL), ("wsb", 0))], None)
+    assert f(ws=ctypes.c_void_p(0x10010), wsb=1024) == -1 and f(q=NULL) == -1 and f(Hq=7) == -1
+    assert f(D=96) == -2 and f(B=0) == 0 and f(Lq=0) == 0
+    s = lib.attn_prefill_workspace_size
+    assert s(1, 8, 2, 16, 16, 96, 1) == 0 and s(0, 8, 2, 16, 16, 128, 1) == 0 and s(1, 8, 3, 16, 16, 128, 1) == 0
+
+
 def test_decode_host_rejects(lib):
     f = lambda **kw: lib.attn_decode_host(*[kw.get(n, d) for n, d in (
         ("q", A), ("k", A), ("v", A), ("sl", A), ("out", A), ("lse", NULL), ("B", 2), ("Hq", 8), ("Hkv", 2),

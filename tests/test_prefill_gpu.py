@@ -9,7 +9,7 @@ import numpy as np
 import pytest
 import torch
 
-from exact_tiled_attention_gqa_b200 import device_error, prefill
+from exact_tiled_attention_gqa_b200 import device_error, prefill, prefill_workspace_size
 from exact_tiled_attention_gqa_b200 import workloads as W
 from parity import assert_close
 
@@ -183,3 +183,25 @@ def test_full_size_every_row(oracle_mod, shape):
         ref_o, ref_l = oracle_mod.attention_prefill(q[b:b + 1], k[b:b + 1], v[b:b + 1], shape.scale, shape.is_causal)
         assert_close(out[b:b + 1], lse[b:b + 1], ref_o, ref_l, f"{shape.name} b{b}")
         del ref_o, ref_l
+
+
+@pytest.mark.parametrize("D,Lq,Lk,causal", [(128, 2048, 4096, True), (64, 2048, 3000, True), (128, 2048, 1500, False)])
+def test_key_split_tail(oracle_mod, D, Lq, Lk, causal):
+    """256 near-equal work units on 148 SMs: the 108 units of the part-filled second
+    wave are cut into 4 runs of key tiles, written as fp32 partials and merged.  Every
+    element against the oracle, and against the unsplit launch within rounding."""
+    B, Hq, Hkv = 1, 32, 8
+    need = prefill_workspace_size(B, Hq, Hkv, Lq, Lk, D, causal)
+    assert need > 0, "the key split should apply to this launch"
+    q, k, v = W.prefill_inputs(B, Hq, Hkv, Lq, Lk, D, seed=Lq + Lk + D, spike_every=97)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    scale = 1.0 / math.sqrt(D)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+    out, lse = prefill(qd, kd, vd, scale=scale, is_causal=causal, workspace=ws)
+    plain_o, plain_l = prefill(qd, kd, vd, scale=scale, is_causal=causal, split=False)
+    torch.cuda.synchronize()
+    assert device_error(reset=True) == 0
+    ref_o, ref_l = oracle_mod.attention_prefill(q, k, v, scale, causal)
+    assert_close(out, lse, ref_o, ref_l, f"key split D{D} Lq{Lq} Lk{Lk} causal{causal}")
+    assert (out.float() - plain_o.float()).abs().max().item() <= 2e-2
+    assert (lse - plain_l).abs().max().item() <= 1e-3
