@@ -209,6 +209,8 @@ def run_ours(args, rank, world, local_rank):
     ws_bytes = (attn.decode_kv8_workspace_size(dshape.B, dshape.Hq, dshape.Hkv, 1, dshape.Lmax, dshape.D) if kv8
                 else attn.decode_workspace_size(dshape.B, dshape.Hq, dshape.Hkv, dshape.Lmax, dshape.D))
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    p_ws = torch.empty(max(1, attn.prefill_workspace_size(PREFILL.B, PREFILL.Hq, PREFILL.Hkv, PREFILL.Lq, PREFILL.Lk,
+                                                          PREFILL.D, PREFILL.is_causal)), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     do_pre = args.only in (None, "prefill")
@@ -217,7 +219,7 @@ def run_ours(args, rank, world, local_rank):
     def call_prefill():
         if do_pre:
             attn.prefill(q, k, v, scale=PREFILL.scale, is_causal=PREFILL.is_causal, out=p_out, lse=p_lse,
-                         stream=stream)
+                         workspace=p_ws, stream=stream)
 
     def call_decode():
         if do_dec and kv8:
@@ -467,8 +469,11 @@ def run_sweeps(attn, dev, stream, seed, max_over_ranks):
         o = torch.empty_like(q)
         l = torch.empty((shape.B, shape.Hq, shape.Lq), dtype=torch.float32, device=dev)
         small = (q.numel() + 2 * k.numel()) * 2 < 126e6
+        ws = torch.empty(max(1, attn.prefill_workspace_size(shape.B, shape.Hq, shape.Hkv, shape.Lq, shape.Lk,
+                                                            shape.D, True)), dtype=torch.uint8, device=dev)
         ms = max_over_ranks(_time_calls(lambda: attn.prefill(q, k, v, scale=shape.scale, is_causal=True, out=o,
-                                                              lse=l, stream=stream), stream, n=20, flush=small))
+                                                              lse=l, workspace=ws, stream=stream),
+                                        stream, n=20, flush=small))
         fl = RL.prefill_flops(shape.B, shape.Hq, shape.Lq, shape.Lk, shape.D, True)
         out["prefill"].append({"workload": shape.name, "ms": round(ms, 4), "tflops": round(fl / ms / 1e9, 1),
                                "frac_of_measured_bf16": round(fl / ms / 1e9 / float(peaks["bf16_tflops"]), 4),

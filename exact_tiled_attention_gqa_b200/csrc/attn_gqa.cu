@@ -157,21 +157,47 @@ int device_sms_and_sched(cudaStream_t stream, int* n_sm, int** sched) {
     return ATTN_OK;
 }
 
-// The split combine: one warp per row (four rows per CTA) when rows have few
-// splits, four warps per row when they have more than 16 (their reads then take
-// four times fewer dependent rounds).
-template <int D, bool F32>
-void launch_combine(const DecodeParams& prm, void* out, float* lse, int rows, cudaStream_t stream) {
-    if (prm.n_splits > 16)
-        attn_decode_combine_kernel<D, F32, 4><<<rows, 128, 0, stream>>>(prm, out, lse);
-    else
-        attn_decode_combine_kernel<D, F32, 1><<<(rows + 3) / 4, 128, 0, stream>>>(prm, out, lse);
-}
-
 int check_launch(const char* what) {
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return fail(ATTN_ERR_CUDA, "%s launch failed: %s", what, cudaGetErrorString(e));
     return ATTN_OK;
+}
+
+// Launches a kernel that starts with grid_dep_wait() as a programmatic dependent
+// of the kernel before it on the stream: it may be scheduled while that kernel's
+// last CTAs still run (they release it when they start), and reads nothing before
+// that kernel has completed.  Saves the launch gap between a split kernel and its
+// combine.  Static shared memory only.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kernel)(KArgs...), unsigned grid, unsigned block, cudaStream_t stream,
+                             Args... args) {
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
+// The split combine: one warp per row (four rows per CTA) when rows have few
+// splits, four warps per row when they have more than 16 (their reads then take
+// four times fewer dependent rounds).
+template <int D, bool F32>
+int launch_combine(const DecodeParams& prm, void* out, float* lse, int rows, cudaStream_t stream) {
+    const cudaError_t e =
+        (prm.n_splits > 16)
+            ? launch_dependent(attn_decode_combine_kernel<D, F32, 4>, static_cast<unsigned>(rows), 128u, stream, prm,
+                               out, lse)
+            : launch_dependent(attn_decode_combine_kernel<D, F32, 1>, static_cast<unsigned>((rows + 3) / 4), 128u,
+                               stream, prm, out, lse);
+    if (e != cudaSuccess)
+        return fail(ATTN_ERR_CUDA, "attn_decode_combine_kernel launch failed: %s", cudaGetErrorString(e));
+    return check_launch("attn_decode_combine_kernel");
 }
 
 // Rows that see no key at all (Lk == 0): O = 0, LSE = -inf.
@@ -264,7 +290,7 @@ template <int D>
 int launch_prefill(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq, int Hkv,
                    int Lq, int Lk, float scale, int is_causal, cudaStream_t stream, bool ws_call = false,
                    void* workspace = nullptr, size_t workspace_bytes = 0) {
-    static int smem_done[64];
+    static int smem_done[64], smem_done_split[64];
     using L = PrefillSmem<D>;
     constexpr int NQ = L::kNQ;
     const int G = Hq / Hkv;
@@ -276,7 +302,6 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
     if ((st = encode_bf16_3d(&tv, v, D, Lk, static_cast<uint64_t>(B) * Hkv, 64, kBN, 1, "v")) != ATTN_OK) return st;
     CUtensorMap to;   // O is written in the same boxes Q is read in
     if ((st = encode_bf16_3d(&to, out, D, Lq, static_cast<uint64_t>(B) * Hq, 64, P, G, "out")) != ATTN_OK) return st;
-    if ((st = ensure_smem(attn_prefill_sm100_kernel<D, NQ>, L::kAlloc, smem_done)) != ATTN_OK) return st;
     PrefillParams prm = prefill_params<D>(B, Hq, Hkv, Lq, Lk, scale, is_causal);
     if (prm.n_units < 0) return fail(ATTN_ERR_UNSUPPORTED, "prefill has too many work units");
     prm.out = out;
@@ -303,12 +328,23 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
         }
         grid = std::min<long long>(prm.n_units, n_sm);
     }
-    attn_prefill_sm100_kernel<D, NQ>
-        <<<static_cast<unsigned>(grid), prefill_threads<NQ>(), L::kAlloc, stream>>>(tq, tk, tv, to, prm);
-    if ((st = check_launch("attn_prefill_sm100_kernel")) != ATTN_OK || !split) return st;
+    if (!split) {
+        if ((st = ensure_smem(attn_prefill_sm100_kernel<D, NQ, false>, L::kAlloc, smem_done)) != ATTN_OK) return st;
+        attn_prefill_sm100_kernel<D, NQ, false>
+            <<<static_cast<unsigned>(grid), prefill_threads<NQ>(), L::kAlloc, stream>>>(tq, tk, tv, to, prm);
+        return check_launch("attn_prefill_sm100_kernel");
+    }
     if constexpr (L::kPersistent) {
+        if ((st = ensure_smem(attn_prefill_sm100_kernel<D, NQ, true>, L::kAlloc, smem_done_split)) != ATTN_OK)
+            return st;
+        attn_prefill_sm100_kernel<D, NQ, true>
+            <<<static_cast<unsigned>(grid), prefill_threads<NQ>(), L::kAlloc, stream>>>(tq, tk, tv, to, prm);
+        if ((st = check_launch("attn_prefill_sm100_kernel")) != ATTN_OK) return st;
         const long long rows = static_cast<long long>(prm.n_units - prm.n_full) / prm.n_parts * NQ * kBM;
-        attn_prefill_merge_kernel<D, NQ><<<static_cast<unsigned>((rows + 3) / 4), 128, 0, stream>>>(prm);
+        const cudaError_t e =
+            launch_dependent(attn_prefill_merge_kernel<D, NQ>, static_cast<unsigned>((rows + 3) / 4), 128u, stream, prm);
+        if (e != cudaSuccess)
+            return fail(ATTN_ERR_CUDA, "attn_prefill_merge_kernel launch failed: %s", cudaGetErrorString(e));
         return check_launch("attn_prefill_merge_kernel");
     }
     return st;
@@ -472,8 +508,7 @@ int launch_decode_kv8(const void* q, const void* kc, const void* vc, const void*
         st = launch_decode_kv8_split<D, 64, FMT>(tk, tv, tks, tvs, prm, stream);
     if (st != ATTN_OK) return st;
     const int n_rows = B * Hq * Lq;
-    launch_combine<D, false>(prm, out, lse, n_rows, stream);
-    return check_launch("attn_decode_combine_kernel");
+    return launch_combine<D, false>(prm, out, lse, n_rows, stream);
 }
 
 
@@ -533,11 +568,8 @@ int launch_decode(const void* q, const void* kc, const void* vc, const int32_t* 
         st = launch_decode_split<D, 64>(tk, tv, prm, stream);
     if (st != ATTN_OK) return st;
     const int rows = B * Hq * Lq;
-    if (f32_out)
-        launch_combine<D, true>(prm, out, lse, rows, stream);
-    else
-        launch_combine<D, false>(prm, out, lse, rows, stream);
-    return check_launch("attn_decode_combine_kernel");
+    return f32_out ? launch_combine<D, true>(prm, out, lse, rows, stream)
+                   : launch_combine<D, false>(prm, out, lse, rows, stream);
 }
 
 // q/out may be null only when they are empty (B == 0 or L1 == 0); k/v only when

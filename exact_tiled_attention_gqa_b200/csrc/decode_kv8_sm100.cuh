@@ -164,6 +164,7 @@ __global__ void __maxnreg__(200)
     attn_decode_kv8_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                            const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
                            const DecodeParams p) {
+    grid_dep_release();   // the combine launch may be scheduled now
     using L = DecodeKv8Smem<D, FMT>;
     constexpr int kNT = KPW / 8;          // 8-key n-tiles of S per warp
     constexpr int kWPM = kDecKT / KPW;    // warps per 16-row block
@@ -510,6 +511,7 @@ __global__ void __launch_bounds__(kDecThreads, kv8t_min_blocks<NR>())
     attn_decode_kv8t_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                             const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
                             const DecodeParams p) {
+    grid_dep_release();   // the combine launch may be scheduled now
     using L = DecodeKv8tSmem<D, FMT>;
     constexpr int kBlk = D / 32;
     extern __shared__ uint8_t smem_raw[];

@@ -107,6 +107,7 @@ template <int D, int KPW>
 __global__ void __maxnreg__(200)
     attn_decode_split_kernel(const __grid_constant__ CUtensorMap tm_k,
                              const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
+    grid_dep_release();   // the combine launch may be scheduled now
     using L = DecodeSmem<D>;
     constexpr int kNT = KPW / 8;          // 8-key n-tiles of S per warp
     constexpr int kWPM = kDecKT / KPW;    // warps per 16-row block
@@ -414,6 +415,7 @@ __global__ void __maxnreg__(200)
 template <int D, bool F32 = false, int WPR = 1>
 __global__ void __launch_bounds__(128)
     attn_decode_combine_kernel(const DecodeParams p, void* out_ptr, float* lse) {
+    grid_dep_wait();   // launched as a programmatic dependent of the split kernel
     static_assert(WPR == 1 || WPR == 4, "one or four warps per row");
     constexpr int kPer = D / 32;                  // columns per lane
     constexpr int kChunk = (D >= 256) ? 8 : 16;   // splits per warp whose O rows are in registers

@@ -81,6 +81,7 @@ template <int D>
 __global__ void __launch_bounds__(kDtcThreads, DecodeTcSmem<D>::kCtasPerSm)
     attn_decode_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v, const DecodeParams p) {
+    grid_dep_release();   // the combine launch may be scheduled now
     using L = DecodeTcSmem<D>;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw_base = smem_u32(smem_raw);

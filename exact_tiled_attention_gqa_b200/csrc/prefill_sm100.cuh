@@ -180,10 +180,11 @@ struct PrefillUnit {
 // a causal launch short, since the last units handed out are the lightest.
 // Items past n_full are the parts of the units n_full .. of this order (the
 // lightest, handed out last), each a contiguous run of about n_kt / n_parts key tiles.
-template <int NQ>
+// kSplit = false: a launch without a key split (every item a whole unit).
+template <int NQ, bool kSplit = true>
 __host__ __device__ __forceinline__ PrefillUnit prefill_unit(const PrefillParams& p, int idx) {
     int part = -1, kpart = 0;
-    if (idx >= p.n_full) {
+    if (kSplit && idx >= p.n_full) {
         part = idx - p.n_full;
         kpart = part % p.n_parts;
         idx = p.n_full + part / p.n_parts;
@@ -207,7 +208,7 @@ __host__ __device__ __forceinline__ PrefillUnit prefill_unit(const PrefillParams
     u.n_kt = last_key < 0 ? 0 : static_cast<int>(last_key / kBN) + 1;
     u.kt0 = 0;
     u.part = part;
-    if (part >= 0) {
+    if (kSplit && part >= 0) {
         const int total = u.n_kt;
         u.kt0 = kpart * total / p.n_parts;
         u.n_kt = (kpart + 1) * total / p.n_parts - u.kt0;
@@ -215,12 +216,15 @@ __host__ __device__ __forceinline__ PrefillUnit prefill_unit(const PrefillParams
     return u;
 }
 
-template <int D, int NQ>
+// kSplit: the launch has a key-split tail (items past p.n_full write partials);
+// launches without one use the kSplit = false build of the kernel.
+template <int D, int NQ, bool kSplit>
 __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
     attn_prefill_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                               const __grid_constant__ CUtensorMap tm_k,
                               const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
                               const PrefillParams p) {
+    if constexpr (kSplit) grid_dep_release();   // the merge launch may be scheduled now
     using L = PrefillSmem<D>;
     static_assert(L::kNQ == NQ, "Q tiles per CTA follow from D");
     constexpr bool kPersistent = L::kPersistent;
@@ -338,7 +342,7 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
                 unit_slot[s] = have ? idx : -1;
                 mbar_arrive(bar_unit_full(s));
                 if (!have) break;
-                const PrefillUnit u = prefill_unit<NQ>(p, idx);
+                const PrefillUnit u = prefill_unit<NQ, kSplit>(p, idx);
                 ATTN_CHECK(idx >= 0 && u.b >= 0 && u.b < p.B && u.g >= 0 && u.g < p.Hkv && u.p_begin >= 0 &&
                            u.p_begin < p.Lq && u.p_begin % (NQ * P) == 0 && u.n_kt >= 0 && u.kt0 >= 0 &&
                            u.kt0 + u.n_kt <= (p.Lk + kBN - 1) / kBN);
@@ -489,7 +493,7 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
                 const int idx = unit_slot[s];
                 mbar_arrive(bar_unit_empty(s));
                 if (idx < 0) break;
-                const int n_kt = prefill_unit<NQ>(p, idx).n_kt;
+                const int n_kt = prefill_unit<NQ, kSplit>(p, idx).n_kt;
                 if (n_kt == 0) continue;
                 ok = mbar_wait(bar_q_full, static_cast<uint32_t>(nu) & 1u, abort_flag, &g_attn_err, kDevErrTimeout);
               if constexpr (kSplitP) {
@@ -692,7 +696,7 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
             // slot before the warp's release of it.
             if (named_bar_or(wg_bar, 128, !ok || idx < 0)) break;
             if (lane == 0) mbar_arrive(bar_unit_empty(s));
-            const PrefillUnit u = prefill_unit<NQ>(p, idx);
+            const PrefillUnit u = prefill_unit<NQ, kSplit>(p, idx);
             const int n_kt = u.n_kt;
             const int pos = u.p_begin + q * P + (r % P);
             const bool row_valid = (r < rows_used) && (pos < p.Lq);
@@ -868,7 +872,7 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
                 tc_fence_after_sync();
             }
             const float inv_l = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
-            if (u.part >= 0) {
+            if (kSplit && u.part >= 0) {
                 // a run of the unit's key tiles: O / l in fp32 and the log2-sum-exp to
                 // this item's slot, every row of the tile (attn_prefill_merge_kernel
                 // combines the unit's parts and skips padding rows)
@@ -986,6 +990,7 @@ __global__ void __launch_bounds__(prefill_threads<NQ>(), 1)
 // past G * P or past Lq are padding: skipped.
 template <int D, int NQ>
 __global__ void __launch_bounds__(128) attn_prefill_merge_kernel(const PrefillParams p) {
+    grid_dep_wait();   // launched as a programmatic dependent of the prefill kernel
     constexpr int kPer = D / 32;
     constexpr int kParts = kPrefillSplitParts;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

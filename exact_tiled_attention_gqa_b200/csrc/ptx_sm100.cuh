@@ -86,6 +86,17 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 }
 
 // -------------------------------------------------------------------------
+// Programmatic dependent launch.  A kernel launched with the programmatic
+// stream-serialization attribute may be scheduled once every CTA of the kernel
+// before it on the stream has executed grid_dep_release() or exited, so its
+// launch overlaps that kernel's tail; grid_dep_wait() then blocks until that
+// kernel has completed and its memory writes are visible.  Both are no-ops
+// for kernels launched without the attribute.
+// -------------------------------------------------------------------------
+__device__ __forceinline__ void grid_dep_release() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// -------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor), no multicast
 // -------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

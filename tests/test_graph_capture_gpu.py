@@ -1,7 +1,8 @@
 """The device-buffer calls can be captured into a CUDA graph and replayed (the
 inner loop of a serving step): after one ordinary call on the device (which sets
-each kernel's shared-memory limit), prefill, decode and 8-bit decode are captured
-with fixed shapes and buffers, replayed with new inputs copied into those
+each kernel's shared-memory limit), prefill, a prefill that takes the key-split
+tail (a merge kernel launched as a programmatic dependent), decode and 8-bit
+decode are captured with fixed shapes and buffers, replayed with new inputs copied into those
 buffers, and must equal ordinary calls bit for bit."""
 import pytest
 import torch
@@ -32,9 +33,14 @@ def test_capture_and_replay_step():
     k_out, k_lse = torch.empty_like(q8), torch.empty(4, 32, 1, device=dev)
     ws = torch.empty(attn.decode_workspace_size(4, 32, 8, 3000, 128), dtype=torch.uint8, device=dev)
     ws8 = torch.empty(attn.decode_kv8_workspace_size(4, 32, 8, 1, 3000, 128), dtype=torch.uint8, device=dev)
+    sq, sk, sv = (t.to(dev) for t in W.prefill_inputs(1, 32, 8, 2048, 4096, 128, seed=4))
+    s_out, s_lse = torch.empty_like(sq), torch.empty(1, 32, 2048, device=dev)
+    pws = torch.empty(attn.prefill_workspace_size(1, 32, 8, 2048, 4096, 128), dtype=torch.uint8, device=dev)
+    assert pws.numel() > 0
 
     def step(stream=None):
         attn.prefill(q, k, v, out=p_out, lse=p_lse, stream=stream)
+        attn.prefill(sq, sk, sv, out=s_out, lse=s_lse, workspace=pws, stream=stream)
         attn.decode(dq, dk, dv, dsl, out=d_out, lse=d_lse, workspace=ws, stream=stream)
         attn.decode_kv8(q8, k8, v8, ks8, vs8, sl8, out=k_out, lse=k_lse, workspace=ws8, stream=stream)
 
@@ -48,12 +54,13 @@ def test_capture_and_replay_step():
     q.copy_(torch.randn_like(q, dtype=torch.float32).to(torch.bfloat16))
     dq.copy_(torch.randn_like(dq, dtype=torch.float32).to(torch.bfloat16))
     q8.copy_(torch.randn_like(q8, dtype=torch.float32).to(torch.bfloat16))
+    sq.copy_(torch.randn_like(sq, dtype=torch.float32).to(torch.bfloat16))
     g.replay()
     torch.cuda.synchronize()
-    got = [t.clone() for t in (p_out, p_lse, d_out, d_lse, k_out, k_lse)]
+    got = [t.clone() for t in (p_out, p_lse, s_out, s_lse, d_out, d_lse, k_out, k_lse)]
     step()
     torch.cuda.synchronize()
-    want = (p_out, p_lse, d_out, d_lse, k_out, k_lse)
+    want = (p_out, p_lse, s_out, s_lse, d_out, d_lse, k_out, k_lse)
     assert all(torch.equal(a, b) for a, b in zip(got, want))
     del g
 
