@@ -85,6 +85,10 @@ def main():
     prefill_case(1, 32, 8, 256, 16384, 128, True, seed=3, spike=97)
     prefill_case(2, 32, 8, 300, 10000, 128, True, seed=4)
     prefill_case(2, 32, 8, 300, 10000, 64, True, seed=5)
+    # the key-split tail: 256 near-equal units, the last 108 cut into key runs
+    for D, Lk in ((128, 4096), (64, 3000)):
+        assert attn.prefill_workspace_size(1, 32, 8, 2048, Lk, D, True) > 0
+        prefill_case(1, 32, 8, 2048, Lk, D, True, seed=6 + D)
     for G, D in ((4, 128), (16, 64), (32, 128), (64, 128), (4, 256)):
         decode_case(3, 2 * G, 2, 5000, D, [5000, 1, 2500], seed=G + D)
     decode_case(2, 8, 2, 900, 128, [900, 3], seed=9, Lq=4)

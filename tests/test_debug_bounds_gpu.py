@@ -1,8 +1,9 @@
 """The bounds-checking build: the same sources compiled with -DATTN_DEBUG_BOUNDS=1,
 whose kernels check their work-unit mapping, ring positions, TMA coordinates and
 output indices and report a violation in the device error word (they never trap).
-Small parity cases for every kernel family, and persistent prefills whose units
-run in bands of KV groups, go through it in a child process; each must match the
+Small parity cases for every kernel family, persistent prefills whose units run
+in bands of KV groups, and prefills with a key-split tail go through it in a child
+process; each must match the
 oracle with the error word clear."""
 import os
 import subprocess

@@ -6,7 +6,8 @@ run): batch, heads and group size (including group sizes that do not divide
 the 128-row tile), query and key lengths from 1 to a few tiles on either side of
 a tile boundary, head dims 64 / 128 / 256, causal and full attention; decode
 with cache lengths from 0 to Lmax, one to sixteen new rows per sequence, bf16 and
-8-bit caches.  They complement the hand-picked edge cases
+8-bit caches; and prefills of 149 to 591 long work units, whose part-filled last
+wave is cut into key runs and merged.  They complement the hand-picked edge cases
 of the other parity files with combinations nobody chose.
 """
 import math
@@ -15,7 +16,7 @@ import numpy as np
 import pytest
 import torch
 
-from exact_tiled_attention_gqa_b200 import decode, decode_kv8, decode_mq, device_error, prefill
+from exact_tiled_attention_gqa_b200 import decode, decode_kv8, decode_mq, device_error, prefill, prefill_workspace_size
 from exact_tiled_attention_gqa_b200 import workloads as W
 from parity import assert_close
 
@@ -67,6 +68,39 @@ def _decode_cases(n=48, seed=20251204):
         seqlens[int(rng.integers(0, B))] = Lmax   # one full-length sequence per case
         cases.append((B, G * Hkv, Hkv, Lmax, D, seqlens, seed + i))
     return cases
+
+
+def _key_split_cases(n=6, seed=20251207):
+    """Launches of 149 .. 591 units, all of at least 8 key tiles, and not a whole number
+    of 148-unit waves: the shapes whose last wave is cut into key runs."""
+    rng = np.random.default_rng(seed)
+    cases = []
+    while len(cases) < n:
+        D = int(rng.choice([64, 128]))
+        G = int(rng.choice([1, 2, 4, 8]))
+        P = 128 // G
+        Hkv = int(rng.choice([1, 2, 4, 8]))
+        B = int(rng.integers(1, 3))
+        n_mblk = -(-int(rng.integers(160, 580)) // (B * Hkv))
+        Lq = n_mblk * 2 * P - int(rng.integers(0, 2 * P))
+        causal = bool(rng.random() < 0.7)
+        Lk = Lq + int(rng.integers(1024, 3000)) if causal else int(rng.integers(1024, 5000))
+        units = B * Hkv * -(-Lq // (2 * P))
+        if 148 < units < 592 and units % 148 and B * G * Hkv * Lq * Lk <= 3e8:
+            cases.append((B, G * Hkv, Hkv, Lq, Lk, D, causal, seed + len(cases)))
+    return cases
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,Lq,Lk,D,causal,seed", _key_split_cases())
+def test_random_prefill_key_split(oracle_mod, B, Hq, Hkv, Lq, Lk, D, causal, seed):
+    assert prefill_workspace_size(B, Hq, Hkv, Lq, Lk, D, causal) > 0, "the key split should apply"
+    q, k, v = W.prefill_inputs(B, Hq, Hkv, Lq, Lk, D, seed=seed)
+    scale = 1.0 / math.sqrt(D)
+    out, lse = prefill(q.cuda(), k.cuda(), v.cuda(), scale=scale, is_causal=causal)
+    torch.cuda.synchronize()
+    assert device_error(reset=True) == 0
+    ref_o, ref_l = oracle_mod.attention_prefill(q, k, v, scale, causal)
+    assert_close(out, lse, ref_o, ref_l, f"key split B{B} Hq{Hq} Hkv{Hkv} Lq{Lq} Lk{Lk} D{D} causal{causal}")
 
 
 @pytest.mark.parametrize("B,Hq,Hkv,Lq,Lk,D,causal,seed", _prefill_cases())
