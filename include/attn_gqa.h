@@ -30,7 +30,12 @@
  *     row: LSE_i = m_i + ln(sum_j exp(scale * q_i.k_j - m_i)).  A row that
  *     sees no key gets O = 0 and LSE = -inf.
  *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
- *     call only enqueues work on it; none synchronises the host.
+ *     call only enqueues work on it; none synchronises the host.  A call that
+ *     launches two kernels (a split kernel and the combine or merge of its
+ *     partial results) launches the second as a programmatic dependent of the
+ *     first: it may be scheduled while the first is finishing but reads
+ *     nothing before the first has completed, so stream order, events and
+ *     graph capture see the call as one piece of work.
  *   - Return value: ATTN_OK, or a negative attn_status_t.  Argument checks
  *     happen before anything is enqueued, so a failed call has no effect.
  *     attn_last_error() gives a one-line description of the last failure on
