@@ -37,6 +37,7 @@ _vp, _i32, _f32, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_s
 SIGNATURES = {
     "attn_prefill": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp]),
     "attn_prefill_workspace_size": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32, _i32]),
+    "attn_prefill_split_plan": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
     "attn_prefill_ws": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _sz, _vp]),
     "attn_prefill_host_scratch_size": (_sz, [_i32, _i32, _i32, _i32, _i32, _i32]),
     "attn_prefill_host": (_i32, [_vp, _vp, _vp, _vp, _vp, _i32, _i32, _i32, _i32, _i32, _i32, _f32, _i32, _vp, _sz,

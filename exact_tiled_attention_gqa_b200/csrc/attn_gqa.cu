@@ -634,21 +634,30 @@ extern "C" int attn_prefill(const void* q, const void* k, const void* v, void* o
     return prefill_checked(q, k, v, out, lse, B, Hq, Hkv, Lq, Lk, D, scale, is_causal, false, nullptr, 0, stream);
 }
 
+extern "C" size_t attn_prefill_split_plan(int B, int Hq, int Hkv, int Lq, int Lk, int D, int is_causal, int n_sm,
+                                          int* n_full, int* n_items) {
+    PrefillSplit sp;
+    if (B >= 1 && Hq >= 1 && Hkv >= 1 && Hq % Hkv == 0 && Hq / Hkv <= kBM && Lq >= 1 && Lk >= 1 && n_sm >= 1) {
+        if (D == 128) {
+            const PrefillParams prm = prefill_params<128>(B, Hq, Hkv, Lq, Lk, 1.0f, is_causal);
+            if (prm.n_units > 0) sp = prefill_split_plan<128>(prm, n_sm);
+        } else if (D == 64) {
+            const PrefillParams prm = prefill_params<64>(B, Hq, Hkv, Lq, Lk, 1.0f, is_causal);
+            if (prm.n_units > 0) sp = prefill_split_plan<64>(prm, n_sm);
+        }
+    }
+    if (n_full) *n_full = sp.n_full;
+    if (n_items) *n_items = sp.n_items;
+    return sp.total;
+}
+
 extern "C" size_t attn_prefill_workspace_size(int B, int Hq, int Hkv, int Lq, int Lk, int D, int is_causal) {
     if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0 || Hq / Hkv > kBM || Lq < 1 || Lk < 1 ||
         (D != 64 && D != 128 && D != 256))
         return 0;
     int n_sm = 0;
     if (device_sm_count(&n_sm) != ATTN_OK) return 0;
-    PrefillSplit sp;
-    if (D == 128) {
-        const PrefillParams prm = prefill_params<128>(B, Hq, Hkv, Lq, Lk, 1.0f, is_causal);
-        if (prm.n_units > 0) sp = prefill_split_plan<128>(prm, n_sm);
-    } else if (D == 64) {
-        const PrefillParams prm = prefill_params<64>(B, Hq, Hkv, Lq, Lk, 1.0f, is_causal);
-        if (prm.n_units > 0) sp = prefill_split_plan<64>(prm, n_sm);
-    }
-    return sp.total;
+    return attn_prefill_split_plan(B, Hq, Hkv, Lq, Lk, D, is_causal, n_sm, nullptr, nullptr);
 }
 
 extern "C" int attn_prefill_ws(const void* q, const void* k, const void* v, void* out, float* lse, int B, int Hq,

@@ -540,6 +540,18 @@ int attn_selftest_wait(unsigned long long limit_ns, int* result, void* stream);
  */
 int attn_prefill_sched_busy(int* busy);
 
+/*
+ * attn_prefill_split_plan -- diagnostic, host only (no device call): the
+ * key-split plan attn_prefill_ws would use on a device with n_sm SMs.  Writes
+ * *n_full (whole work units handed out first) and *n_items (work items of the
+ * launch: n_full plus 4 per cut unit; n_items == n_full when nothing is cut;
+ * both 0 for head dim 256, whose launches are not persistent, and for invalid
+ * arguments) and returns the workspace bytes (attn_prefill_workspace_size on
+ * such a device; 0 when nothing is cut).  n_full / n_items may be NULL.
+ */
+size_t attn_prefill_split_plan(int B, int Hq, int Hkv, int Lq, int Lk, int D, int is_causal, int n_sm,
+                               int* n_full, int* n_items);
+
 /* attn_status_string -- a static name for a status code; never NULL. */
 const char* attn_status_string(int status);
 
