@@ -357,11 +357,13 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
 //    carry more setup than the split kernel's (TMEM, the Q tile, a partial per
 //    row for the combine), so splits are long, and the split length balances
 //    the waves: of the multiples of 64 in [512, 8192], the one that minimises
-//    waves x (rows per split + 512), with waves = splits / (148 SMs x 2 CTAs)
-//    rounded up and the split count taken at Lmax.  Measured on B200 at 131072
-//    cached rows: G = 32 got 7296-row splits (288 CTAs, one wave) and went from
-//    0.179 to 0.169 ms against 4096-row splits (512 CTAs); G = 64 (3584-row
-//    splits, 296 CTAs) was unchanged.
+//    waves x (rows per split + 512), with waves = splits / 256 rounded up and
+//    the split count taken at Lmax.  256 CTAs per wave is measured, not the
+//    148 SMs x 2 CTAs that fit: at 131072 cached rows and batch 8, splits of
+//    4096 rows (G = 64, 256 CTAs) took 0.0938 ms against 0.0960 for 3584 (296
+//    CTAs), 0.098 for 4608 and 0.106 for 1792; splits of 8192 rows (G = 32,
+//    256 CTAs) took 0.163-0.164 ms against 0.165-0.166 for 7296 (288 CTAs) and
+//    0.178 for 10240.
 //  - tcgen05 kernel, D = 256 (one CTA per SM): the largest power of two in
 //    [512, 4096] that still gives 148 CTAs (the balanced rule above, at one CTA
 //    per SM, made the head-dim-256 decode batch 8 % slower: with lengths spread
@@ -378,7 +380,7 @@ int decode_chunk(int B, int Hkv, int Lmax, bool tc_path, int D) {
         while (chunk > min_chunk && groups * ((Lmax + chunk - 1) / chunk) < target) chunk >>= 1;
         return chunk;
     }
-    const long long slots = 148LL * 2;
+    const long long slots = 256;
     int best = 512;
     long long best_cost = -1;
     for (int c = 512; c <= 8192; c += 64) {
