@@ -116,6 +116,23 @@ def test_workspace_size(lib):
     assert f(64, 32, 8, 32768, 128) >= 64 * 32 * (128 + 1) * 4
 
 
+def _decode_ws(splits, B, Hq, D=128):
+    rows = B * Hq * splits
+    return -(-rows * D * 4 // 256) * 256 + -(-rows * 4 // 256) * 256
+
+
+def test_decode_split_lengths(lib):
+    """The split lengths the decode picks for the measured workloads, seen through the
+    workspace size (one fp32 partial row and LSE per query row and split)."""
+    f = lib.attn_decode_workspace_size
+    # group sweep, batch 8, 131072 cached rows: tcgen05 kernel, splits of 4096 rows at
+    # G = 64 (32 splits, 256 CTAs) and 8192 rows at G = 32 (16 splits, 256 CTAs)
+    assert f(8, 64, 1, 131072, 128) == _decode_ws(32, 8, 64)
+    assert f(8, 64, 2, 131072, 128) == _decode_ws(16, 8, 64)
+    # Qwen3-8B decode batch (G = 4): mma.sync kernel, splits of 4096 rows at Lmax 32768
+    assert f(64, 32, 8, 32768, 128) == _decode_ws(8, 64, 32)
+
+
 def test_missing_library_raises(monkeypatch, tmp_path):
     monkeypatch.setattr(_native, "_lib", None)
     monkeypatch.setattr(_native, "LIB_PATH", str(tmp_path / "absent.so"))
