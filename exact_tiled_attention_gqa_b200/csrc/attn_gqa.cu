@@ -365,19 +365,16 @@ int launch_prefill(const void* q, const void* k, const void* v, void* out, float
 //    256 CTAs) took 0.163-0.164 ms against 0.165-0.166 for 7296 (288 CTAs) and
 //    0.178 for 10240.
 //  - tcgen05 kernel, D = 256 (one CTA per SM): the largest power of two in
-//    [512, 4096] that still gives about four waves of CTAs at Lmax (592).  With
-//    lengths spread over [1024, 32768] the split count at Lmax says little about
-//    the real waves, so the target is several: on the head-dim-256 decode batch
-//    (B 32, Hkv 2, Lmax 32768) 2048-row splits took 0.154-0.155 ms against 0.171
-//    for 4096 (the earlier one-wave target) and 0.159 for 8192.  (The balanced
-//    rule above, at one CTA per SM, made that batch 8 % slower.)
+//    [512, 4096] that still gives 148 CTAs (the balanced rule above, at one CTA
+//    per SM, made the head-dim-256 decode batch 8 % slower: with lengths spread
+//    over [1024, 32768] the split count at Lmax says little about real waves).
 // The result depends only on the arguments (workspace sizes do too).
 bool decode_uses_tc(int D, int rows_per_group) { return D == 256 || rows_per_group > 16; }
 
 int decode_chunk(int B, int Hkv, int Lmax, bool tc_path, int D) {
     const long long groups = static_cast<long long>(B) * Hkv;
     if (!tc_path || D == 256) {
-        const long long target = tc_path ? 148LL * 4 : 148LL * 2 * 4;
+        const long long target = tc_path ? 148LL : 148LL * 2 * 4;
         const int min_chunk = tc_path ? 512 : 256;
         int chunk = 4096;
         while (chunk > min_chunk && groups * ((Lmax + chunk - 1) / chunk) < target) chunk >>= 1;
